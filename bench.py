@@ -1,0 +1,515 @@
+"""Throughput of the DoRA hot path on B200, as a fraction of roofline.
+
+One step = one pass of the whole path over one batch of synthetic input on the
+headline module (d_out = d_in = 8192, r = 384, alpha = 768, bf16) with
+[4096, 8192] activations:
+    factored norm (Gram, fused norm GEMM, finalize with g = m / max(n, eps))
+    -> compose forward -> compose backward (d_base, d_lora, dm).
+
+Metric: "norm TFLOP/s + compose GB/s (% of B200 roofline)".  `value` is the
+roofline time of the step's work (norm: the slower of its 2 d_out d_in r
+FLOPs at the measured bf16 tensor peak and its W0 + A + B bytes at the
+measured HBM bandwidth; compose forward / backward: 3 / 5 activation passes at
+HBM bandwidth) divided by the measured step time, in percent, summed over
+ranks (each rank runs its own module and batch: weak scaling, no collective on
+the data path).  The per-part TFLOP/s and GB/s are reported under
+"components".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = "headline_8192_r384"
+METRIC = "norm TFLOP/s + compose GB/s (% of B200 roofline), d=8192 r=384 bf16"
+UNIT = "% of B200 roofline"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# --------------------------------------------------------------------------- peaks
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def work_model(d_out, d_in, r, T):
+    """Algorithmic work of one step."""
+    norm_flops = 2.0 * d_out * d_in * r
+    norm_bytes = 2.0 * (d_out * d_in + r * d_in + d_out * r)
+    act = 2.0 * T * d_out
+    return {"norm_flops": norm_flops, "norm_bytes": norm_bytes,
+            "fwd_bytes": 3 * act, "bwd_bytes": 5 * act}
+
+
+def roofline_times(wm, peaks):
+    t_norm = max(wm["norm_flops"] / (peaks["bf16_tflops"] * 1e12),
+                 wm["norm_bytes"] / (peaks["hbm_gbs"] * 1e9))
+    t_fwd = wm["fwd_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_bwd = wm["bwd_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    return t_norm, t_fwd, t_bwd
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        import tempfile
+        self.path = os.path.join(tempfile.gettempdir(), f"dora_bench_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(1.0)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        if not sm:
+            return None
+        loaded = [x for x in sm if mx is None or x > 0.3 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- distributed
+
+def dist_setup(n_gpus: int):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        import torch
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+    return rank, world, local, pg
+
+
+def barrier(pg, local):
+    if pg is not None:
+        import torch
+        pg.barrier(device_ids=[local])
+
+
+def max_over_ranks(pg, x: float) -> float:
+    if pg is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- oracle arm
+
+def oracle_step_seconds(W0, A, B, m, base, lora, dy, s, eps, rows, tokens, T_full=4096):
+    """Times the fp64 oracle on a sample (`rows` rows of the norm, `tokens` rows
+    of the compose) and scales it to the full step."""
+    import numpy as np
+    import oracle
+    d_out = W0.shape[0]
+    T = T_full
+    Wr = W0[:rows].astype(np.float64)
+    Br = B[:rows].astype(np.float64)
+    Af = A.astype(np.float64)
+    t0 = time.perf_counter()
+    n_rows = oracle.rows_dense_row_norm(Wr, Af, Br, s)
+    oracle.magnitude_scale(m[:rows], n_rows, eps)
+    t1 = time.perf_counter()
+    n_full = np.full(d_out, float(np.mean(n_rows)))
+    b = base[:tokens].astype(np.float64)
+    l = lora[:tokens].astype(np.float64)
+    d = dy[:tokens].astype(np.float64)
+    oracle.compose_fwd(b, l, m, n_full, s, eps)
+    oracle.compose_bwd(d, b, l, m, n_full, s, eps)
+    t2 = time.perf_counter()
+    return (t1 - t0) * d_out / rows + (t2 - t1) * T / tokens
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max([int(i.get("num_threads", 1)) for i in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def host_sample_inputs(seed=7):
+    """The headline workload's inputs on the host, drawn with the same recipe
+    (bf16-rounded values) as the GPU run."""
+    import numpy as np
+    import torch
+    from dora_adapter_factored_b200 import synth
+    w = synth.WORKLOADS[WORKLOAD]
+    W0, A, B = synth.module_weights(w)
+    m = synth.magnitude_from_base_rows(w, W0).double().numpy()
+    base, lora, dy = synth.activations(w, 256, W0.shape[0])
+    f = lambda t: t.float().numpy()
+    return f(W0), f(A), f(B), m, f(base), f(lora), f(dy), w.modules[0].s, synth.eps_for("bf16")
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+    from dora_adapter_factored_b200 import synth
+    w = synth.WORKLOADS[WORKLOAD]
+    ms = w.modules[0]
+    peaks = load_peaks()
+    wm = work_model(ms.d_out, ms.d_in, ms.r, w.tokens)
+    t_roof = sum(roofline_times(wm, peaks))
+    W0, A, B, m, base, lora, dy, s, eps = host_sample_inputs()
+    rows, tokens = 16, 8
+    for _ in range(args.warmup):
+        oracle_step_seconds(W0, A, B, m, base, lora, dy, s, eps, rows, tokens)
+    ts = [oracle_step_seconds(W0, A, B, m, base, lora, dy, s, eps, rows, tokens)
+          for _ in range(args.steps)]
+    t = statistics.mean(ts)
+    value = 100.0 * t_roof / t
+    sample = (f"per step: fp64 dense norm of {rows} of {ms.d_out} rows and compose fwd+bwd on "
+              f"{tokens} of {w.tokens} tokens, scaled to the full step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_dict(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w):
+    ms = w.modules[0]
+    return {"workload": w.key, "d_out": ms.d_out, "d_in": ms.d_in, "r": ms.r, "alpha": ms.alpha,
+            "tokens": w.tokens, "storage": "bf16",
+            "step": "gram + fused norm GEMM + finalize(g) + compose fwd + compose bwd(dm)",
+            "l2": "inputs larger than L2 (W0 134 MB, activations 3 x 64 MB) and 2 rotating input sets"}
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args):
+    import torch
+    import dora_adapter_factored_b200 as dora
+    from dora_adapter_factored_b200 import synth
+
+    rank, world, local, pg = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = synth.WORKLOADS[WORKLOAD]
+    ms = w.modules[0]
+    d_out, d_in, r, T, s = ms.d_out, ms.d_in, ms.r, w.tokens, ms.s
+    eps = synth.eps_for("bf16")
+    peaks = load_peaks()
+    wm = work_model(d_out, d_in, r, T)
+    t_roof_norm, t_roof_fwd, t_roof_bwd = roofline_times(wm, peaks)
+    t_roof = t_roof_norm + t_roof_fwd + t_roof_bwd
+    stream = torch.cuda.current_stream()
+
+    # Two independent input sets (weights + activations), rotated every step.
+    sets = []
+    for k in range(2):
+        W0, A, B = synth.module_weights(w, device=dev)
+        base, lora, dy = synth.activations(w, T, d_out, device=dev, index=k)
+        n_tmp, _ = dora.dora_factored_norm(W0, A, B, s)
+        m = synth.magnitude_near_unity(w, n_tmp, index=k)  # |g - 1| < 1e-2, as the workload asks
+        if k == 1:  # a distinct module for the second set
+            W0 = W0.flip(0).contiguous()
+            B = B.flip(0).contiguous()
+            m = m.flip(0).contiguous()
+        sets.append(dict(W0=W0, A=A, B=B, m=m, base=base, lora=lora, dy=dy))
+    outs = dict(n=torch.empty(d_out, device=dev), g=torch.empty(d_out, device=dev),
+                y=torch.empty(T, d_out, dtype=torch.bfloat16, device=dev),
+                d_base=torch.empty(T, d_out, dtype=torch.bfloat16, device=dev),
+                d_lora=torch.empty(T, d_out, dtype=torch.bfloat16, device=dev),
+                dm=torch.empty(d_out, device=dev))
+    ws_norm = torch.empty(dora.dora_factored_norm_workspace_size(d_out, d_in, r, torch.bfloat16),
+                          dtype=torch.uint8, device=dev)
+    ws_bwd = torch.empty(max(256, dora.dora_compose_bwd_workspace_size(T, d_out, torch.bfloat16)),
+                         dtype=torch.uint8, device=dev)
+
+    def step(i, ev=None):
+        S_ = sets[i % 2]
+        if ev is not None:
+            ev["s0"].record(stream)
+            dora.dora_set_timing_events(ev["nk0"], ev["nk1"])
+        dora.dora_factored_norm(S_["W0"], S_["A"], S_["B"], s, S_["m"], eps, n_out=outs["n"],
+                                g_out=outs["g"], ws=ws_norm)
+        if ev is not None:
+            ev["s1"].record(stream)
+            dora.dora_set_timing_events(ev["fk0"], ev["fk1"])
+        dora.dora_compose_fwd(S_["base"], S_["lora"], S_["m"], outs["n"], s, eps, y=outs["y"])
+        if ev is not None:
+            ev["s2"].record(stream)
+            dora.dora_set_timing_events(ev["bk0"], ev["bk1"])
+        dora.dora_compose_bwd(S_["dy"], S_["base"], S_["lora"], S_["m"], outs["n"], s, eps,
+                              d_base=outs["d_base"], d_lora=outs["d_lora"], dm=outs["dm"],
+                              ws=ws_bwd)
+        if ev is not None:
+            ev["s3"].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if dora.dora_get_device_status() != 0:
+        raise RuntimeError("a kernel reported an error during warm-up")
+
+    names = ("s0", "s1", "s2", "s3", "nk0", "nk1", "fk0", "fk1", "bk0", "bk1")
+    evs = []
+    for _ in range(args.steps):
+        e = {k: torch.cuda.Event(enable_timing=True) for k in names}
+        for x in e.values():  # create the underlying CUDA events
+            x.record(stream)
+        evs.append(e)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    launches0 = dora.dora_launch_count()
+    barrier(pg, local)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(i, evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(pg, local)
+    launches = dora.dora_launch_count() - launches0
+    clk = clocks.stop()
+    if dora.dora_get_device_status() != 0:
+        raise RuntimeError("a kernel reported an error in the timed region")
+
+    total_ms = t_start.elapsed_time(t_end)
+    total_ms = max_over_ranks(pg, total_ms)
+    ms_step = total_ms / args.steps
+    avg = lambda a, b: statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
+    t_norm_call = avg("s0", "s1") * 1e-3
+    t_norm_k = avg("nk0", "nk1") * 1e-3
+    t_fwd_k = avg("fk0", "fk1") * 1e-3
+    t_bwd_call = avg("s2", "s3") * 1e-3
+    t_bwd_k = avg("bk0", "bk1") * 1e-3
+    t_fwd_call = avg("s1", "s2") * 1e-3
+    value = world * 100.0 * t_roof / (ms_step * 1e-3)
+
+    tc_peak, hbm_peak = peaks["bf16_tflops"], peaks["hbm_gbs"]
+    kernels = {
+        "norm_main_kernel": {"us": t_norm_k * 1e6, "bound": "tensor",
+                             "achieved": wm["norm_flops"] / t_norm_k / 1e12, "peak": tc_peak,
+                             "unit": "TFLOP/s"},
+        "compose_fwd_kernel": {"us": t_fwd_k * 1e6, "bound": "hbm",
+                               "achieved": wm["fwd_bytes"] / t_fwd_k / 1e9, "peak": hbm_peak,
+                               "unit": "GB/s"},
+        "compose_bwd_kernel": {"us": t_bwd_k * 1e6, "bound": "hbm",
+                               "achieved": wm["bwd_bytes"] / t_bwd_k / 1e9, "peak": hbm_peak,
+                               "unit": "GB/s"},
+    }
+    for k in kernels.values():
+        k["frac"] = k["achieved"] / k["peak"]
+    dominant = max(kernels, key=lambda k: kernels[k]["us"])
+    dk = kernels[dominant]
+    traffic = load_traffic(dominant)
+    components = {
+        "norm_tflops": wm["norm_flops"] / t_norm_call / 1e12,
+        "norm_frac_of_roofline": t_roof_norm / t_norm_call,
+        "norm_us": t_norm_call * 1e6,
+        "compose_fwd_gbs": wm["fwd_bytes"] / t_fwd_call / 1e9,
+        "compose_fwd_frac_of_hbm": wm["fwd_bytes"] / t_fwd_call / 1e9 / hbm_peak,
+        "compose_fwd_us": t_fwd_call * 1e6,
+        "compose_bwd_gbs": wm["bwd_bytes"] / t_bwd_call / 1e9,
+        "compose_bwd_frac_of_hbm": wm["bwd_bytes"] / t_bwd_call / 1e9 / hbm_peak,
+        "compose_bwd_us": t_bwd_call * 1e6,
+        "roofline_us": {"norm": t_roof_norm * 1e6, "compose_fwd": t_roof_fwd * 1e6,
+                        "compose_bwd": t_roof_bwd * 1e6},
+        "peaks": f"{peaks['source']}: HBM {hbm_peak} GB/s, bf16 {tc_peak} TFLOP/s (burst)",
+    }
+
+    e2e = measure_e2e(args, dora, w, sets[0], s, eps, t_roof, dev, stream, pg, local, world)
+
+    cpu = None
+    if rank == 0 and world == 1:
+        cpu = measure_cpu_baseline(t_roof)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; bf16 weights and activations, no checkpoint)",
+            "config": config_dict(w),
+            "roofline": {"kernel": dominant, "bound": dk["bound"], "achieved": dk["achieved"],
+                         "peak": dk["peak"], "unit": dk["unit"], "frac": dk["frac"],
+                         "traffic": traffic, "peak_source": peaks["source"]},
+            "kernels": kernels,
+            "components": components,
+            "clocks": clk,
+            "gpu_launches": int(launches),
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+    return 0
+
+
+def load_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary, if one
+    exists for the current kernel build (profiles/traffic.json)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        return t.get(WORKLOAD, {}).get(kernel)
+    except Exception:
+        return None
+
+
+def measure_e2e(args, dora, w, S_, s, eps, t_roof, dev, stream, pg, local, world):
+    """The same step through the public API with host (pinned) buffers: every
+    step copies its inputs host->device and reads its results back."""
+    import torch
+    host = {k: S_[k].cpu().pin_memory() for k in ("W0", "A", "B", "m", "base", "lora", "dy")}
+    dev_in = {k: torch.empty_like(S_[k]) for k in host}
+    T, d_out = S_["base"].shape
+    outs_dev = dict(n=torch.empty(d_out, device=dev), g=torch.empty(d_out, device=dev),
+                    y=torch.empty(T, d_out, dtype=torch.bfloat16, device=dev),
+                    d_base=torch.empty(T, d_out, dtype=torch.bfloat16, device=dev),
+                    d_lora=torch.empty(T, d_out, dtype=torch.bfloat16, device=dev),
+                    dm=torch.empty(d_out, device=dev))
+    outs_host = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in outs_dev.items()}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs_host.values())
+
+    def e2e_step():
+        for k in host:
+            dev_in[k].copy_(host[k], non_blocking=True)
+        dora.dora_factored_norm(dev_in["W0"], dev_in["A"], dev_in["B"], s, dev_in["m"], eps,
+                                n_out=outs_dev["n"], g_out=outs_dev["g"])
+        dora.dora_compose_fwd(dev_in["base"], dev_in["lora"], dev_in["m"], outs_dev["n"], s, eps,
+                              y=outs_dev["y"])
+        dora.dora_compose_bwd(dev_in["dy"], dev_in["base"], dev_in["lora"], dev_in["m"],
+                              outs_dev["n"], s, eps, d_base=outs_dev["d_base"],
+                              d_lora=outs_dev["d_lora"], dm=outs_dev["dm"])
+        for k in outs_dev:
+            outs_host[k].copy_(outs_dev[k], non_blocking=True)
+
+    steps = max(3, min(20, args.steps))
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(pg, local)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(pg, local)
+    ms = max_over_ranks(pg, a.elapsed_time(b)) / steps
+    return {"value": world * 100.0 * t_roof / (ms * 1e-3), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": ms, "steps": steps}
+
+
+def measure_cpu_baseline(t_roof):
+    """The oracle as it stands on the host cores, on a bounded sample of the
+    same workload (about 10 s of CPU work), scaled to one full step."""
+    W0, A, B, m, base, lora, dy, s, eps = host_sample_inputs()
+    rows, tokens = 512, 64
+    oracle_step_seconds(W0, A, B, m, base, lora, dy, s, eps, 16, 4)  # warm
+    ts = []
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < 10.0 and len(ts) < 200:
+        ts.append(oracle_step_seconds(W0, A, B, m, base, lora, dy, s, eps, rows, tokens))
+    t = statistics.mean(ts)
+    return {"value": 100.0 * t_roof / t, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"{len(ts)} repeats of: fp64 dense norm of {rows} of 8192 rows and "
+                       f"compose fwd+bwd on {tokens} of 4096 tokens, scaled to one full step "
+                       f"({t:.2f} s per full step)")}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

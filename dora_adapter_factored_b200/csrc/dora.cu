@@ -1,0 +1,687 @@
+// C ABI of the DoRA hot path (declared in include/dora.h).  Host code only:
+// argument validation, tensor-map encoding, workspace carving and launches.
+// The kernels live in the .cuh files included below (one translation unit).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "dora.h"
+#include "common.cuh"
+#include "compose.cuh"
+#include "norm_simt.cuh"
+#include "norm_tc.cuh"
+
+namespace dora {
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
+constexpr int kMaxDevices = 64;
+
+std::atomic<uint64_t> g_launches{0};
+std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
+
+// One-shot timing events around the principal kernel of the next call.
+thread_local cudaEvent_t t_ev_before = nullptr;
+thread_local cudaEvent_t t_ev_after = nullptr;
+
+struct TimedLaunch {
+  cudaStream_t st;
+  explicit TimedLaunch(cudaStream_t s) : st(s) {
+    if (t_ev_before != nullptr) cudaEventRecord(t_ev_before, st);
+  }
+  ~TimedLaunch() {
+    if (t_ev_after != nullptr) cudaEventRecord(t_ev_after, st);
+    t_ev_before = t_ev_after = nullptr;
+  }
+};
+
+struct DeviceInfo {
+  bool init = false;
+  bool supported = false;
+  int sms = 0;
+  bool attrs_set = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Current device's info; nullptr if the device cannot be queried.
+const DeviceInfo* device_info() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return nullptr;
+    d.supported = (major == 10);
+    d.sms = sms;
+    d.init = true;
+  }
+  return &d;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+dora_status_t launch_status() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? DORA_OK : DORA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ tensor maps
+
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Row-major bf16 matrix [rows, cols] with `ld` elements per row, loaded in
+// boxes of box_cols x box_rows with 128-byte swizzle; out-of-range elements
+// read as zero.
+bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint64_t ld,
+                    uint32_t box_cols, uint32_t box_rows) {
+  auto enc = tmap_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------ norm planning
+
+struct ModulePlan {
+  // N side
+  int n_pad, n0, n1, box_rows, nbox, tmem_cols;
+  uint32_t b_region;
+  // K / tiles
+  int kb_w, kb_r, kb_tile, tiles;
+  long long units;
+  // Gram
+  int r8, tiles_r, pairs, kb_gram, S;
+  // workspace (relative offsets inside the module's region)
+  size_t off_g, off_gp, off_np, bytes;
+  int seg_slots;
+};
+
+void plan_n_side(int r, ModulePlan& p) {
+  p.n_pad = round_up_int(r, 16);
+  if (p.n_pad <= 256) {
+    p.n0 = p.n_pad;
+    p.n1 = 0;
+    p.nbox = 1;
+  } else {
+    p.n0 = round_up_int((p.n_pad + 1) / 2, 16);
+    p.n1 = p.n_pad - p.n0;
+    p.nbox = 2;
+  }
+  p.box_rows = p.n0;
+  p.b_region = static_cast<uint32_t>(p.nbox * p.box_rows * 128);
+  int tc = 32;
+  while (tc < p.n_pad) tc <<= 1;
+  p.tmem_cols = tc;
+}
+
+void plan_module(int64_t d_out, int64_t d_in, int64_t r, ModulePlan& p) {
+  plan_n_side(static_cast<int>(r), p);
+  p.kb_w = static_cast<int>(ceil_div_ll(d_in, kBlockK));
+  p.kb_r = static_cast<int>(ceil_div_ll(r, kBlockK));
+  p.kb_tile = p.kb_w + p.kb_r;
+  p.tiles = static_cast<int>(ceil_div_ll(d_out, kTileM));
+  p.units = static_cast<long long>(p.tiles) * p.kb_tile;
+  p.r8 = round_up_int(static_cast<int>(r), 8);
+  p.tiles_r = static_cast<int>(ceil_div_ll(r, kTileM));
+  p.pairs = p.tiles_r * (p.tiles_r + 1) / 2;
+  p.kb_gram = p.kb_w;
+  const int by_k = std::max(1, p.kb_gram / 8);
+  const int by_sm = std::max(1, 148 / p.pairs);
+  p.S = std::max(1, std::min(by_k, by_sm));
+}
+
+// Largest number of stream-K segments on any tile of any module.
+int max_seg_slots(const std::vector<ModulePlan>& plans, long long total_units, int C) {
+  int best = 1;
+  long long begin = 0;
+  for (const auto& p : plans) {
+    for (int t = 0; t < p.tiles; ++t) {
+      const long long x0 = begin + static_cast<long long>(t) * p.kb_tile;
+      const int c0 = first_cta_of_unit(x0, total_units, C);
+      const int c1 = first_cta_of_unit(x0 + p.kb_tile - 1, total_units, C);
+      best = std::max(best, c1 - c0 + 1);
+    }
+    begin += p.units;
+  }
+  return best;
+}
+
+struct GroupLayout {
+  std::vector<ModulePlan> plans;
+  long long total_units = 0;
+  int ctas = 0;
+  int seg_slots = 1;
+  uint32_t b_region = 0;
+  int tmem_cols = 32;
+  int stages = 0;
+  size_t smem_bytes = 0;
+  int gram_jobs = 0;
+  int max_pairs = 0;
+  int max_d_out = 0;
+  size_t table_bytes = 0;  // descriptor tables at the start of the workspace (grouped)
+  size_t total_bytes = 0;
+};
+
+bool layout_group(const int64_t* d_out, const int64_t* d_in, const int64_t* r, int count,
+                  bool grouped, int sms, GroupLayout& L) {
+  L.plans.resize(count);
+  L.total_units = 0;
+  for (int i = 0; i < count; ++i) {
+    plan_module(d_out[i], d_in[i], r[i], L.plans[i]);
+    L.total_units += L.plans[i].units;
+    L.b_region = std::max(L.b_region, L.plans[i].b_region);
+    L.tmem_cols = std::max(L.tmem_cols, L.plans[i].tmem_cols);
+    L.gram_jobs += L.plans[i].pairs * L.plans[i].S;
+    L.max_pairs = std::max(L.max_pairs, L.plans[i].pairs);
+    L.max_d_out = std::max(L.max_d_out, static_cast<int>(d_out[i]));
+  }
+  L.ctas = static_cast<int>(std::min<long long>(sms, L.total_units));
+  if (L.ctas < 1) return false;
+  L.seg_slots = max_seg_slots(L.plans, L.total_units, L.ctas);
+  const uint32_t stage_bytes = kTileABytes + L.b_region;
+  L.stages = std::min<int>(kMaxStages, (kMaxDynSmem - 1024 - 256) / stage_bytes);
+  if (L.stages < 2) return false;
+  L.smem_bytes = 1024 + static_cast<size_t>(L.stages) * stage_bytes + 256;
+  size_t off = 0;
+  if (grouped) {
+    off = align_up(sizeof(NormProblemDev) * count, 256) + align_up(sizeof(GramProblemDev) * count, 256);
+  }
+  L.table_bytes = off;
+  for (auto& p : L.plans) {
+    p.seg_slots = L.seg_slots;
+    p.off_g = off;
+    off += align_up(static_cast<size_t>(p.n_pad) * p.r8 * 2 + 0, 256);
+    p.off_gp = off;
+    off += align_up(static_cast<size_t>(p.pairs) * p.S * kTileM * kTileM * 4, 256);
+    p.off_np = off;
+    off += align_up(static_cast<size_t>(p.tiles) * L.seg_slots * kTileM * 4, 256);
+  }
+  L.total_bytes = off;
+  return true;
+}
+
+bool ensure_tc_attrs(int smem_norm) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (d.attrs_set) return true;
+  (void)smem_norm;
+  const int gram_smem = 1024 + kGramStages * kGramStageBytes + 256;
+  bool ok = true;
+  ok &= cudaFuncSetAttribute(norm_main_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kMaxDynSmem) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(norm_main_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kMaxDynSmem) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(gram_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gram_smem) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(gram_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gram_smem) == cudaSuccess;
+  d.attrs_set = ok;
+  return ok;
+}
+
+// Fills the device descriptors of one module.
+bool fill_descriptors(const dora_norm_problem_t& pr, const ModulePlan& p, uint8_t* ws_base,
+                      long long unit_begin, int gram_job_begin, NormProblemDev& nd,
+                      GramProblemDev& gd) {
+  std::memset(&nd, 0, sizeof(nd));
+  std::memset(&gd, 0, sizeof(gd));
+  uint16_t* gprime = reinterpret_cast<uint16_t*>(ws_base + p.off_g);
+  bool ok = true;
+  ok &= make_tmap_bf16(&nd.tm_w0, pr.W0, pr.d_out, pr.d_in, pr.d_in, kBlockK, kTileM);
+  ok &= make_tmap_bf16(&nd.tm_a, pr.A, pr.r, pr.d_in, pr.d_in, kBlockK, p.box_rows);
+  ok &= make_tmap_bf16(&nd.tm_b, pr.B, pr.d_out, pr.r, pr.r, kBlockK, kTileM);
+  ok &= make_tmap_bf16(&nd.tm_g, gprime, pr.r, pr.r, p.r8, kBlockK, p.box_rows);
+  ok &= make_tmap_bf16(&gd.tm_a, pr.A, pr.r, pr.d_in, pr.d_in, kBlockK, kTileM);
+  nd.B = static_cast<const uint16_t*>(pr.B);
+  nd.partial = reinterpret_cast<float*>(ws_base + p.off_np);
+  nd.m = pr.m;
+  nd.n_out = pr.n_out;
+  nd.g_out = pr.g_out;
+  nd.unit_begin = unit_begin;
+  nd.d_out = static_cast<int>(pr.d_out);
+  nd.r = static_cast<int>(pr.r);
+  nd.n0 = p.n0;
+  nd.n1 = p.n1;
+  nd.box_rows = p.box_rows;
+  nd.nbox = p.nbox;
+  nd.kb_w = p.kb_w;
+  nd.kb_r = p.kb_r;
+  nd.kb_tile = p.kb_tile;
+  nd.tiles = p.tiles;
+  nd.seg_slots = p.seg_slots;
+  nd.stage_tx = kTileABytes + p.b_region;
+  nd.idesc0 = idesc_bf16_f32(kTileM, p.n0);
+  nd.idesc1 = p.n1 > 0 ? idesc_bf16_f32(kTileM, p.n1) : 0u;
+  nd.two_s = 2.0f * pr.s;
+
+  gd.partial = reinterpret_cast<float*>(ws_base + p.off_gp);
+  gd.g_out = gprime;
+  gd.r = static_cast<int>(pr.r);
+  gd.r8 = p.r8;
+  gd.kb = p.kb_gram;
+  gd.tiles_r = p.tiles_r;
+  gd.pairs = p.pairs;
+  gd.S = p.S;
+  gd.job_begin = gram_job_begin;
+  gd.half_s = 0.5f * pr.s;
+  return ok;
+}
+
+bool tc_eligible(const dora_norm_problem_t& p) {
+  return p.d_in % 8 == 0 && p.r % 8 == 0 && aligned16(p.W0) && aligned16(p.A) && aligned16(p.B);
+}
+
+dora_status_t check_problem(const dora_norm_problem_t& p) {
+  if (p.W0 == nullptr || p.A == nullptr || p.B == nullptr || p.n_out == nullptr)
+    return DORA_ERR_INVALID_ARG;
+  if (p.d_out < 1 || p.d_in < 1 || p.r < 1) return DORA_ERR_INVALID_ARG;
+  if (p.d_out > (1ll << 31) - 1 || p.d_in > (1ll << 31) - 1) return DORA_ERR_UNSUPPORTED;
+  if (p.r > DORA_MAX_RANK) return DORA_ERR_UNSUPPORTED;
+  if ((p.m == nullptr) != (p.g_out == nullptr)) return DORA_ERR_INVALID_ARG;
+  const size_t nb = static_cast<size_t>(p.d_out) * 4;
+  if (p.g_out != nullptr && overlaps(p.n_out, nb, p.g_out, nb)) return DORA_ERR_INVALID_ARG;
+  return DORA_OK;
+}
+
+dora_status_t run_tc_group(const dora_norm_problem_t* probs, int count, bool grouped, float eps,
+                           void* ws, size_t ws_bytes, cudaStream_t st) {
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return DORA_ERR_CUDA;
+  if (!di->supported) return DORA_ERR_UNSUPPORTED;
+  std::vector<int64_t> d_out(count), d_in(count), r(count);
+  for (int i = 0; i < count; ++i) {
+    d_out[i] = probs[i].d_out;
+    d_in[i] = probs[i].d_in;
+    r[i] = probs[i].r;
+  }
+  GroupLayout L;
+  if (!layout_group(d_out.data(), d_in.data(), r.data(), count, grouped, di->sms, L))
+    return DORA_ERR_UNSUPPORTED;
+  if (ws == nullptr || ws_bytes < L.total_bytes || !aligned256(ws)) return DORA_ERR_WORKSPACE;
+  if (!ensure_tc_attrs(static_cast<int>(L.smem_bytes))) return DORA_ERR_CUDA;
+
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  std::vector<NormProblemDev> nds(count);
+  std::vector<GramProblemDev> gds(count);
+  long long ub = 0;
+  int jb = 0;
+  for (int i = 0; i < count; ++i) {
+    if (!fill_descriptors(probs[i], L.plans[i], base, ub, jb, nds[i], gds[i]))
+      return DORA_ERR_INVALID_ARG;
+    ub += L.plans[i].units;
+    jb += L.plans[i].pairs * L.plans[i].S;
+  }
+  const unsigned long long tmo = g_timeout_ns.load();
+  const int gram_smem = 1024 + kGramStages * kGramStageBytes + 256;
+  dora_status_t s;
+  if (!grouped) {
+    gram_kernel<false><<<L.gram_jobs, kTcThreads, gram_smem, st>>>(gds[0], nullptr, 1, tmo);
+    if ((s = launch_status()) != DORA_OK) return s;
+    gram_reduce_kernel<false><<<dim3(kTileM * kTileM / 256, L.max_pairs, 1), 256, 0, st>>>(
+        gds[0], nullptr);
+    if ((s = launch_status()) != DORA_OK) return s;
+    {
+      TimedLaunch tl(st);
+      norm_main_kernel<false><<<L.ctas, kTcThreads, L.smem_bytes, st>>>(
+          nds[0], nullptr, 1, L.total_units, L.stages, L.b_region, L.tmem_cols, tmo);
+      if ((s = launch_status()) != DORA_OK) return s;
+    }
+    norm_finalize_kernel<false>
+        <<<dim3(static_cast<unsigned>(ceil_div_ll(L.max_d_out, 256)), 1), 256, 0, st>>>(
+            nds[0], nullptr, L.total_units, L.ctas, eps);
+    return launch_status();
+  }
+  NormProblemDev* ntab = reinterpret_cast<NormProblemDev*>(base);
+  GramProblemDev* gtab =
+      reinterpret_cast<GramProblemDev*>(base + align_up(sizeof(NormProblemDev) * count, 256));
+  if (cudaMemcpyAsync(ntab, nds.data(), sizeof(NormProblemDev) * count, cudaMemcpyHostToDevice,
+                      st) != cudaSuccess ||
+      cudaMemcpyAsync(gtab, gds.data(), sizeof(GramProblemDev) * count, cudaMemcpyHostToDevice,
+                      st) != cudaSuccess)
+    return DORA_ERR_CUDA;
+  gram_kernel<true><<<L.gram_jobs, kTcThreads, gram_smem, st>>>(gds[0], gtab, count, tmo);
+  if ((s = launch_status()) != DORA_OK) return s;
+  gram_reduce_kernel<true><<<dim3(kTileM * kTileM / 256, L.max_pairs, count), 256, 0, st>>>(
+      gds[0], gtab);
+  if ((s = launch_status()) != DORA_OK) return s;
+  {
+    TimedLaunch tl(st);
+    norm_main_kernel<true><<<L.ctas, kTcThreads, L.smem_bytes, st>>>(
+        nds[0], ntab, count, L.total_units, L.stages, L.b_region, L.tmem_cols, tmo);
+    if ((s = launch_status()) != DORA_OK) return s;
+  }
+  norm_finalize_kernel<true>
+      <<<dim3(static_cast<unsigned>(ceil_div_ll(L.max_d_out, 256)), count), 256, 0, st>>>(
+          nds[0], ntab, L.total_units, L.ctas, eps);
+  return launch_status();
+}
+
+// One thread waits on a barrier that nothing arrives on; the bounded wait
+// gives up and records DORA_ERR_TIMEOUT.
+__global__ void unsignalled_wait_kernel(unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  if (!mbar_wait(&bar, 0, timeout_ns, nullptr)) record_error(DORA_ERR_TIMEOUT);
+}
+
+size_t simt_workspace(int64_t r) { return align_up(static_cast<size_t>(r) * r * 4, 256); }
+
+}  // namespace
+}  // namespace dora
+
+using namespace dora;
+
+extern "C" {
+
+size_t dora_factored_norm_workspace_size(int64_t d_out, int64_t d_in, int64_t r,
+                                         dora_dtype_t dt) {
+  if (d_out < 1 || d_in < 1 || r < 1 || r > DORA_MAX_RANK) return 0;
+  if (dt == DORA_F32 || d_in % 8 != 0 || r % 8 != 0) return simt_workspace(r);
+  const DeviceInfo* di = device_info();
+  const int sms = (di != nullptr && di->sms > 0) ? di->sms : 148;
+  GroupLayout L;
+  if (!layout_group(&d_out, &d_in, &r, 1, false, sms, L)) return 0;
+  return std::max(L.total_bytes, simt_workspace(r));
+}
+
+dora_status_t dora_factored_norm(const void* W0, const void* A, const void* B, dora_dtype_t dt,
+                                 int64_t d_out, int64_t d_in, int64_t r, float s, const float* m,
+                                 float eps, float* n_out, float* g_out, void* ws, size_t ws_bytes,
+                                 dora_stream_t stream) {
+  if (dt != DORA_F32 && dt != DORA_BF16) return DORA_ERR_INVALID_ARG;
+  dora_norm_problem_t p{W0, A, B, m, n_out, g_out, d_out, d_in, r, s};
+  dora_status_t st = check_problem(p);
+  if (st != DORA_OK) return st;
+  if (!(eps >= 0.f)) return DORA_ERR_INVALID_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (dt == DORA_BF16 && tc_eligible(p)) return run_tc_group(&p, 1, false, eps, ws, ws_bytes, cs);
+
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return DORA_ERR_CUDA;
+  if (!di->supported) return DORA_ERR_UNSUPPORTED;
+  if (ws == nullptr || ws_bytes < simt_workspace(r) || !aligned256(ws)) return DORA_ERR_WORKSPACE;
+  float* G = static_cast<float*>(ws);
+  const long long warps = r * r;
+  const unsigned gblocks = static_cast<unsigned>(ceil_div_ll(warps * 32, 256));
+  if (dt == DORA_F32) {
+    gram_simt_kernel<float><<<gblocks, 256, 0, cs>>>(static_cast<const float*>(A), (int)r,
+                                                     (int)d_in, G);
+    if ((st = launch_status()) != DORA_OK) return st;
+    norm_simt_kernel<float><<<(unsigned)d_out, 256, 0, cs>>>(
+        static_cast<const float*>(W0), static_cast<const float*>(A),
+        static_cast<const float*>(B), G, (int)d_out, (int)d_in, (int)r, s, m, eps, n_out, g_out);
+  } else {
+    gram_simt_kernel<__nv_bfloat16><<<gblocks, 256, 0, cs>>>(
+        static_cast<const __nv_bfloat16*>(A), (int)r, (int)d_in, G);
+    if ((st = launch_status()) != DORA_OK) return st;
+    norm_simt_kernel<__nv_bfloat16><<<(unsigned)d_out, 256, 0, cs>>>(
+        static_cast<const __nv_bfloat16*>(W0), static_cast<const __nv_bfloat16*>(A),
+        static_cast<const __nv_bfloat16*>(B), G, (int)d_out, (int)d_in, (int)r, s, m, eps, n_out,
+        g_out);
+  }
+  return launch_status();
+}
+
+size_t dora_factored_norm_grouped_workspace_size(const dora_norm_problem_t* problems, int count,
+                                                 dora_dtype_t dt) {
+  if (problems == nullptr || count < 1 || count > DORA_MAX_GROUP || dt != DORA_BF16) return 0;
+  std::vector<int64_t> d_out(count), d_in(count), r(count);
+  for (int i = 0; i < count; ++i) {
+    if (problems[i].d_out < 1 || problems[i].d_in < 1 || problems[i].r < 1 ||
+        problems[i].r > DORA_MAX_RANK)
+      return 0;
+    d_out[i] = problems[i].d_out;
+    d_in[i] = problems[i].d_in;
+    r[i] = problems[i].r;
+  }
+  const DeviceInfo* di = device_info();
+  const int sms = (di != nullptr && di->sms > 0) ? di->sms : 148;
+  GroupLayout L;
+  if (!layout_group(d_out.data(), d_in.data(), r.data(), count, true, sms, L)) return 0;
+  return L.total_bytes;
+}
+
+dora_status_t dora_factored_norm_grouped(const dora_norm_problem_t* problems, int count,
+                                         dora_dtype_t dt, float eps, void* ws, size_t ws_bytes,
+                                         dora_stream_t stream) {
+  if (problems == nullptr || count < 1) return DORA_ERR_INVALID_ARG;
+  if (count > DORA_MAX_GROUP) return DORA_ERR_UNSUPPORTED;
+  if (dt != DORA_BF16) return DORA_ERR_UNSUPPORTED;
+  if (!(eps >= 0.f)) return DORA_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    dora_status_t st = check_problem(problems[i]);
+    if (st != DORA_OK) return st;
+    if (!tc_eligible(problems[i])) return DORA_ERR_UNSUPPORTED;
+  }
+  return run_tc_group(problems, count, true, eps, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+dora_status_t dora_compose_fwd(const void* base, const void* lora, const float* m, const float* n,
+                               float s, float eps, dora_dtype_t dt, int64_t T, int64_t d_out,
+                               void* y, dora_stream_t stream) {
+  if (dt != DORA_F32 && dt != DORA_BF16) return DORA_ERR_INVALID_ARG;
+  if (T < 0 || d_out < 1) return DORA_ERR_INVALID_ARG;
+  if (m == nullptr || n == nullptr) return DORA_ERR_INVALID_ARG;
+  if (T > 0 && (base == nullptr || lora == nullptr || y == nullptr)) return DORA_ERR_INVALID_ARG;
+  if (d_out > (1ll << 31) - 1) return DORA_ERR_UNSUPPORTED;
+  if (!(eps >= 0.f)) return DORA_ERR_INVALID_ARG;
+  const size_t es = dt == DORA_BF16 ? 2 : 4;
+  const size_t nbytes = static_cast<size_t>(T) * d_out * es;
+  if (y != base && overlaps(y, nbytes, base, nbytes)) return DORA_ERR_INVALID_ARG;
+  if (overlaps(y, nbytes, lora, nbytes)) return DORA_ERR_INVALID_ARG;
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return DORA_ERR_CUDA;
+  if (!di->supported) return DORA_ERR_UNSUPPORTED;
+  if (T == 0) return DORA_OK;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  TimedLaunch tl(cs);
+  const bool al = aligned16(base) && aligned16(lora) && aligned16(y);
+  if (dt == DORA_BF16) {
+    using B16 = __nv_bfloat16;
+    if (al && d_out % 8 == 0) {
+      const StreamGrid g = stream_grid(T, static_cast<int>(d_out / 8));
+      compose_fwd_kernel<B16, 8><<<dim3(g.gx, g.gy), dim3(g.bx, g.by), 0, cs>>>(
+          static_cast<const B16*>(base), static_cast<const B16*>(lora), m, n, s, eps, T,
+          (int)d_out, static_cast<B16*>(y));
+    } else {
+      const StreamGrid g = stream_grid(T, static_cast<int>(d_out));
+      compose_fwd_kernel<B16, 1><<<dim3(g.gx, g.gy), dim3(g.bx, g.by), 0, cs>>>(
+          static_cast<const B16*>(base), static_cast<const B16*>(lora), m, n, s, eps, T,
+          (int)d_out, static_cast<B16*>(y));
+    }
+  } else {
+    if (al && d_out % 4 == 0) {
+      const StreamGrid g = stream_grid(T, static_cast<int>(d_out / 4));
+      compose_fwd_kernel<float, 4><<<dim3(g.gx, g.gy), dim3(g.bx, g.by), 0, cs>>>(
+          static_cast<const float*>(base), static_cast<const float*>(lora), m, n, s, eps, T,
+          (int)d_out, static_cast<float*>(y));
+    } else {
+      const StreamGrid g = stream_grid(T, static_cast<int>(d_out));
+      compose_fwd_kernel<float, 1><<<dim3(g.gx, g.gy), dim3(g.bx, g.by), 0, cs>>>(
+          static_cast<const float*>(base), static_cast<const float*>(lora), m, n, s, eps, T,
+          (int)d_out, static_cast<float*>(y));
+    }
+  }
+  return launch_status();
+}
+
+namespace {
+struct BwdShape {
+  int vec;
+  StreamGrid g;
+};
+BwdShape bwd_shape(int64_t T, int64_t d_out, dora_dtype_t dt, bool aligned) {
+  BwdShape b;
+  const int v = dt == DORA_BF16 ? 8 : 4;
+  b.vec = (aligned && d_out % v == 0) ? v : 1;
+  b.g = stream_grid(T, static_cast<int>(d_out / b.vec));
+  return b;
+}
+}  // namespace
+
+size_t dora_compose_bwd_workspace_size(int64_t T, int64_t d_out, dora_dtype_t dt) {
+  if (T < 0 || d_out < 1) return 0;
+  // The chunk count does not depend on the vector width chosen at call time:
+  // take the larger of the two layouts.
+  const BwdShape a = bwd_shape(T, d_out, dt, true);
+  const BwdShape b = bwd_shape(T, d_out, dt, false);
+  const int chunks = std::max(a.g.gy, b.g.gy);
+  return align_up(static_cast<size_t>(chunks) * d_out * 4, 256);
+}
+
+dora_status_t dora_compose_bwd(const void* dy, const void* base, const void* lora, const float* m,
+                               const float* n, float s, float eps, dora_dtype_t dt, int64_t T,
+                               int64_t d_out, void* d_base, void* d_lora, float* dm, void* ws,
+                               size_t ws_bytes, dora_stream_t stream) {
+  if (dt != DORA_F32 && dt != DORA_BF16) return DORA_ERR_INVALID_ARG;
+  if (T < 0 || d_out < 1) return DORA_ERR_INVALID_ARG;
+  if (m == nullptr || n == nullptr || dm == nullptr) return DORA_ERR_INVALID_ARG;
+  if (T > 0 && (dy == nullptr || base == nullptr || lora == nullptr || d_base == nullptr ||
+                d_lora == nullptr))
+    return DORA_ERR_INVALID_ARG;
+  if (d_out > (1ll << 31) - 1) return DORA_ERR_UNSUPPORTED;
+  if (!(eps >= 0.f)) return DORA_ERR_INVALID_ARG;
+  const size_t es = dt == DORA_BF16 ? 2 : 4;
+  const size_t nbytes = static_cast<size_t>(T) * d_out * es;
+  const size_t vb = static_cast<size_t>(d_out) * 4;
+  if (d_base != dy && overlaps(d_base, nbytes, dy, nbytes)) return DORA_ERR_INVALID_ARG;
+  if (overlaps(d_base, nbytes, base, nbytes) || overlaps(d_base, nbytes, lora, nbytes) ||
+      overlaps(d_base, nbytes, d_lora, nbytes) || overlaps(d_lora, nbytes, dy, nbytes) ||
+      overlaps(d_lora, nbytes, base, nbytes) || overlaps(d_lora, nbytes, lora, nbytes))
+    return DORA_ERR_INVALID_ARG;
+  if (overlaps(dm, vb, m, vb) || overlaps(dm, vb, n, vb)) return DORA_ERR_INVALID_ARG;
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return DORA_ERR_CUDA;
+  if (!di->supported) return DORA_ERR_UNSUPPORTED;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const bool al = aligned16(dy) && aligned16(base) && aligned16(lora) && aligned16(d_base) &&
+                  aligned16(d_lora);
+  const BwdShape b = bwd_shape(T, d_out, dt, al);
+  const size_t need = static_cast<size_t>(b.g.gy) * d_out * 4;
+  if (ws == nullptr || ws_bytes < need || !aligned256(ws)) return DORA_ERR_WORKSPACE;
+  float* partial = static_cast<float*>(ws);
+  const dim3 grid(b.g.gx, b.g.gy), block(b.g.bx, b.g.by);
+  dora_status_t st;
+  {
+  TimedLaunch tl(cs);
+  if (dt == DORA_BF16) {
+    using B16 = __nv_bfloat16;
+    if (b.vec == 8)
+      compose_bwd_kernel<B16, 8><<<grid, block, 0, cs>>>(
+          static_cast<const B16*>(dy), static_cast<const B16*>(base),
+          static_cast<const B16*>(lora), m, n, s, eps, T, (int)d_out, static_cast<B16*>(d_base),
+          static_cast<B16*>(d_lora), partial);
+    else
+      compose_bwd_kernel<B16, 1><<<grid, block, 0, cs>>>(
+          static_cast<const B16*>(dy), static_cast<const B16*>(base),
+          static_cast<const B16*>(lora), m, n, s, eps, T, (int)d_out, static_cast<B16*>(d_base),
+          static_cast<B16*>(d_lora), partial);
+  } else {
+    if (b.vec == 4)
+      compose_bwd_kernel<float, 4><<<grid, block, 0, cs>>>(
+          static_cast<const float*>(dy), static_cast<const float*>(base),
+          static_cast<const float*>(lora), m, n, s, eps, T, (int)d_out,
+          static_cast<float*>(d_base), static_cast<float*>(d_lora), partial);
+    else
+      compose_bwd_kernel<float, 1><<<grid, block, 0, cs>>>(
+          static_cast<const float*>(dy), static_cast<const float*>(base),
+          static_cast<const float*>(lora), m, n, s, eps, T, (int)d_out,
+          static_cast<float*>(d_base), static_cast<float*>(d_lora), partial);
+  }
+  st = launch_status();
+  }
+  if (st != DORA_OK) return st;
+  colsum_finalize_kernel<<<(unsigned)ceil_div_ll(d_out, 256), 256, 0, cs>>>(partial, b.g.gy,
+                                                                           (int)d_out, n, eps, dm);
+  return launch_status();
+}
+
+dora_status_t dora_get_device_status(dora_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DORA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return DORA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess)
+      return DORA_ERR_CUDA;
+  }
+  return static_cast<dora_status_t>(v);
+}
+
+const char* dora_status_string(dora_status_t status) {
+  switch (status) {
+    case DORA_OK: return "ok";
+    case DORA_ERR_INVALID_ARG: return "invalid argument";
+    case DORA_ERR_UNSUPPORTED: return "unsupported size, dtype or device";
+    case DORA_ERR_WORKSPACE: return "workspace missing, too small or not 256-byte aligned";
+    case DORA_ERR_CUDA: return "CUDA runtime error";
+    case DORA_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+  }
+  return "unknown status";
+}
+
+int dora_version(void) { return kVersion; }
+
+dora_status_t dora_debug_unsignalled_wait(uint64_t timeout_ns, dora_stream_t stream) {
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return DORA_ERR_CUDA;
+  if (!di->supported) return DORA_ERR_UNSUPPORTED;
+  const unsigned long long t = std::min<unsigned long long>(
+      std::max<unsigned long long>(timeout_ns, 1000ull), 1000000000ull);
+  unsignalled_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(t);
+  return launch_status();
+}
+
+uint64_t dora_launch_count(void) { return g_launches.load(); }
+
+void dora_set_timing_events(void* before, void* after) {
+  t_ev_before = static_cast<cudaEvent_t>(before);
+  t_ev_after = static_cast<cudaEvent_t>(after);
+}
+
+void dora_set_wait_timeout_ns(uint64_t ns) {
+  g_timeout_ns.store(ns == 0 ? kDefaultTimeoutNs : static_cast<unsigned long long>(ns));
+}
+
+}  // extern "C"

@@ -1,0 +1,194 @@
+/*
+ * dora.h -- C ABI of the DoRA (weight-decomposed low-rank adaptation)
+ * linear-layer hot path on NVIDIA B200 (sm_100a).
+ *
+ * What is computed (sources are named by page title and section):
+ *
+ *   LoRA update  W = W0 + s B A,  s = alpha / r
+ *       ["LoRA & DoRA: The Math, Memory, and Trade-offs", section 1]
+ *   DoRA weight  W' = m * (W0 + s B A) / ||W0 + s B A||, one magnitude and one
+ *       Euclidean norm per OUTPUT ROW of the [d_out, d_in] weight, the norm
+ *       detached from autograd  ["DoRA" (aiwiki), DoRALinear listing;
+ *       "Scaling DoRA: High-Rank Adaptation via Factored Norms and Fused
+ *       Kernels", Data Availability]
+ *   Factored norm  n_i^2 = ||W0_i||^2 + 2 s B_i.(W0 A^T)_i + s^2 B_i G B_i^T,
+ *       G = A A^T, never forming the dense product B A
+ *       ["Scaling DoRA ...", section 2 "Factored Norm Computation"]
+ *   Scale  g = m / max(n, eps)  ["Scaling DoRA ...", section 4, precision]
+ *   Compose  y = base + (g - 1) * base + g * s * lora, with (g - 1) formed in
+ *       fp32 as (m - n_c) / n_c  ["Scaling DoRA ...", section 3 numerical
+ *       stability; Data Availability composition contract]
+ *   Backward  d_base = g dy, d_lora = g s dy,
+ *       dm = sum_t dy (base + s lora) / n_c  ["Scaling DoRA ...", section 3
+ *       backward kernel]
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers unless a comment says "host".  The caller
+ *     owns every buffer, including workspaces; the library never allocates or
+ *     frees device memory.
+ *   - All matrices are row-major and contiguous: W0 [d_out, d_in],
+ *     A [r, d_in], B [d_out, r], activations [T, d_out] (d_out contiguous; the
+ *     per-row magnitude of the weight broadcasts along the activations' last
+ *     axis).  m, n, g, dm are fp32 [d_out].
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream).
+ *     Arguments are validated on the host before anything is launched; a
+ *     rejected call launches nothing.  A launch failure returns
+ *     DORA_ERR_CUDA.  A kernel that gives up on a bounded internal wait
+ *     records DORA_ERR_TIMEOUT in a device status word, read (and cleared)
+ *     by dora_get_device_status.
+ *   - Aliasing: outputs must not overlap inputs, except y == base in
+ *     dora_compose_fwd and d_base == dy in dora_compose_bwd (both
+ *     element-for-element).
+ *   - dtype DORA_BF16: W0, A, B and the activations are bf16; arithmetic is
+ *     fp32 (tensor-core bf16 products with fp32 accumulation for the norm).
+ *     dtype DORA_F32: everything fp32, CUDA-core fp32 arithmetic.
+ *   - Requires an sm_100 device (B200); otherwise DORA_ERR_UNSUPPORTED.
+ */
+#ifndef DORA_H_
+#define DORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st *dora_stream_t;
+
+typedef enum {
+  DORA_OK = 0,
+  DORA_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, bad alias  */
+  DORA_ERR_UNSUPPORTED = 2,   /* r > 512, not an sm_100 device, too many problems */
+  DORA_ERR_WORKSPACE = 3,     /* workspace missing, too small or misaligned   */
+  DORA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed         */
+  DORA_ERR_TIMEOUT = 5        /* a kernel gave up on a bounded wait           */
+} dora_status_t;
+
+typedef enum { DORA_F32 = 0, DORA_BF16 = 1 } dora_dtype_t;
+
+/* Largest adapter rank (one fp32 TMEM column per rank index). */
+#define DORA_MAX_RANK 512
+/* Largest number of modules in one grouped norm call. */
+#define DORA_MAX_GROUP 1024
+
+/* ------------------------------------------------------------------------
+ * Factored per-output-row norm  ["Scaling DoRA ...", section 2]
+ *
+ * n_out[i] = sqrt(max(||W0_i||^2 + 2 s B_i.(W0 A^T)_i + s^2 B_i (A A^T) B_i^T, 0))
+ * and, when both m and g_out are non-NULL, g_out[i] = m[i] / max(n_out[i], eps)
+ * ["Scaling DoRA ...", section 4 precision bullet; appendix B clamp].
+ *
+ * W0 [d_out, d_in], A [r, d_in], B [d_out, r] in dtype `dt`; 1 <= r <= 512.
+ * The dense [d_out, d_in] product is never formed: on the bf16 path, W0 A^T
+ * and B (s/2)(A A^T) accumulate in tensor memory and W0 is read from HBM
+ * once.  Workspace: dora_factored_norm_workspace_size() bytes, 256-byte
+ * aligned, contents undefined on entry and exit.  The result is bitwise
+ * reproducible for fixed inputs and sizes.
+ * ---------------------------------------------------------------------- */
+size_t dora_factored_norm_workspace_size(int64_t d_out, int64_t d_in, int64_t r,
+                                         dora_dtype_t dt);
+dora_status_t dora_factored_norm(const void *W0, const void *A, const void *B,
+                                 dora_dtype_t dt, int64_t d_out, int64_t d_in,
+                                 int64_t r, float s, const float *m, float eps,
+                                 float *n_out, float *g_out, void *ws,
+                                 size_t ws_bytes, dora_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Grouped factored norm: the same computation for `count` independent
+ * modules (e.g. every adapted projection of a layer stack) in one launch
+ * per stage.  `problems` is a HOST array of `count` descriptors, read during
+ * the call only; the pointers inside are device pointers.  Per problem, m and
+ * g_out may be NULL (then g is not written).  All problems share `dt` and
+ * `eps`.  1 <= count <= DORA_MAX_GROUP.  bf16 only.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  const void *W0;   /* [d_out, d_in] */
+  const void *A;    /* [r, d_in]     */
+  const void *B;    /* [d_out, r]    */
+  const float *m;   /* [d_out] or NULL */
+  float *n_out;     /* [d_out]         */
+  float *g_out;     /* [d_out] or NULL */
+  int64_t d_out, d_in, r;
+  float s;
+} dora_norm_problem_t;
+
+size_t dora_factored_norm_grouped_workspace_size(const dora_norm_problem_t *problems,
+                                                 int count, dora_dtype_t dt);
+dora_status_t dora_factored_norm_grouped(const dora_norm_problem_t *problems,
+                                         int count, dora_dtype_t dt, float eps,
+                                         void *ws, size_t ws_bytes,
+                                         dora_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Fused compose forward  ["Scaling DoRA ...", section 3 and Data Availability]
+ *
+ * With n_c = max(n, eps), g = m / n_c and (g - 1) = (m - n_c) / n_c in fp32:
+ *   y[t, j] = base[t, j] + ((g_j - 1) base[t, j] + (g_j s) lora[t, j])
+ * evaluated in fp32 and rounded once to the output dtype (round to nearest
+ * even).  base, lora, y: [T, d_out] in dtype `dt`; m, n: fp32 [d_out].
+ * One pass: two reads and one write per element.  y may equal base.
+ * T == 0 launches nothing (the activation pointers may then be NULL).
+ * ---------------------------------------------------------------------- */
+dora_status_t dora_compose_fwd(const void *base, const void *lora, const float *m,
+                               const float *n, float s, float eps, dora_dtype_t dt,
+                               int64_t T, int64_t d_out, void *y,
+                               dora_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Fused compose backward  ["Scaling DoRA ...", section 3 backward kernel]
+ *
+ *   d_base[t, j] = g_j dy[t, j],  d_lora[t, j] = (g_j s) dy[t, j]
+ *   dm[j] = (sum_t dy[t, j] (base[t, j] + s lora[t, j])) / n_c,j
+ * The norm is detached (no gradient flows to W0, A or B through n).  dm is
+ * accumulated in fp32 as per-chunk column partials summed in a fixed order
+ * (no atomics): bitwise reproducible.  d_base may equal dy.  With T == 0
+ * the activation pointers may be NULL and dm is set to zero.
+ * Workspace: dora_compose_bwd_workspace_size() bytes, 256-byte aligned.
+ * ---------------------------------------------------------------------- */
+size_t dora_compose_bwd_workspace_size(int64_t T, int64_t d_out, dora_dtype_t dt);
+dora_status_t dora_compose_bwd(const void *dy, const void *base, const void *lora,
+                               const float *m, const float *n, float s, float eps,
+                               dora_dtype_t dt, int64_t T, int64_t d_out,
+                               void *d_base, void *d_lora, float *dm, void *ws,
+                               size_t ws_bytes, dora_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Status and diagnostics
+ * ---------------------------------------------------------------------- */
+/* Synchronises `stream`, returns the first error any kernel of this library
+ * recorded on the current device since the last call (DORA_OK if none), and
+ * clears it. */
+dora_status_t dora_get_device_status(dora_stream_t stream);
+/* Static English description of a status code; never NULL. */
+const char *dora_status_string(dora_status_t status);
+/* Library version, major * 10000 + minor * 100 + patch. */
+int dora_version(void);
+/* Number of kernels this library has launched in this process. */
+uint64_t dora_launch_count(void);
+/* Upper bound, in nanoseconds, on any single internal wait of the
+ * tensor-core kernels (default 2e9).  0 restores the default.  Host-side
+ * setting, applied to launches made after the call; exists so that tests can
+ * exercise the give-up path without a real hang. */
+void dora_set_wait_timeout_ns(uint64_t ns);
+/* Timing hook: the next entry-point call made by the calling host thread
+ * records `before` immediately before, and `after` immediately after, the
+ * launch of its principal kernel (the fused norm GEMM of the norm calls, the
+ * compose kernel of the compose calls) on that call's stream; the hook then
+ * clears itself.  Both are cudaEvent_t handles created by the caller (NULL,
+ * NULL clears the hook).  Lets a caller time that one kernel with CUDA events
+ * on the stream it runs on. */
+void dora_set_timing_events(void *before, void *after);
+/* Launches one thread that waits, with the same bounded wait the
+ * tensor-core pipelines use, on a barrier that nothing ever signals, giving
+ * up after `timeout_ns` (clamped to [1 us, 1 s]).  The give-up is recorded as
+ * DORA_ERR_TIMEOUT for dora_get_device_status.  Diagnostic: it lets a test
+ * check the give-up path deterministically without a real hang. */
+dora_status_t dora_debug_unsignalled_wait(uint64_t timeout_ns, dora_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DORA_H_ */

@@ -1,0 +1,116 @@
+"""CPU-side checks of the C ABI: the library loads, exports every function
+include/dora.h declares, and rejects bad arguments on the host before any
+launch.  No compute call runs here (there is no GPU in this suite)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import dora_adapter_factored_b200 as dora
+from dora_adapter_factored_b200 import _abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dora.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(dora_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary(built_library):
+    names = _declared_functions()
+    for required in ("dora_factored_norm", "dora_factored_norm_grouped", "dora_compose_fwd",
+                     "dora_compose_bwd"):
+        assert required in names
+    assert sorted(_abi.EXPORTED) == names
+
+
+def test_library_exports_every_declared_symbol(built_library):
+    lib = ctypes.CDLL(built_library)
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version(built_library):
+    lib = dora.load_library(built_library)
+    for code in range(6):
+        assert len(dora.status_string(code)) > 0
+    assert dora.status_string(99) == "unknown status"
+    assert dora.dora_version() == 100
+
+
+def test_host_validation_rejects_before_launch(built_library):
+    lib = dora.load_library(built_library)
+    before = dora.dora_launch_count()
+    p = ctypes.c_void_p(0x10000)   # never dereferenced: validation fails first
+    # null pointers
+    assert lib.dora_factored_norm(None, p, p, _abi.DORA_BF16, 8, 8, 8, 2.0, None, 0.0, p, None,
+                                  p, 1 << 20, None) == _abi.DORA_ERR_INVALID_ARG
+    # rank above the TMEM limit
+    assert lib.dora_factored_norm(p, p, p, _abi.DORA_BF16, 8, 8, 513, 2.0, None, 0.0, p, None,
+                                  p, 1 << 20, None) == _abi.DORA_ERR_UNSUPPORTED
+    # non-positive sizes
+    assert lib.dora_factored_norm(p, p, p, _abi.DORA_BF16, 0, 8, 8, 2.0, None, 0.0, p, None,
+                                  p, 1 << 20, None) == _abi.DORA_ERR_INVALID_ARG
+    # m without g_out
+    assert lib.dora_factored_norm(p, p, p, _abi.DORA_BF16, 8, 8, 8, 2.0, p, 0.0, p, None,
+                                  p, 1 << 20, None) == _abi.DORA_ERR_INVALID_ARG
+    # bad dtype
+    assert lib.dora_factored_norm(p, p, p, 7, 8, 8, 8, 2.0, None, 0.0, p, None,
+                                  p, 1 << 20, None) == _abi.DORA_ERR_INVALID_ARG
+    # compose: y overlapping lora
+    assert lib.dora_compose_fwd(p, ctypes.c_void_p(0x10000), p, p, 2.0, 0.0, _abi.DORA_BF16, 4, 8,
+                                ctypes.c_void_p(0x10008), None) == _abi.DORA_ERR_INVALID_ARG
+    # compose: negative T
+    assert lib.dora_compose_fwd(p, p, p, p, 2.0, 0.0, _abi.DORA_BF16, -1, 8, p,
+                                None) == _abi.DORA_ERR_INVALID_ARG
+    # backward: d_lora aliasing dy
+    assert lib.dora_compose_bwd(p, ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000), p, p, 2.0,
+                                0.0, _abi.DORA_BF16, 4, 8, ctypes.c_void_p(0x40000), p,
+                                ctypes.c_void_p(0x50000), p, 1 << 20,
+                                None) == _abi.DORA_ERR_INVALID_ARG
+    # grouped: too many problems, bad dtype
+    arr = (_abi.NormProblem * 1)()
+    assert lib.dora_factored_norm_grouped(arr, 0, _abi.DORA_BF16, 0.0, p, 1 << 20,
+                                          None) == _abi.DORA_ERR_INVALID_ARG
+    assert lib.dora_factored_norm_grouped(arr, 1, _abi.DORA_F32, 0.0, p, 1 << 20,
+                                          None) == _abi.DORA_ERR_UNSUPPORTED
+    assert dora.dora_launch_count() == before
+
+
+def test_workspace_sizes_are_host_computable(built_library):
+    lib = dora.load_library(built_library)
+    # headline module: G' + Gram partials + norm partials, all modest
+    ws = lib.dora_factored_norm_workspace_size(8192, 8192, 384, _abi.DORA_BF16)
+    assert 384 * 384 * 2 < ws < 64 << 20
+    # fp32 path: the fp32 Gram matrix
+    assert lib.dora_factored_norm_workspace_size(64, 48, 8, _abi.DORA_F32) >= 8 * 8 * 4
+    assert lib.dora_factored_norm_workspace_size(8, 8, 600, _abi.DORA_BF16) == 0
+    # backward partials: chunks x d_out fp32
+    wb = lib.dora_compose_bwd_workspace_size(8192, 25600, _abi.DORA_BF16)
+    assert 25600 * 4 <= wb < 64 << 20
+    assert lib.dora_compose_bwd_workspace_size(0, 16, _abi.DORA_BF16) >= 0
+
+
+def test_binding_rejects_cpu_tensors(built_library):
+    import torch
+    dora.load_library(built_library)
+    x = torch.zeros(4, 8, dtype=torch.bfloat16)
+    m = torch.ones(8)
+    with pytest.raises(ValueError):
+        dora.dora_compose_fwd(x, x, m, m, 2.0)
+
+
+def test_calls_without_a_device_fail_cleanly(built_library):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    lib = dora.load_library(built_library)
+    p = ctypes.c_void_p(0x10000)
+    st = lib.dora_compose_fwd(p, ctypes.c_void_p(0x90000), p, p, 2.0, 0.0, _abi.DORA_BF16, 4, 8,
+                              ctypes.c_void_p(0x20000), None)
+    assert st == _abi.DORA_ERR_CUDA
