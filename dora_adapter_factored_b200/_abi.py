@@ -32,13 +32,17 @@ EXPORTED = (
     "dora_compose_fwd", "dora_compose_bwd_workspace_size", "dora_compose_bwd",
     "dora_get_device_status", "dora_status_string", "dora_version", "dora_launch_count",
     "dora_set_wait_timeout_ns", "dora_debug_unsignalled_wait", "dora_set_timing_events",
+    "dora_last_error",
 )
 
 
 class DoraError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        detail = ""
+        if status == DORA_ERR_CUDA:
+            detail = " [" + load_library().dora_last_error().decode() + "]"
+        super().__init__(f"{where}: {status_string(status)} (status {status}){detail}")
 
 
 class NormProblem(ctypes.Structure):
@@ -100,6 +104,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.dora_debug_unsignalled_wait.restype = c_i
         lib.dora_set_timing_events.argtypes = [c_vp, c_vp]
         lib.dora_set_timing_events.restype = None
+        lib.dora_last_error.argtypes = []
+        lib.dora_last_error.restype = ctypes.c_char_p
         _lib = lib
         return lib
 

@@ -5,27 +5,30 @@
 //
 // Both kernels are HBM-bound streams: 16-byte vector loads/stores along
 // d_out, each thread keeps its columns' coefficients in registers and walks
-// rows; four rows are loaded before any is used so that enough bytes are in
-// flight.  No tensor cores.
+// rows; several rows are loaded (as raw 16-byte registers) before any is
+// used so that enough bytes are in flight.  No tensor cores.
 #pragma once
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace dora {
 
-// Grid shaping for the [T, d_out] streams.  Depends on the shape only (not on
-// the device), so that the backward's partial layout -- and therefore dm's
-// summation order -- is the same on every run.
+// Grid shaping for the [T, d_out] streams: a persistent grid of about two
+// blocks per SM (one wave), each block walking rows.  It depends on the shape
+// only (not on the device), so that the backward's partial layout -- and
+// therefore dm's summation order -- is the same on every run.
 constexpr int kStreamThreads = 256;
-constexpr int kStreamRowUnroll = 4;
-constexpr int kStreamTargetBlocks = 148 * 8;
+constexpr int kFwdRowUnroll = 8;
+constexpr int kBwdRowUnroll = 4;
+constexpr int kStreamSlots = 148 * 2;
 
 struct StreamGrid {
   int bx, by;
   int gx, gy;
 };
 
-inline StreamGrid stream_grid(long long T, int ncv) {
+inline StreamGrid stream_grid(long long T, int ncv, int unroll) {
   StreamGrid g;
   int best = 256;
   long long best_waste = -1;
@@ -39,69 +42,94 @@ inline StreamGrid stream_grid(long long T, int ncv) {
   g.bx = best;
   g.by = kStreamThreads / best;
   g.gx = static_cast<int>(ceil_div_ll(ncv, g.bx));
-  long long want_y = kStreamTargetBlocks / g.gx;
+  long long want_y = kStreamSlots / g.gx;
   if (want_y < 1) want_y = 1;
-  const long long max_y = ceil_div_ll(T, static_cast<long long>(g.by) * kStreamRowUnroll);
+  const long long max_y = ceil_div_ll(T, static_cast<long long>(g.by) * unroll);
   g.gy = static_cast<int>(want_y < max_y ? want_y : max_y);
   if (g.gy < 1) g.gy = 1;
   return g;
 }
 
+// Raw 16-byte (or scalar) register images of VEC consecutive elements, so that
+// several rows can be in flight without unpacking them first.
 template <typename T, int VEC>
-struct VecIO;
+struct Pack;
 
 template <>
-struct VecIO<__nv_bfloat16, 8> {
-  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[8]) {
-    const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
+struct Pack<__nv_bfloat16, 8> {
+  using raw = uint4;
+  static __device__ __forceinline__ raw load(const __nv_bfloat16* p) {
+    return __ldcs(reinterpret_cast<const uint4*>(p));
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const raw& u) {
+    __stcs(reinterpret_cast<uint4*>(p), u);
+  }
+  static __device__ __forceinline__ void unpack(const raw& u, float (&v)[8]) {
     v[0] = bf16lo_to_f32(u.x); v[1] = bf16hi_to_f32(u.x);
     v[2] = bf16lo_to_f32(u.y); v[3] = bf16hi_to_f32(u.y);
     v[4] = bf16lo_to_f32(u.z); v[5] = bf16hi_to_f32(u.z);
     v[6] = bf16lo_to_f32(u.w); v[7] = bf16hi_to_f32(u.w);
   }
-  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[8]) {
+  static __device__ __forceinline__ raw pack(const float (&v)[8]) {
     uint4 u;
     u.x = pack_bf16x2_rn(v[0], v[1]);
     u.y = pack_bf16x2_rn(v[2], v[3]);
     u.z = pack_bf16x2_rn(v[4], v[5]);
     u.w = pack_bf16x2_rn(v[6], v[7]);
-    __stcs(reinterpret_cast<uint4*>(p), u);
+    return u;
   }
 };
 
 template <>
-struct VecIO<float, 4> {
-  static __device__ __forceinline__ void load(const float* p, float (&v)[4]) {
-    const float4 u = __ldcs(reinterpret_cast<const float4*>(p));
+struct Pack<float, 4> {
+  using raw = float4;
+  static __device__ __forceinline__ raw load(const float* p) {
+    return __ldcs(reinterpret_cast<const float4*>(p));
+  }
+  static __device__ __forceinline__ void store(float* p, const raw& u) {
+    __stcs(reinterpret_cast<float4*>(p), u);
+  }
+  static __device__ __forceinline__ void unpack(const raw& u, float (&v)[4]) {
     v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
   }
-  static __device__ __forceinline__ void store(float* p, const float (&v)[4]) {
-    __stcs(reinterpret_cast<float4*>(p), make_float4(v[0], v[1], v[2], v[3]));
+  static __device__ __forceinline__ raw pack(const float (&v)[4]) {
+    return make_float4(v[0], v[1], v[2], v[3]);
   }
 };
 
 template <>
-struct VecIO<__nv_bfloat16, 1> {
-  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[1]) {
-    v[0] = __bfloat162float(*p);
+struct Pack<__nv_bfloat16, 1> {
+  using raw = __nv_bfloat16;
+  static __device__ __forceinline__ raw load(const __nv_bfloat16* p) { return *p; }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const raw& u) { *p = u; }
+  static __device__ __forceinline__ void unpack(const raw& u, float (&v)[1]) {
+    v[0] = __bfloat162float(u);
   }
-  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[1]) {
-    *p = __float2bfloat16_rn(v[0]);
+  static __device__ __forceinline__ raw pack(const float (&v)[1]) {
+    return __float2bfloat16_rn(v[0]);
   }
 };
 
 template <>
-struct VecIO<float, 1> {
-  static __device__ __forceinline__ void load(const float* p, float (&v)[1]) { v[0] = *p; }
-  static __device__ __forceinline__ void store(float* p, const float (&v)[1]) { *p = v[0]; }
+struct Pack<float, 1> {
+  using raw = float;
+  static __device__ __forceinline__ raw load(const float* p) { return *p; }
+  static __device__ __forceinline__ void store(float* p, const raw& u) { *p = u; }
+  static __device__ __forceinline__ void unpack(const raw& u, float (&v)[1]) { v[0] = u; }
+  static __device__ __forceinline__ raw pack(const float (&v)[1]) { return v[0]; }
 };
 
 // y = base + ((g - 1) base + (g s) lora), (g - 1) = (m - n_c)/n_c, g = m/n_c.
-template <typename T, int VEC>
-__global__ void __launch_bounds__(kStreamThreads)
+// Idx is the element-offset type: 32-bit when T * d_out < 2^31 (fewer live
+// registers per in-flight row), 64-bit otherwise.
+template <typename T, int VEC, typename Idx>
+__global__ void __launch_bounds__(kStreamThreads, 2)
     compose_fwd_kernel(const T* __restrict__ base, const T* __restrict__ lora,
                        const float* __restrict__ m, const float* __restrict__ n, float s,
                        float eps, long long T_rows, int d_out, T* y) {
+  using P = Pack<T, VEC>;
+  grid_dependency_wait();
+  grid_dependency_trigger();
   const int cv = blockIdx.x * blockDim.x + threadIdx.x;
   const int col0 = cv * VEC;
   if (col0 >= d_out) return;
@@ -115,25 +143,28 @@ __global__ void __launch_bounds__(kStreamThreads)
   }
   const long long stride = static_cast<long long>(gridDim.y) * blockDim.y;
   long long t = static_cast<long long>(blockIdx.y) * blockDim.y + threadIdx.y;
-  for (; t < T_rows; t += kStreamRowUnroll * stride) {
-    float b[kStreamRowUnroll][VEC], l[kStreamRowUnroll][VEC];
+  for (; t < T_rows; t += kFwdRowUnroll * stride) {
+    typename P::raw rb[kFwdRowUnroll], rl[kFwdRowUnroll];
 #pragma unroll
-    for (int u = 0; u < kStreamRowUnroll; ++u) {
+    for (int u = 0; u < kFwdRowUnroll; ++u) {
       const long long tt = t + u * stride;
       if (tt < T_rows) {
-        const size_t off = static_cast<size_t>(tt) * d_out + col0;
-        VecIO<T, VEC>::load(base + off, b[u]);
-        VecIO<T, VEC>::load(lora + off, l[u]);
+        const Idx off = static_cast<Idx>(tt) * static_cast<Idx>(d_out) + static_cast<Idx>(col0);
+        rb[u] = P::load(base + off);
+        rl[u] = P::load(lora + off);
       }
     }
 #pragma unroll
-    for (int u = 0; u < kStreamRowUnroll; ++u) {
+    for (int u = 0; u < kFwdRowUnroll; ++u) {
       const long long tt = t + u * stride;
       if (tt < T_rows) {
-        float o[VEC];
+        float b[VEC], l[VEC], o[VEC];
+        P::unpack(rb[u], b);
+        P::unpack(rl[u], l);
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) o[e] = b[u][e] + fmaf(gm1[e], b[u][e], gs[e] * l[u][e]);
-        VecIO<T, VEC>::store(y + static_cast<size_t>(tt) * d_out + col0, o);
+        for (int e = 0; e < VEC; ++e) o[e] = b[e] + fmaf(gm1[e], b[e], gs[e] * l[e]);
+        const Idx off = static_cast<Idx>(tt) * static_cast<Idx>(d_out) + static_cast<Idx>(col0);
+        P::store(y + off, P::pack(o));
       }
     }
   }
@@ -141,13 +172,16 @@ __global__ void __launch_bounds__(kStreamThreads)
 
 // d_base = g dy, d_lora = (g s) dy, and per-block column partials of
 // sum_t dy (base + s lora) written to partial[blockIdx.y][d_out].
-template <typename T, int VEC>
-__global__ void __launch_bounds__(kStreamThreads)
+template <typename T, int VEC, typename Idx>
+__global__ void __launch_bounds__(kStreamThreads, 2)
     compose_bwd_kernel(const T* dy, const T* __restrict__ base, const T* __restrict__ lora,
                        const float* __restrict__ m, const float* __restrict__ n, float s,
                        float eps, long long T_rows, int d_out, T* d_base, T* __restrict__ d_lora,
                        float* __restrict__ partial) {
+  using P = Pack<T, VEC>;
   __shared__ float red[kStreamThreads * VEC];
+  grid_dependency_wait();
+  grid_dependency_trigger();
   const int cv = blockIdx.x * blockDim.x + threadIdx.x;
   const int col0 = cv * VEC;
   const bool active = col0 < d_out;
@@ -165,60 +199,79 @@ __global__ void __launch_bounds__(kStreamThreads)
   if (active) {
     const long long stride = static_cast<long long>(gridDim.y) * blockDim.y;
     long long t = static_cast<long long>(blockIdx.y) * blockDim.y + threadIdx.y;
-    for (; t < T_rows; t += kStreamRowUnroll * stride) {
-      float d[kStreamRowUnroll][VEC], b[kStreamRowUnroll][VEC], l[kStreamRowUnroll][VEC];
+    for (; t < T_rows; t += kBwdRowUnroll * stride) {
+      typename P::raw rd[kBwdRowUnroll], rb[kBwdRowUnroll], rl[kBwdRowUnroll];
 #pragma unroll
-      for (int u = 0; u < kStreamRowUnroll; ++u) {
+      for (int u = 0; u < kBwdRowUnroll; ++u) {
         const long long tt = t + u * stride;
         if (tt < T_rows) {
-          const size_t off = static_cast<size_t>(tt) * d_out + col0;
-          VecIO<T, VEC>::load(dy + off, d[u]);
-          VecIO<T, VEC>::load(base + off, b[u]);
-          VecIO<T, VEC>::load(lora + off, l[u]);
+          const Idx off = static_cast<Idx>(tt) * static_cast<Idx>(d_out) + static_cast<Idx>(col0);
+          rd[u] = P::load(dy + off);
+          rb[u] = P::load(base + off);
+          rl[u] = P::load(lora + off);
         }
       }
 #pragma unroll
-      for (int u = 0; u < kStreamRowUnroll; ++u) {
+      for (int u = 0; u < kBwdRowUnroll; ++u) {
         const long long tt = t + u * stride;
         if (tt < T_rows) {
-          float ob[VEC], ol[VEC];
+          float d[VEC], b[VEC], l[VEC], ob[VEC], ol[VEC];
+          P::unpack(rd[u], d);
+          P::unpack(rb[u], b);
+          P::unpack(rl[u], l);
 #pragma unroll
           for (int e = 0; e < VEC; ++e) {
-            ob[e] = g[e] * d[u][e];
-            ol[e] = gs[e] * d[u][e];
-            acc[e] = fmaf(d[u][e], fmaf(s, l[u][e], b[u][e]), acc[e]);
+            ob[e] = g[e] * d[e];
+            ol[e] = gs[e] * d[e];
+            acc[e] = fmaf(d[e], fmaf(s, l[e], b[e]), acc[e]);
           }
-          const size_t off = static_cast<size_t>(tt) * d_out + col0;
-          VecIO<T, VEC>::store(d_base + off, ob);
-          VecIO<T, VEC>::store(d_lora + off, ol);
+          const Idx off = static_cast<Idx>(tt) * static_cast<Idx>(d_out) + static_cast<Idx>(col0);
+          P::store(d_base + off, P::pack(ob));
+          P::store(d_lora + off, P::pack(ol));
         }
       }
     }
   }
   // Reduce the block's rows (threadIdx.y) in a fixed order.
   const int tx = threadIdx.x, ty = threadIdx.y;
+  if (blockDim.y > 1) {
 #pragma unroll
-  for (int e = 0; e < VEC; ++e) red[(ty * blockDim.x + tx) * VEC + e] = acc[e];
-  __syncthreads();
+    for (int e = 0; e < VEC; ++e) red[(ty * blockDim.x + tx) * VEC + e] = acc[e];
+    __syncthreads();
+    if (ty == 0 && active) {
+      for (int yy = 1; yy < static_cast<int>(blockDim.y); ++yy)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] += red[(yy * blockDim.x + tx) * VEC + e];
+    }
+  }
   if (ty == 0 && active) {
-    for (int yy = 1; yy < static_cast<int>(blockDim.y); ++yy)
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) acc[e] += red[(yy * blockDim.x + tx) * VEC + e];
     float* dst = partial + static_cast<size_t>(blockIdx.y) * d_out + col0;
 #pragma unroll
     for (int e = 0; e < VEC; ++e) dst[e] = acc[e];
   }
 }
 
-// dm_j = (sum over row chunks, in chunk order) / max(n_j, eps).
+// dm_j = (sum over row chunks, in a fixed order) / max(n_j, eps).  Block
+// (32, 8): thread (x, y) sums chunks y, y + 8, ... of column x, then the
+// eight sums are added in y order.
 __global__ void __launch_bounds__(256)
     colsum_finalize_kernel(const float* __restrict__ partial, int chunks, int d_out,
                            const float* __restrict__ n, float eps, float* __restrict__ dm) {
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= d_out) return;
+  __shared__ float red[8][33];
+  grid_dependency_wait();
+  grid_dependency_trigger();
+  const int j = blockIdx.x * 32 + threadIdx.x;
   float s = 0.f;
-  for (int c = 0; c < chunks; ++c) s += partial[static_cast<size_t>(c) * d_out + j];
-  dm[j] = __fdiv_rn(s, fmaxf(__ldg(n + j), eps));
+  if (j < d_out)
+    for (int c = threadIdx.y; c < chunks; c += 8) s += partial[static_cast<size_t>(c) * d_out + j];
+  red[threadIdx.y][threadIdx.x] = s;
+  __syncthreads();
+  if (threadIdx.y == 0 && j < d_out) {
+    float t = red[0][threadIdx.x];
+#pragma unroll
+    for (int y = 1; y < 8; ++y) t += red[y][threadIdx.x];
+    dm[j] = __fdiv_rn(t, fmaxf(__ldg(n + j), eps));
+  }
 }
 
 }  // namespace dora

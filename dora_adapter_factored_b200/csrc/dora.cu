@@ -7,8 +7,10 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "dora.h"
@@ -78,9 +80,66 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   return x < y + nb && y < x + na;
 }
 
+// Launch with programmatic stream serialization: the kernel may start while
+// its predecessor drains; every kernel of the library executes
+// griddepcontrol.wait before it reads anything a predecessor writes, and
+// before it lets its own dependents launch.
+// If the runtime rejects the programmatic attribute for this stream, the
+// kernel is launched again without it (plain stream order).
+thread_local char t_last_error[512] = "";
+thread_local bool launch_failed = false;
+
+void note_error(const char* where, cudaError_t e) {
+  snprintf(t_last_error, sizeof(t_last_error), "%s: %s (%d)", where, cudaGetErrorString(e),
+           static_cast<int>(e));
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    cfg.numAttrs = 0;
+    e = cudaLaunchKernelEx(&cfg, kernel, args...);
+    if (e != cudaSuccess) {
+      // Describe the kernel that could not be launched.
+      cudaFuncAttributes fa = {};
+      cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(kernel));
+      snprintf(t_last_error, sizeof(t_last_error),
+               "launch of grid (%u,%u,%u) x block (%u,%u,%u), %zu B dynamic smem: %s (%d); "
+               "kernel: %d regs, max %d threads/block, %zu B static smem, max %d B dynamic, "
+               "%zu B local",
+               grid.x, grid.y, grid.z, block.x, block.y, block.z, smem, cudaGetErrorString(e),
+               static_cast<int>(e), fa.numRegs, fa.maxThreadsPerBlock, fa.sharedSizeBytes,
+               fa.maxDynamicSharedSizeBytes, fa.localSizeBytes);
+      cudaGetLastError();
+      launch_failed = true;
+    }
+  }
+  return e;
+}
+
 dora_status_t launch_status() {
   g_launches.fetch_add(1, std::memory_order_relaxed);
-  return cudaGetLastError() == cudaSuccess ? DORA_OK : DORA_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  if (launch_failed) {
+    launch_failed = false;  // the launch helper already described it
+    return DORA_ERR_CUDA;
+  }
+  if (e == cudaSuccess) return DORA_OK;
+  note_error("kernel launch", e);
+  return DORA_ERR_CUDA;
 }
 
 // ------------------------------------------------------------ tensor maps
@@ -153,7 +212,7 @@ void plan_module(int64_t d_out, int64_t d_in, int64_t r, ModulePlan& p) {
   plan_n_side(static_cast<int>(r), p);
   p.kb_w = static_cast<int>(ceil_div_ll(d_in, kBlockK));
   p.kb_r = static_cast<int>(ceil_div_ll(r, kBlockK));
-  p.kb_tile = p.kb_w + p.kb_r;
+  p.kb_tile = p.kb_w + 2 * p.kb_r;  // W0 blocks, then B.G'_hi, then B.G'_lo
   p.tiles = static_cast<int>(ceil_div_ll(d_out, kTileM));
   p.units = static_cast<long long>(p.tiles) * p.kb_tile;
   p.r8 = round_up_int(static_cast<int>(r), 8);
@@ -214,9 +273,10 @@ bool layout_group(const int64_t* d_out, const int64_t* d_in, const int64_t* r, i
   if (L.ctas < 1) return false;
   L.seg_slots = max_seg_slots(L.plans, L.total_units, L.ctas);
   const uint32_t stage_bytes = kTileABytes + L.b_region;
-  L.stages = std::min<int>(kMaxStages, (kMaxDynSmem - 1024 - 256) / stage_bytes);
+  const int tail_bytes = static_cast<int>(align_up(sizeof(NormSmemTail), 128));
+  L.stages = std::min<int>(kMaxStages, (kMaxDynSmem - 1024 - tail_bytes) / stage_bytes);
   if (L.stages < 2) return false;
-  L.smem_bytes = 1024 + static_cast<size_t>(L.stages) * stage_bytes + 256;
+  L.smem_bytes = 1024 + static_cast<size_t>(L.stages) * stage_bytes + tail_bytes;
   size_t off = 0;
   if (grouped) {
     off = align_up(sizeof(NormProblemDev) * count, 256) + align_up(sizeof(GramProblemDev) * count, 256);
@@ -225,7 +285,7 @@ bool layout_group(const int64_t* d_out, const int64_t* d_in, const int64_t* r, i
   for (auto& p : L.plans) {
     p.seg_slots = L.seg_slots;
     p.off_g = off;
-    off += align_up(static_cast<size_t>(p.n_pad) * p.r8 * 2 + 0, 256);
+    off += align_up(static_cast<size_t>(2) * p.n_pad * p.r8 * 2, 256);  // G'_hi, G'_lo
     p.off_gp = off;
     off += align_up(static_cast<size_t>(p.pairs) * p.S * kTileM * kTileM * 4, 256);
     p.off_np = off;
@@ -243,17 +303,22 @@ bool ensure_tc_attrs(int smem_norm) {
   if (d.attrs_set) return true;
   (void)smem_norm;
   const int gram_smem = 1024 + kGramStages * kGramStageBytes + 256;
-  bool ok = true;
-  ok &= cudaFuncSetAttribute(norm_main_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kMaxDynSmem) == cudaSuccess;
-  ok &= cudaFuncSetAttribute(norm_main_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kMaxDynSmem) == cudaSuccess;
-  ok &= cudaFuncSetAttribute(gram_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             gram_smem) == cudaSuccess;
-  ok &= cudaFuncSetAttribute(gram_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             gram_smem) == cudaSuccess;
-  d.attrs_set = ok;
-  return ok;
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(norm_main_kernel<false>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem)) !=
+          cudaSuccess ||
+      (e = cudaFuncSetAttribute(norm_main_kernel<true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem)) !=
+          cudaSuccess ||
+      (e = cudaFuncSetAttribute(gram_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                gram_smem)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(gram_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                gram_smem)) != cudaSuccess) {
+    note_error("cudaFuncSetAttribute", e);
+    return false;
+  }
+  d.attrs_set = true;
+  return true;
 }
 
 // Fills the device descriptors of one module.
@@ -263,11 +328,13 @@ bool fill_descriptors(const dora_norm_problem_t& pr, const ModulePlan& p, uint8_
   std::memset(&nd, 0, sizeof(nd));
   std::memset(&gd, 0, sizeof(gd));
   uint16_t* gprime = reinterpret_cast<uint16_t*>(ws_base + p.off_g);
+  uint16_t* gprime_lo = gprime + static_cast<size_t>(p.n_pad) * p.r8;
   bool ok = true;
   ok &= make_tmap_bf16(&nd.tm_w0, pr.W0, pr.d_out, pr.d_in, pr.d_in, kBlockK, kTileM);
   ok &= make_tmap_bf16(&nd.tm_a, pr.A, pr.r, pr.d_in, pr.d_in, kBlockK, p.box_rows);
   ok &= make_tmap_bf16(&nd.tm_b, pr.B, pr.d_out, pr.r, pr.r, kBlockK, kTileM);
   ok &= make_tmap_bf16(&nd.tm_g, gprime, pr.r, pr.r, p.r8, kBlockK, p.box_rows);
+  ok &= make_tmap_bf16(&nd.tm_glo, gprime_lo, pr.r, pr.r, p.r8, kBlockK, p.box_rows);
   ok &= make_tmap_bf16(&gd.tm_a, pr.A, pr.r, pr.d_in, pr.d_in, kBlockK, kTileM);
   nd.B = static_cast<const uint16_t*>(pr.B);
   nd.partial = reinterpret_cast<float*>(ws_base + p.off_np);
@@ -293,6 +360,7 @@ bool fill_descriptors(const dora_norm_problem_t& pr, const ModulePlan& p, uint8_
 
   gd.partial = reinterpret_cast<float*>(ws_base + p.off_gp);
   gd.g_out = gprime;
+  gd.g_lo = gprime_lo;
   gd.r = static_cast<int>(pr.r);
   gd.r8 = p.r8;
   gd.kb = p.kb_gram;
@@ -351,21 +419,24 @@ dora_status_t run_tc_group(const dora_norm_problem_t* probs, int count, bool gro
   const unsigned long long tmo = g_timeout_ns.load();
   const int gram_smem = 1024 + kGramStages * kGramStageBytes + 256;
   dora_status_t s;
+  const unsigned fin_x = static_cast<unsigned>(ceil_div_ll(L.max_d_out, 256));
+  const dim3 red_grid(kTileM * kTileM / 256, L.max_pairs, grouped ? count : 1);
   if (!grouped) {
-    gram_kernel<false><<<L.gram_jobs, kTcThreads, gram_smem, st>>>(gds[0], nullptr, 1, tmo);
+    launch_pdl(gram_kernel<false>, dim3(L.gram_jobs), dim3(kTcThreads), gram_smem, st, gds[0],
+               static_cast<const GramProblemDev*>(nullptr), 1, tmo);
     if ((s = launch_status()) != DORA_OK) return s;
-    gram_reduce_kernel<false><<<dim3(kTileM * kTileM / 256, L.max_pairs, 1), 256, 0, st>>>(
-        gds[0], nullptr);
+    launch_pdl(gram_reduce_kernel<false>, red_grid, dim3(256), 0, st, gds[0],
+               static_cast<const GramProblemDev*>(nullptr));
     if ((s = launch_status()) != DORA_OK) return s;
     {
       TimedLaunch tl(st);
-      norm_main_kernel<false><<<L.ctas, kTcThreads, L.smem_bytes, st>>>(
-          nds[0], nullptr, 1, L.total_units, L.stages, L.b_region, L.tmem_cols, tmo);
+      launch_pdl(norm_main_kernel<false>, dim3(L.ctas), dim3(kNormThreads), L.smem_bytes, st,
+                 nds[0], static_cast<const NormProblemDev*>(nullptr), 1, L.total_units, L.stages,
+                 L.b_region, static_cast<uint32_t>(L.tmem_cols), tmo);
       if ((s = launch_status()) != DORA_OK) return s;
     }
-    norm_finalize_kernel<false>
-        <<<dim3(static_cast<unsigned>(ceil_div_ll(L.max_d_out, 256)), 1), 256, 0, st>>>(
-            nds[0], nullptr, L.total_units, L.ctas, eps);
+    launch_pdl(norm_finalize_kernel<false>, dim3(fin_x, 1), dim3(256), 0, st, nds[0],
+               static_cast<const NormProblemDev*>(nullptr), L.total_units, L.ctas, eps);
     return launch_status();
   }
   NormProblemDev* ntab = reinterpret_cast<NormProblemDev*>(base);
@@ -376,22 +447,24 @@ dora_status_t run_tc_group(const dora_norm_problem_t* probs, int count, bool gro
       cudaMemcpyAsync(gtab, gds.data(), sizeof(GramProblemDev) * count, cudaMemcpyHostToDevice,
                       st) != cudaSuccess)
     return DORA_ERR_CUDA;
-  gram_kernel<true><<<L.gram_jobs, kTcThreads, gram_smem, st>>>(gds[0], gtab, count, tmo);
+  launch_pdl(gram_kernel<true>, dim3(L.gram_jobs), dim3(kTcThreads), gram_smem, st, gds[0],
+             static_cast<const GramProblemDev*>(gtab), count, tmo);
   if ((s = launch_status()) != DORA_OK) return s;
-  gram_reduce_kernel<true><<<dim3(kTileM * kTileM / 256, L.max_pairs, count), 256, 0, st>>>(
-      gds[0], gtab);
+  launch_pdl(gram_reduce_kernel<true>, red_grid, dim3(256), 0, st, gds[0],
+             static_cast<const GramProblemDev*>(gtab));
   if ((s = launch_status()) != DORA_OK) return s;
   {
     TimedLaunch tl(st);
-    norm_main_kernel<true><<<L.ctas, kTcThreads, L.smem_bytes, st>>>(
-        nds[0], ntab, count, L.total_units, L.stages, L.b_region, L.tmem_cols, tmo);
+    launch_pdl(norm_main_kernel<true>, dim3(L.ctas), dim3(kNormThreads), L.smem_bytes, st, nds[0],
+               static_cast<const NormProblemDev*>(ntab), count, L.total_units, L.stages,
+               L.b_region, static_cast<uint32_t>(L.tmem_cols), tmo);
     if ((s = launch_status()) != DORA_OK) return s;
   }
-  norm_finalize_kernel<true>
-      <<<dim3(static_cast<unsigned>(ceil_div_ll(L.max_d_out, 256)), count), 256, 0, st>>>(
-          nds[0], ntab, L.total_units, L.ctas, eps);
+  launch_pdl(norm_finalize_kernel<true>, dim3(fin_x, count), dim3(256), 0, st, nds[0],
+             static_cast<const NormProblemDev*>(ntab), L.total_units, L.ctas, eps);
   return launch_status();
 }
+
 
 // One thread waits on a barrier that nothing arrives on; the bounded wait
 // gives up and records DORA_ERR_TIMEOUT.
@@ -405,6 +478,42 @@ __global__ void unsignalled_wait_kernel(unsigned long long timeout_ns) {
 
 size_t simt_workspace(int64_t r) { return align_up(static_cast<size_t>(r) * r * 4, 256); }
 
+}  // namespace
+}  // namespace dora
+
+namespace dora {
+namespace {
+template <typename E, int VEC>
+void launch_fwd(bool small, int64_t rows, int64_t d_out, const void* base, const void* lora,
+                const float* m, const float* n, float s, float eps, void* y, cudaStream_t cs) {
+  const StreamGrid g = stream_grid(rows, static_cast<int>(d_out / VEC), kFwdRowUnroll);
+  const dim3 grid(g.gx, g.gy), block(g.bx, g.by);
+  if (small)
+    launch_pdl(compose_fwd_kernel<E, VEC, uint32_t>, grid, block, 0, cs,
+               static_cast<const E*>(base), static_cast<const E*>(lora), m, n, s, eps,
+               static_cast<long long>(rows), (int)d_out, static_cast<E*>(y));
+  else
+    launch_pdl(compose_fwd_kernel<E, VEC, uint64_t>, grid, block, 0, cs,
+               static_cast<const E*>(base), static_cast<const E*>(lora), m, n, s, eps,
+               static_cast<long long>(rows), (int)d_out, static_cast<E*>(y));
+}
+
+template <typename E, int VEC>
+void launch_bwd(bool small, const StreamGrid& g, int64_t rows, int64_t d_out, const void* dy,
+                const void* base, const void* lora, const float* m, const float* n, float s,
+                float eps, void* d_base, void* d_lora, float* partial, cudaStream_t cs) {
+  const dim3 grid(g.gx, g.gy), block(g.bx, g.by);
+  if (small)
+    launch_pdl(compose_bwd_kernel<E, VEC, uint32_t>, grid, block, 0, cs,
+               static_cast<const E*>(dy), static_cast<const E*>(base),
+               static_cast<const E*>(lora), m, n, s, eps, static_cast<long long>(rows),
+               (int)d_out, static_cast<E*>(d_base), static_cast<E*>(d_lora), partial);
+  else
+    launch_pdl(compose_bwd_kernel<E, VEC, uint64_t>, grid, block, 0, cs,
+               static_cast<const E*>(dy), static_cast<const E*>(base),
+               static_cast<const E*>(lora), m, n, s, eps, static_cast<long long>(rows),
+               (int)d_out, static_cast<E*>(d_base), static_cast<E*>(d_lora), partial);
+}
 }  // namespace
 }  // namespace dora
 
@@ -516,31 +625,19 @@ dora_status_t dora_compose_fwd(const void* base, const void* lora, const float* 
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   TimedLaunch tl(cs);
   const bool al = aligned16(base) && aligned16(lora) && aligned16(y);
+  const bool small = static_cast<unsigned long long>(T) * static_cast<unsigned long long>(d_out) <
+                     (1ull << 31);
   if (dt == DORA_BF16) {
     using B16 = __nv_bfloat16;
-    if (al && d_out % 8 == 0) {
-      const StreamGrid g = stream_grid(T, static_cast<int>(d_out / 8));
-      compose_fwd_kernel<B16, 8><<<dim3(g.gx, g.gy), dim3(g.bx, g.by), 0, cs>>>(
-          static_cast<const B16*>(base), static_cast<const B16*>(lora), m, n, s, eps, T,
-          (int)d_out, static_cast<B16*>(y));
-    } else {
-      const StreamGrid g = stream_grid(T, static_cast<int>(d_out));
-      compose_fwd_kernel<B16, 1><<<dim3(g.gx, g.gy), dim3(g.bx, g.by), 0, cs>>>(
-          static_cast<const B16*>(base), static_cast<const B16*>(lora), m, n, s, eps, T,
-          (int)d_out, static_cast<B16*>(y));
-    }
+    if (al && d_out % 8 == 0)
+      launch_fwd<B16, 8>(small, T, d_out, base, lora, m, n, s, eps, y, cs);
+    else
+      launch_fwd<B16, 1>(small, T, d_out, base, lora, m, n, s, eps, y, cs);
   } else {
-    if (al && d_out % 4 == 0) {
-      const StreamGrid g = stream_grid(T, static_cast<int>(d_out / 4));
-      compose_fwd_kernel<float, 4><<<dim3(g.gx, g.gy), dim3(g.bx, g.by), 0, cs>>>(
-          static_cast<const float*>(base), static_cast<const float*>(lora), m, n, s, eps, T,
-          (int)d_out, static_cast<float*>(y));
-    } else {
-      const StreamGrid g = stream_grid(T, static_cast<int>(d_out));
-      compose_fwd_kernel<float, 1><<<dim3(g.gx, g.gy), dim3(g.bx, g.by), 0, cs>>>(
-          static_cast<const float*>(base), static_cast<const float*>(lora), m, n, s, eps, T,
-          (int)d_out, static_cast<float*>(y));
-    }
+    if (al && d_out % 4 == 0)
+      launch_fwd<float, 4>(small, T, d_out, base, lora, m, n, s, eps, y, cs);
+    else
+      launch_fwd<float, 1>(small, T, d_out, base, lora, m, n, s, eps, y, cs);
   }
   return launch_status();
 }
@@ -554,7 +651,7 @@ BwdShape bwd_shape(int64_t T, int64_t d_out, dora_dtype_t dt, bool aligned) {
   BwdShape b;
   const int v = dt == DORA_BF16 ? 8 : 4;
   b.vec = (aligned && d_out % v == 0) ? v : 1;
-  b.g = stream_grid(T, static_cast<int>(d_out / b.vec));
+  b.g = stream_grid(T, static_cast<int>(d_out / b.vec), kBwdRowUnroll);
   return b;
 }
 }  // namespace
@@ -600,39 +697,31 @@ dora_status_t dora_compose_bwd(const void* dy, const void* base, const void* lor
   const size_t need = static_cast<size_t>(b.g.gy) * d_out * 4;
   if (ws == nullptr || ws_bytes < need || !aligned256(ws)) return DORA_ERR_WORKSPACE;
   float* partial = static_cast<float*>(ws);
-  const dim3 grid(b.g.gx, b.g.gy), block(b.g.bx, b.g.by);
+  const bool small = static_cast<unsigned long long>(T) * static_cast<unsigned long long>(d_out) <
+                     (1ull << 31);
   dora_status_t st;
   {
-  TimedLaunch tl(cs);
-  if (dt == DORA_BF16) {
-    using B16 = __nv_bfloat16;
-    if (b.vec == 8)
-      compose_bwd_kernel<B16, 8><<<grid, block, 0, cs>>>(
-          static_cast<const B16*>(dy), static_cast<const B16*>(base),
-          static_cast<const B16*>(lora), m, n, s, eps, T, (int)d_out, static_cast<B16*>(d_base),
-          static_cast<B16*>(d_lora), partial);
-    else
-      compose_bwd_kernel<B16, 1><<<grid, block, 0, cs>>>(
-          static_cast<const B16*>(dy), static_cast<const B16*>(base),
-          static_cast<const B16*>(lora), m, n, s, eps, T, (int)d_out, static_cast<B16*>(d_base),
-          static_cast<B16*>(d_lora), partial);
-  } else {
-    if (b.vec == 4)
-      compose_bwd_kernel<float, 4><<<grid, block, 0, cs>>>(
-          static_cast<const float*>(dy), static_cast<const float*>(base),
-          static_cast<const float*>(lora), m, n, s, eps, T, (int)d_out,
-          static_cast<float*>(d_base), static_cast<float*>(d_lora), partial);
-    else
-      compose_bwd_kernel<float, 1><<<grid, block, 0, cs>>>(
-          static_cast<const float*>(dy), static_cast<const float*>(base),
-          static_cast<const float*>(lora), m, n, s, eps, T, (int)d_out,
-          static_cast<float*>(d_base), static_cast<float*>(d_lora), partial);
-  }
-  st = launch_status();
+    TimedLaunch tl(cs);
+    if (dt == DORA_BF16) {
+      if (b.vec == 8)
+        launch_bwd<__nv_bfloat16, 8>(small, b.g, T, d_out, dy, base, lora, m, n, s, eps, d_base,
+                                     d_lora, partial, cs);
+      else
+        launch_bwd<__nv_bfloat16, 1>(small, b.g, T, d_out, dy, base, lora, m, n, s, eps, d_base,
+                                     d_lora, partial, cs);
+    } else {
+      if (b.vec == 4)
+        launch_bwd<float, 4>(small, b.g, T, d_out, dy, base, lora, m, n, s, eps, d_base, d_lora,
+                             partial, cs);
+      else
+        launch_bwd<float, 1>(small, b.g, T, d_out, dy, base, lora, m, n, s, eps, d_base, d_lora,
+                             partial, cs);
+    }
+    st = launch_status();
   }
   if (st != DORA_OK) return st;
-  colsum_finalize_kernel<<<(unsigned)ceil_div_ll(d_out, 256), 256, 0, cs>>>(partial, b.g.gy,
-                                                                           (int)d_out, n, eps, dm);
+  launch_pdl(colsum_finalize_kernel, dim3((unsigned)ceil_div_ll(d_out, 32)), dim3(32, 8), 0, cs,
+             static_cast<const float*>(partial), b.g.gy, (int)d_out, n, eps, dm);
   return launch_status();
 }
 
@@ -674,6 +763,8 @@ dora_status_t dora_debug_unsignalled_wait(uint64_t timeout_ns, dora_stream_t str
 }
 
 uint64_t dora_launch_count(void) { return g_launches.load(); }
+
+const char* dora_last_error(void) { return t_last_error; }
 
 void dora_set_timing_events(void* before, void* after) {
   t_ev_before = static_cast<cudaEvent_t>(before);

@@ -7,18 +7,23 @@
 // Three kernels per module (the grouped call runs each once for all modules):
 //   gram_kernel      G' = (s/2) A A^T: 128x128 upper-triangle tiles, split
 //                    over K, fp32 partial tiles in the workspace.
-//   gram_reduce      sums the K splits in a fixed order, rounds G' to bf16 and
+//   gram_reduce      sums the K splits in a fixed order and writes G' as two
+//                    bf16 matrices, G'_hi = bf16(G') and G'_lo = bf16(G' - G'_hi),
+//                    so that the Gram term keeps fp32-level accuracy (the pages'
+//                    norm accumulates in fp32 whatever the weight dtype);
 //                    mirrors the off-diagonal tiles.
 //   norm_main_kernel one 128-row tile of W0 at a time, stream-K over the
 //                    (tile, k-block) sequence.  Per tile the accumulator in
 //                    TMEM collects  W0_tile A^T  (k-blocks over d_in) and then
-//                    B_tile G'  (k-blocks over r), so that
+//                    B_tile G'_hi and B_tile G'_lo  (k-blocks over r), so that
 //                    B_i . acc_i = B_i.(W0 A^T)_i + (s/2) B_i G B_i^T.
 //                    While the MMAs run, four warps square and sum the same
 //                    W0 tile straight from shared memory (||W0_i||^2), so W0
-//                    crosses HBM exactly once.  The epilogue drains TMEM, dots
-//                    each row with B_i and writes the per-row partial
-//                    ||W0_i||^2_part + 2 s B_i.acc_i for its k-range.
+//                    crosses HBM exactly once.  The epilogue (eight warps, each
+//                    half of a row's columns, with B_i prefetched into registers
+//                    while the MMAs run) drains TMEM, dots each row with B_i
+//                    and writes the per-row partial ||W0_i||^2_part +
+//                    2 s B_i.acc_i for its k-range.
 //   norm_finalize    n_i = sqrt(max(sum of partials, 0)) in a fixed order,
 //                    g_i = m_i / max(n_i, eps)  (section 4, precision bullet).
 #pragma once
@@ -31,7 +36,14 @@ namespace dora {
 constexpr int kTileM = 128;                  // W0 rows per tile = TMEM lanes
 constexpr int kBlockK = 64;                  // bf16 of K per stage: one 128-byte swizzle row
 constexpr int kMaxStages = 8;
-constexpr int kTcThreads = 192;              // warps 0-3: reduction/epilogue, 4: TMA, 5: MMA
+constexpr int kTcThreads = 192;              // Gram: warps 0-3 epilogue, 4 TMA, 5 MMA
+constexpr int kEpiWarps = 8;                 // norm: warps 0-7 reduction/epilogue
+constexpr int kNormThreads = (kEpiWarps + 2) * 32;  // + warp 8 TMA, warp 9 MMA
+constexpr int kMaxChunksPerHalf = 8;         // 32-column TMEM chunks per epilogue half (r <= 512)
+constexpr int kPrefetchChunks = 6;           // of which B is prefetched into registers (r <= 384)
+// Registers are granted to a block in groups of four warps, so the 10-warp
+// norm kernel is charged as 12 warps: 65536 / 384 threads = 170 -> 168.
+constexpr int kNormMaxRegs = 168;
 constexpr uint32_t kTileABytes = kTileM * kBlockK * 2;  // 16 KiB
 constexpr int kMaxDynSmem = 232448;          // 227 KiB opt-in per block on sm_100
 
@@ -43,7 +55,8 @@ struct alignas(64) NormProblemDev {
   CUtensorMap tm_w0;     // W0 [d_out, d_in], box 64 x 128
   CUtensorMap tm_a;      // A  [r, d_in],     box 64 x box_rows
   CUtensorMap tm_b;      // B  [d_out, r],    box 64 x 128
-  CUtensorMap tm_g;      // G' [r, r],        box 64 x box_rows
+  CUtensorMap tm_g;      // G'_hi [r, r],     box 64 x box_rows
+  CUtensorMap tm_glo;    // G'_lo [r, r],     box 64 x box_rows
   const uint16_t* B;     // bf16 bits of B, for the epilogue dot
   float* partial;        // [tiles * seg_slots][128] per-row partials
   const float* m;        // [d_out] or null
@@ -53,7 +66,7 @@ struct alignas(64) NormProblemDev {
   int d_out, r;
   int n0, n1;            // N of the two accumulator chunks (n1 = 0: single chunk)
   int box_rows, nbox;    // N-side operand: boxes per stage and rows per box
-  int kb_w, kb_r, kb_tile, tiles, seg_slots;
+  int kb_w, kb_r, kb_tile, tiles, seg_slots;  // kb_tile = kb_w + 2 kb_r (hi, then lo)
   uint32_t stage_tx;     // bytes landing per stage
   uint32_t idesc0, idesc1;
   float two_s;
@@ -62,7 +75,8 @@ struct alignas(64) NormProblemDev {
 struct alignas(64) GramProblemDev {
   CUtensorMap tm_a;      // A [r, d_in], box 64 x 128
   float* partial;        // [pairs * S][128 * 128]
-  uint16_t* g_out;       // G' [r][r8] bf16 bits
+  uint16_t* g_out;       // G'_hi [r][r8] bf16 bits
+  uint16_t* g_lo;        // G'_lo [r][r8] bf16 bits
   int r, r8, kb, tiles_r, pairs, S, job_begin;
   float half_s;
 };
@@ -150,8 +164,20 @@ struct UnitCursor {
 // ---------------------------------------------------------------------------
 // Fused norm GEMM
 // ---------------------------------------------------------------------------
+struct NormSmemTail {
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
+  uint64_t acc_full;
+  uint64_t acc_empty;
+  uint64_t drain;
+  uint64_t half_ready;        // upper epilogue half has posted its partial
+  float half_part[2][kTileM];  // double-buffered by segment parity
+  uint32_t tmem_slot;
+  int abort_flag;
+};
+
 template <bool kGrouped>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __maxnreg__(kNormMaxRegs)
     norm_main_kernel(const __grid_constant__ NormProblemDev single,
                      const NormProblemDev* __restrict__ table, int nprob, long long total_units,
                      int stages, uint32_t b_region, uint32_t tmem_cols,
@@ -159,13 +185,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const uint32_t stage_bytes = kTileABytes + b_region;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes);
-  uint64_t* empty = full + kMaxStages;
-  uint64_t* acc_full = empty + kMaxStages;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* drain = acc_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  NormSmemTail* tail = reinterpret_cast<NormSmemTail*>(smem + stages * stage_bytes);
+  uint64_t* full = tail->full;
+  uint64_t* empty = tail->empty;
+  volatile int* abort_flag = &tail->abort_flag;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -177,43 +200,46 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 4);  // MMA commit + one arrival per reduction warp
+      mbar_init(&empty[s], 1 + kEpiWarps);  // MMA commit + one arrival per epilogue warp
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 128);
-    mbar_init(drain, 1);
-    *abort_flag = 0;
+    mbar_init(&tail->acc_full, 1);
+    mbar_init(&tail->acc_empty, kEpiWarps * 32);
+    mbar_init(&tail->drain, 1);
+    mbar_init(&tail->half_ready, kTileM);
+    tail->abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, tmem_cols);
+    tmem_alloc(&tail->tmem_slot, tmem_cols);
     tmem_relinquish();
   }
-  if (!kGrouped && warp == 4 && lane == 0) {
+  if (!kGrouped && warp == kEpiWarps && lane == 0) {
     prefetch_tmap(&single.tm_w0);
     prefetch_tmap(&single.tm_a);
     prefetch_tmap(&single.tm_b);
     prefetch_tmap(&single.tm_g);
+    prefetch_tmap(&single.tm_glo);
   }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t tmem_base = tail->tmem_slot;
 
   UnitCursor<kGrouped> cur;
   cur.single = &single;
   cur.table = table;
   cur.nprob = nprob;
 
-  if (warp == 4) {
+  if (warp == kEpiWarps) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && u_begin < u_end) {
+    if (lane == 0) {
       const uint64_t pol_stream = policy_evict_first();
       const uint64_t pol_keep = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       long long issued = 0;
-      cur.start(u_begin);
+      bool waited = false;  // G' (written by the preceding kernel) is visible
+      if (u_begin < u_end) cur.start(u_begin);
       for (long long u = u_begin; u < u_end; ++u, ++cur.local) {
         cur.settle(u);
         const NormProblemDev* P = cur.P;
@@ -225,17 +251,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         uint8_t* sa = smem + stage * stage_bytes;
         uint8_t* sb = sa + kTileABytes;
-        mbar_arrive_expect_tx(&full[stage], P->stage_tx);
         if (kb < P->kb_w) {
+          mbar_arrive_expect_tx(&full[stage], P->stage_tx);
           tma_load_2d(sa, &P->tm_w0, &full[stage], kb * kBlockK, t * kTileM, pol_stream);
           for (int j = 0; j < P->nbox; ++j)
             tma_load_2d(sb + j * P->box_rows * 128, &P->tm_a, &full[stage], kb * kBlockK,
                         j * P->box_rows, pol_keep);
         } else {
-          const int kr = kb - P->kb_w;
+          if (!waited) {
+            grid_dependency_wait();
+            grid_dependency_trigger();
+            waited = true;
+          }
+          const bool lo = kb >= P->kb_w + P->kb_r;
+          const int kr = kb - P->kb_w - (lo ? P->kb_r : 0);
+          const CUtensorMap* gm = lo ? &P->tm_glo : &P->tm_g;
+          mbar_arrive_expect_tx(&full[stage], P->stage_tx);
           tma_load_2d(sa, &P->tm_b, &full[stage], kr * kBlockK, t * kTileM, pol_keep);
           for (int j = 0; j < P->nbox; ++j)
-            tma_load_2d(sb + j * P->box_rows * 128, &P->tm_g, &full[stage], kr * kBlockK,
+            tma_load_2d(sb + j * P->box_rows * 128, gm, &full[stage], kr * kBlockK,
                         j * P->box_rows, pol_keep);
         }
         ++issued;
@@ -244,13 +278,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           phase ^= 1u;
         }
       }
+      if (!waited) {
+        grid_dependency_wait();
+        grid_dependency_trigger();
+      }
       // Let every copy already issued land before the block can exit.
       const long long first = issued > stages ? issued - stages : 0;
       for (long long j = first; j < issued; ++j)
         mbar_wait(&full[j % stages], static_cast<uint32_t>((j / stages) & 1), kDrainTimeoutNs,
                   nullptr);
     }
-  } else if (warp == 5) {
+  } else if (warp == kEpiWarps + 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && u_begin < u_end) {
       int stage = 0;
@@ -264,7 +302,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const NormProblemDev* P = cur.P;
         const int kb0 = cur.kblock();
         const long long seg_end = min(u_end, u + (P->kb_tile - kb0));
-        if (!mbar_wait(acc_empty, acc_phase ^ 1u, timeout_ns, abort_flag)) {
+        if (!mbar_wait(&tail->acc_empty, acc_phase ^ 1u, timeout_ns, abort_flag)) {
           give_up(abort_flag);
           break;
         }
@@ -299,19 +337,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
         if (!ok) break;
-        umma_commit(acc_full);
+        umma_commit(&tail->acc_full);
         acc_phase ^= 1u;
       }
       if (issued_any) {
-        umma_commit(drain);
-        mbar_wait(drain, 0, kDrainTimeoutNs, nullptr);
+        umma_commit(&tail->drain);
+        mbar_wait(&tail->drain, 0, kDrainTimeoutNs, nullptr);
       }
     }
   } else {
-    // ------------------------------------------- ||W0_i||^2 + epilogue (warps 0-3)
-    const int row = threadIdx.x;  // TMEM lane == tile row
+    // ------------------------------------ ||W0_i||^2 + epilogue (warps 0-7)
+    // Thread (half h, row): TMEM lane `row`; half h of the row's 16-byte chunks
+    // of each W0 stage and half h of the accumulator's 32-column chunks.
+    const int half = warp / 4;
+    const int row = threadIdx.x & (kTileM - 1);
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     int stage = 0;
-    uint32_t phase = 0, acc_phase = 0;
+    uint32_t phase = 0, acc_phase = 0, seg_count = 0;
     if (u_begin < u_end) {
       cur.start(u_begin);
       long long u = u_begin;
@@ -321,8 +363,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const NormProblemDev* P = cur.P;
         const int t = cur.tile();
         const int kb0 = cur.kblock();
-        const long long seg_first = u;
         const long long seg_end = min(u_end, u + (P->kb_tile - kb0));
+        const int r = P->r;
+        const int grow = t * kTileM + row;
+        const bool valid = grow < P->d_out;
+        // this half's 32-column chunks of the accumulator
+        const int nchunks = (P->n0 + P->n1 + 31) / 32;
+        const int c_lo = half == 0 ? 0 : (nchunks + 1) / 2;
+        const int c_hi = half == 0 ? (nchunks + 1) / 2 : nchunks;
+        // Prefetch B_i for (up to kPrefetchChunks of) those columns while the
+        // MMAs of this segment run.
+        const uint16_t* brow = P->B + static_cast<size_t>(valid ? grow : 0) * r;
+        uint4 bq[kPrefetchChunks][4];
+#pragma unroll
+        for (int c = 0; c < kPrefetchChunks; ++c)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int col = (c_lo + c) * 32 + q * 8;
+            bq[c][q] = (valid && c_lo + c < c_hi && col < r)
+                           ? __ldg(reinterpret_cast<const uint4*>(brow + col))
+                           : make_uint4(0u, 0u, 0u, 0u);
+          }
         float ss = 0.f;
         int kb = kb0;
         for (; u < seg_end; ++u, ++cur.local, ++kb) {
@@ -335,8 +396,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint8_t* rowp = smem + stage * stage_bytes + row * 128;
             float part = 0.f;
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              part += sumsq_bf16x8(*reinterpret_cast<const uint4*>(rowp + ((q ^ (row & 7)) << 4)));
+            for (int q = 0; q < 4; ++q)
+              part += sumsq_bf16x8(
+                  *reinterpret_cast<const uint4*>(rowp + (((half * 4 + q) ^ (row & 7)) << 4)));
             ss += part;
           }
           __syncwarp();
@@ -347,41 +409,57 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
         if (!ok) break;
-        if (!mbar_wait(acc_full, acc_phase, timeout_ns, abort_flag)) {
+        if (!mbar_wait(&tail->acc_full, acc_phase, timeout_ns, abort_flag)) {
           give_up(abort_flag);
           break;
         }
         tc_fence_after_sync();
-        const int grow = t * kTileM + row;
-        const bool valid = grow < P->d_out;
-        const int r = P->r;
-        const uint16_t* brow = P->B + static_cast<size_t>(valid ? grow : 0) * r;
-        const int ncols = P->n0 + P->n1;
         float dot = 0.f;
-        for (int col = 0; col < ncols; col += 32) {
-          float acc[32];
-          tmem_load_32cols(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + col, acc);
-          if (valid) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int cc = col + q * 8;
-              if (cc < r) {
-                const uint4 bv = __ldg(reinterpret_cast<const uint4*>(brow + cc));
-                dot += dot_bf16x8(acc + q * 8, bv);
+        for (int c = 0; c < kMaxChunksPerHalf; ++c) {
+          if (c_lo + c < c_hi) {  // warp-uniform
+            float acc[32];
+            tmem_load_32cols(tmem_base + lane_base + (c_lo + c) * 32, acc);
+            if (c < kPrefetchChunks) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) dot += dot_bf16x8(acc + q * 8, bq[c < kPrefetchChunks ? c : 0][q]);
+            } else {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int col = (c_lo + c) * 32 + q * 8;
+                if (valid && col < r)
+                  dot += dot_bf16x8(acc + q * 8, __ldg(reinterpret_cast<const uint4*>(brow + col)));
               }
             }
           }
         }
         tc_fence_before_sync();
-        mbar_arrive(acc_empty);
         acc_phase ^= 1u;
-        if (valid) {
-          const long long x0 = P->unit_begin + static_cast<long long>(t) * P->kb_tile;
-          const int slot = cta - first_cta_of_unit(x0, total_units, C);
-          P->partial[(static_cast<size_t>(t) * P->seg_slots + slot) * kTileM + row] =
-              fmaf(P->two_s, dot, ss);
+        // Combine the two halves of the row in a fixed order (lower + upper).
+        // The lower half takes the upper half's value before it releases the
+        // accumulator, so the next segment cannot overwrite it early.
+        const float part = fmaf(P->two_s, dot, ss);
+        const int buf = seg_count & 1;
+        if (half == 1) {
+          tail->half_part[buf][row] = part;
+          mbar_arrive(&tail->half_ready);
+          mbar_arrive(&tail->acc_empty);
+        } else {
+          const bool got = mbar_wait(&tail->half_ready, seg_count & 1u, timeout_ns, abort_flag);
+          const float other = tail->half_part[buf][row];
+          mbar_arrive(&tail->acc_empty);
+          if (!got) {
+            give_up(abort_flag);
+            break;
+          }
+          if (valid) {
+            const long long x0 = P->unit_begin + static_cast<long long>(t) * P->kb_tile;
+            const int slot = cta - first_cta_of_unit(x0, total_units, C);
+            P->partial[(static_cast<size_t>(t) * P->seg_slots + slot) * kTileM + row] =
+                part + other;
+          }
         }
-        (void)seg_first;
+        ++seg_count;
       }
     }
   }
@@ -401,6 +479,8 @@ __global__ void __launch_bounds__(256)
     norm_finalize_kernel(const __grid_constant__ NormProblemDev single,
                          const NormProblemDev* __restrict__ table, long long total_units, int ctas,
                          float eps) {
+  grid_dependency_wait();
+  grid_dependency_trigger();
   const NormProblemDev* P = kGrouped ? &table[blockIdx.y] : &single;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= P->d_out) return;
@@ -479,6 +559,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tmem_alloc(tmem_slot, 128);
     tmem_relinquish();
   }
+  grid_dependency_wait();
+  grid_dependency_trigger();
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -569,12 +651,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
-// Sums the K splits of every tile pair in split order, scales by s/2, rounds
-// to bf16 and writes G'[i][j] (and the mirrored G'[j][i] off the diagonal).
+// Sums the K splits of every tile pair in split order, scales by s/2, splits
+// the fp32 value into bf16 hi + lo and writes G'[i][j] (and the mirrored
+// G'[j][i] off the diagonal).
 template <bool kGrouped>
 __global__ void __launch_bounds__(256)
     gram_reduce_kernel(const __grid_constant__ GramProblemDev single,
                        const GramProblemDev* __restrict__ table) {
+  grid_dependency_wait();
+  grid_dependency_trigger();
   const GramProblemDev* P = kGrouped ? &table[blockIdx.z] : &single;
   const int pair = blockIdx.y;
   if (pair >= P->pairs) return;
@@ -587,9 +672,15 @@ __global__ void __launch_bounds__(256)
   const float* src = P->partial + static_cast<size_t>(pair) * P->S * kTileM * kTileM + e;
   float sum = 0.f;
   for (int s = 0; s < P->S; ++s) sum += src[static_cast<size_t>(s) * kTileM * kTileM];
-  const uint16_t v = f32_to_bf16_rn(P->half_s * sum);
-  P->g_out[static_cast<size_t>(gi) * P->r8 + gj] = v;
-  if (ta != tb) P->g_out[static_cast<size_t>(gj) * P->r8 + gi] = v;
+  const float x = P->half_s * sum;
+  const uint16_t hi = f32_to_bf16_rn(x);
+  const uint16_t lo = f32_to_bf16_rn(x - __uint_as_float(static_cast<uint32_t>(hi) << 16));
+  P->g_out[static_cast<size_t>(gi) * P->r8 + gj] = hi;
+  P->g_lo[static_cast<size_t>(gi) * P->r8 + gj] = lo;
+  if (ta != tb) {
+    P->g_out[static_cast<size_t>(gj) * P->r8 + gi] = hi;
+    P->g_lo[static_cast<size_t>(gj) * P->r8 + gi] = lo;
+  }
 }
 
 }  // namespace dora

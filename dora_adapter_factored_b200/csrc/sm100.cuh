@@ -67,6 +67,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
+// ---------------------------------------------------------------- PDL
+// Programmatic dependent launch: wait for the preceding grid (and, through
+// its own wait, everything before it) to complete and be visible; allow the
+// next grid to launch.  Every kernel of the library waits before it triggers.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {

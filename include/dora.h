@@ -163,6 +163,10 @@ dora_status_t dora_compose_bwd(const void *dy, const void *base, const void *lor
 dora_status_t dora_get_device_status(dora_stream_t stream);
 /* Static English description of a status code; never NULL. */
 const char *dora_status_string(dora_status_t status);
+/* Description of the last CUDA runtime failure seen by a call on the calling
+ * host thread (which call, the runtime's message and code), or "" if none.
+ * Owned by the library; valid until the next call on that thread. */
+const char *dora_last_error(void);
 /* Library version, major * 10000 + minor * 100 + patch. */
 int dora_version(void);
 /* Number of kernels this library has launched in this process. */
