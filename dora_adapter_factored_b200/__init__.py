@@ -10,7 +10,7 @@ from ._abi import (  # noqa: F401
     dora_compose_bwd, dora_compose_bwd_workspace_size, dora_debug_unsignalled_wait, dora_compose_fwd, dora_factored_norm,
     dora_factored_norm_grouped, dora_factored_norm_grouped_workspace_size,
     dora_factored_norm_workspace_size, dora_get_device_status, dora_launch_count,
-    dora_set_timing_events, dora_set_wait_timeout_ns, dora_version, load_library, status_string,
+    dora_set_timing_events, dora_set_trace_buffer, dora_set_wait_timeout_ns, dora_version, load_library, status_string,
 )
 
 __version__ = "0.1.0"

@@ -32,7 +32,7 @@ EXPORTED = (
     "dora_compose_fwd", "dora_compose_bwd_workspace_size", "dora_compose_bwd",
     "dora_get_device_status", "dora_status_string", "dora_version", "dora_launch_count",
     "dora_set_wait_timeout_ns", "dora_debug_unsignalled_wait", "dora_set_timing_events",
-    "dora_last_error",
+    "dora_last_error", "dora_set_trace_buffer",
 )
 
 
@@ -106,6 +106,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.dora_set_timing_events.restype = None
         lib.dora_last_error.argtypes = []
         lib.dora_last_error.restype = ctypes.c_char_p
+        lib.dora_set_trace_buffer.argtypes = [c_vp]
+        lib.dora_set_trace_buffer.restype = None
         _lib = lib
         return lib
 
@@ -180,6 +182,11 @@ def dora_set_timing_events(before: Optional[torch.cuda.Event], after: Optional[t
     principal kernel (see include/dora.h)."""
     load_library().dora_set_timing_events(before.cuda_event if before is not None else None,
                                           after.cuda_event if after is not None else None)
+
+
+def dora_set_trace_buffer(buf: Optional[torch.Tensor]) -> None:
+    """Diagnostics: per-CTA trace of the fused norm GEMM (see include/dora.h)."""
+    load_library().dora_set_trace_buffer(_dev(buf, "trace", torch.int64) if buf is not None else None)
 
 
 def dora_debug_unsignalled_wait(timeout_ns: int, stream=None) -> None:

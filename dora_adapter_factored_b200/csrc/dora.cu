@@ -31,6 +31,7 @@ std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
 
 // One-shot timing events around the principal kernel of the next call.
 thread_local cudaEvent_t t_ev_before = nullptr;
+unsigned long long* g_trace = nullptr;  // optional norm-kernel trace (diagnostics)
 thread_local cudaEvent_t t_ev_after = nullptr;
 
 struct TimedLaunch {
@@ -432,7 +433,7 @@ dora_status_t run_tc_group(const dora_norm_problem_t* probs, int count, bool gro
       TimedLaunch tl(st);
       launch_pdl(norm_main_kernel<false>, dim3(L.ctas), dim3(kNormThreads), L.smem_bytes, st,
                  nds[0], static_cast<const NormProblemDev*>(nullptr), 1, L.total_units, L.stages,
-                 L.b_region, static_cast<uint32_t>(L.tmem_cols), tmo);
+                 L.b_region, static_cast<uint32_t>(L.tmem_cols), tmo, g_trace);
       if ((s = launch_status()) != DORA_OK) return s;
     }
     launch_pdl(norm_finalize_kernel<false>, dim3(fin_x, 1), dim3(256), 0, st, nds[0],
@@ -457,7 +458,7 @@ dora_status_t run_tc_group(const dora_norm_problem_t* probs, int count, bool gro
     TimedLaunch tl(st);
     launch_pdl(norm_main_kernel<true>, dim3(L.ctas), dim3(kNormThreads), L.smem_bytes, st, nds[0],
                static_cast<const NormProblemDev*>(ntab), count, L.total_units, L.stages,
-               L.b_region, static_cast<uint32_t>(L.tmem_cols), tmo);
+               L.b_region, static_cast<uint32_t>(L.tmem_cols), tmo, g_trace);
     if ((s = launch_status()) != DORA_OK) return s;
   }
   launch_pdl(norm_finalize_kernel<true>, dim3(fin_x, count), dim3(256), 0, st, nds[0],
@@ -765,6 +766,8 @@ dora_status_t dora_debug_unsignalled_wait(uint64_t timeout_ns, dora_stream_t str
 uint64_t dora_launch_count(void) { return g_launches.load(); }
 
 const char* dora_last_error(void) { return t_last_error; }
+
+void dora_set_trace_buffer(void* buf) { g_trace = static_cast<unsigned long long*>(buf); }
 
 void dora_set_timing_events(void* before, void* after) {
   t_ev_before = static_cast<cudaEvent_t>(before);

@@ -44,6 +44,7 @@ constexpr int kPrefetchChunks = 6;           // of which B is prefetched into re
 // Registers are granted to a block in groups of four warps, so the 10-warp
 // norm kernel is charged as 12 warps: 65536 / 384 threads = 170 -> 168.
 constexpr int kNormMaxRegs = 168;
+
 constexpr uint32_t kTileABytes = kTileM * kBlockK * 2;  // 16 KiB
 constexpr int kMaxDynSmem = 232448;          // 227 KiB opt-in per block on sm_100
 
@@ -181,7 +182,11 @@ __global__ void __maxnreg__(kNormMaxRegs)
     norm_main_kernel(const __grid_constant__ NormProblemDev single,
                      const NormProblemDev* __restrict__ table, int nprob, long long total_units,
                      int stages, uint32_t b_region, uint32_t tmem_cols,
-                     unsigned long long timeout_ns) {
+                     unsigned long long timeout_ns, unsigned long long* __restrict__ trace) {
+  // trace (optional, diagnostics): per CTA 8 words -- entry and exit global
+  // time, MMA-issuer cycles waiting for data / for the accumulator, issued
+  // k-blocks, segments, SM id.
+  const uint64_t t_entry = trace != nullptr ? global_timer_ns() : 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const uint32_t stage_bytes = kTileABytes + b_region;
@@ -254,6 +259,7 @@ __global__ void __maxnreg__(kNormMaxRegs)
         if (kb < P->kb_w) {
           mbar_arrive_expect_tx(&full[stage], P->stage_tx);
           tma_load_2d(sa, &P->tm_w0, &full[stage], kb * kBlockK, t * kTileM, pol_stream);
+
           for (int j = 0; j < P->nbox; ++j)
             tma_load_2d(sb + j * P->box_rows * 128, &P->tm_a, &full[stage], kb * kBlockK,
                         j * P->box_rows, pol_keep);
@@ -294,6 +300,7 @@ __global__ void __maxnreg__(kNormMaxRegs)
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool issued_any = false;
+      long long wait_data = 0, wait_acc = 0, nseg = 0, nkb = 0;
       cur.start(u_begin);
       long long u = u_begin;
       bool ok = true;
@@ -302,20 +309,26 @@ __global__ void __maxnreg__(kNormMaxRegs)
         const NormProblemDev* P = cur.P;
         const int kb0 = cur.kblock();
         const long long seg_end = min(u_end, u + (P->kb_tile - kb0));
+        const long long c0 = clock64();
         if (!mbar_wait(&tail->acc_empty, acc_phase ^ 1u, timeout_ns, abort_flag)) {
           give_up(abort_flag);
           break;
         }
+        wait_acc += clock64() - c0;
+        ++nseg;
         tc_fence_after_sync();
         const uint32_t idesc0 = P->idesc0, idesc1 = P->idesc1;
         const int n0 = P->n0, n1 = P->n1;
         bool first = true;
         for (; u < seg_end; ++u, ++cur.local) {
+          const long long c1 = clock64();
           if (!mbar_wait(&full[stage], phase, timeout_ns, abort_flag)) {
             give_up(abort_flag);
             ok = false;
             break;
           }
+          wait_data += clock64() - c1;
+          ++nkb;
           tc_fence_after_sync();
           const uint32_t a0 = smem_addr(smem + stage * stage_bytes);
           const uint32_t b0 = a0 + kTileABytes;
@@ -343,6 +356,13 @@ __global__ void __maxnreg__(kNormMaxRegs)
       if (issued_any) {
         umma_commit(&tail->drain);
         mbar_wait(&tail->drain, 0, kDrainTimeoutNs, nullptr);
+      }
+      if (trace != nullptr) {
+        unsigned long long* tr = trace + static_cast<size_t>(cta) * 8;
+        tr[2] = static_cast<unsigned long long>(wait_data);
+        tr[3] = static_cast<unsigned long long>(wait_acc);
+        tr[4] = static_cast<unsigned long long>(nkb);
+        tr[5] = static_cast<unsigned long long>(nseg);
       }
     }
   } else {
@@ -470,6 +490,14 @@ __global__ void __maxnreg__(kNormMaxRegs)
   if (warp == 0) {
     tc_fence_after_sync();
     tmem_dealloc(tmem_base, tmem_cols);
+  }
+  if (trace != nullptr && threadIdx.x == 0) {
+    unsigned long long* tr = trace + static_cast<size_t>(cta) * 8;
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    tr[0] = t_entry;
+    tr[1] = global_timer_ns();
+    tr[6] = smid;
   }
 }
 

@@ -184,6 +184,12 @@ void dora_set_wait_timeout_ns(uint64_t ns);
  * NULL clears the hook).  Lets a caller time that one kernel with CUDA events
  * on the stream it runs on. */
 void dora_set_timing_events(void *before, void *after);
+/* Diagnostics: when `buf` is non-NULL, later norm calls record 8 uint64 words
+ * per CTA of the fused norm GEMM into it (device memory, 8 * 148 words for
+ * one B200): entry and exit %globaltimer, cycles the MMA issuer waited for
+ * operands and for the accumulator, k-blocks issued, segments, SM id.  NULL
+ * turns it off.  The buffer must outlive every call made while it is set. */
+void dora_set_trace_buffer(void *buf);
 /* Launches one thread that waits, with the same bounded wait the
  * tensor-core pipelines use, on a barrier that nothing ever signals, giving
  * up after `timeout_ns` (clamped to [1 us, 1 s]).  The give-up is recorded as
