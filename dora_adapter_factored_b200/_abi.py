@@ -32,7 +32,7 @@ EXPORTED = (
     "dora_compose_fwd", "dora_compose_bwd_workspace_size", "dora_compose_bwd",
     "dora_get_device_status", "dora_status_string", "dora_version", "dora_launch_count",
     "dora_set_wait_timeout_ns", "dora_debug_unsignalled_wait", "dora_set_timing_events",
-    "dora_last_error", "dora_set_trace_buffer",
+    "dora_last_error", "dora_set_trace_buffer", "dora_compose_bwd_static",
 )
 
 
@@ -108,6 +108,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.dora_last_error.restype = ctypes.c_char_p
         lib.dora_set_trace_buffer.argtypes = [c_vp]
         lib.dora_set_trace_buffer.restype = None
+        lib.dora_compose_bwd_static.argtypes = [c_vp, c_vp, c_vp, c_vp, c_vp, c_f, c_f, c_i,
+                                                c_i64, c_i64, c_vp, c_vp, c_vp, c_vp]
+        lib.dora_compose_bwd_static.restype = c_i
         _lib = lib
         return lib
 
@@ -308,4 +311,28 @@ def dora_compose_bwd(dy: torch.Tensor, base: torch.Tensor, lora: torch.Tensor, m
         _dev(d_base, "d_base", dy.dtype, (T, d_out)), _dev(d_lora, "d_lora", dy.dtype, (T, d_out)),
         _dev(dm, "dm", torch.float32, (d_out,)), _dev(ws, "ws"), ws.numel() * ws.element_size(),
         _stream(stream)), "dora_compose_bwd")
+    return d_base, d_lora, dm
+
+
+def dora_compose_bwd_static(dy: torch.Tensor, base: torch.Tensor, lora: torch.Tensor,
+                            m: torch.Tensor, n: torch.Tensor, s: float, eps: float = 0.0,
+                            d_base: Optional[torch.Tensor] = None,
+                            d_lora: Optional[torch.Tensor] = None,
+                            dm: Optional[torch.Tensor] = None, stream=None):
+    """dora_compose_bwd without a workspace (the library's fixed scratch array;
+    see include/dora.h for its size limit and sharing rules).  Returns
+    (d_base, d_lora, dm)."""
+    lib = load_library()
+    dt = _dtype_code(dy)
+    T, d_out = dy.shape
+    dev = dy.device
+    d_base = torch.empty_like(dy) if d_base is None else d_base
+    d_lora = torch.empty_like(dy) if d_lora is None else d_lora
+    dm = torch.empty(d_out, dtype=torch.float32, device=dev) if dm is None else dm
+    _check(lib.dora_compose_bwd_static(
+        _dev(dy, "dy", dy.dtype), _dev(base, "base", dy.dtype, (T, d_out)),
+        _dev(lora, "lora", dy.dtype, (T, d_out)), _dev(m, "m", torch.float32, (d_out,)),
+        _dev(n, "n", torch.float32, (d_out,)), float(s), float(eps), dt, T, d_out,
+        _dev(d_base, "d_base", dy.dtype, (T, d_out)), _dev(d_lora, "d_lora", dy.dtype, (T, d_out)),
+        _dev(dm, "dm", torch.float32, (d_out,)), _stream(stream)), "dora_compose_bwd_static")
     return d_base, d_lora, dm

@@ -726,6 +726,73 @@ dora_status_t dora_compose_bwd(const void* dy, const void* base, const void* lor
   return launch_status();
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Compose backward without a caller-provided workspace.
+//
+// Some callers cannot hand the library a workspace: a plain C host program
+// that links libdora.so without any device allocator of its own, or a
+// latency-critical loop in which cudaMalloc is not allowed because it can
+// synchronise the whole device.  For them, the column-partial table of the
+// backward lives in a fixed array in device memory instead.  Every GPU that
+// loads this library holds the array (4 MiB) until the process exits.
+// ---------------------------------------------------------------------------
+namespace dora {
+namespace {
+constexpr size_t kStaticScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+// Device address of g_static_scratch on the current device, looked up once
+// per device (the name is only a host-side stand-in in host code).
+void* static_scratch_address() {
+  static void* addr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) {
+      note_error("cudaGetSymbolAddress(static scratch)", e);
+      return nullptr;
+    }
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+}  // namespace
+}  // namespace dora
+
+extern "C" dora_status_t dora_compose_bwd_static(const void* dy, const void* base,
+                                                 const void* lora, const float* m, const float* n,
+                                                 float s, float eps, dora_dtype_t dt, int64_t T,
+                                                 int64_t d_out, void* d_base, void* d_lora,
+                                                 float* dm, dora_stream_t stream) {
+  if (dt != DORA_F32 && dt != DORA_BF16) return DORA_ERR_INVALID_ARG;
+  if (T < 0 || d_out < 1) return DORA_ERR_INVALID_ARG;
+  const size_t need = dora_compose_bwd_workspace_size(T, d_out, dt);
+  if (need > kStaticScratchBytes) {
+    snprintf(t_last_error, sizeof(t_last_error),
+             "dora_compose_bwd_static: this shape needs %zu bytes of scratch; the built-in array "
+             "holds %zu (use dora_compose_bwd with a workspace)",
+             need, kStaticScratchBytes);
+    return DORA_ERR_UNSUPPORTED;
+  }
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return DORA_ERR_CUDA;
+  if (!di->supported) return DORA_ERR_UNSUPPORTED;
+  void* scratch = static_scratch_address();
+  if (scratch == nullptr) return DORA_ERR_CUDA;
+  // Every slot of the partial table the kernels read is written by the same
+  // call first, so nothing has to be cleared between calls.
+  return dora_compose_bwd(dy, base, lora, m, n, s, eps, dt, T, d_out, d_base, d_lora, dm,
+                          scratch, kStaticScratchBytes, stream);
+}
+
+extern "C" {
+
 dora_status_t dora_get_device_status(dora_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return DORA_ERR_CUDA;

@@ -155,6 +155,35 @@ dora_status_t dora_compose_bwd(const void *dy, const void *base, const void *lor
                                size_t ws_bytes, dora_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Compose backward without a workspace (no counterpart on the pages: it is
+ * an interface convenience, not part of the method).
+ *
+ * Some callers cannot pass the library a workspace: a plain C host program
+ * that links this library without a device allocator of its own, or a
+ * latency-critical loop in which cudaMalloc is not allowed because it can
+ * synchronise the whole device.  This call computes exactly what
+ * dora_compose_bwd computes, with the same arguments minus the workspace:
+ * the dm column partials live in a fixed 4 MiB array of device memory that
+ * every GPU which loads this library holds until the process exits.  It
+ * allocates nothing and calls no allocating routine.
+ *   - Shapes whose partial table exceeds 4 MiB (more than 1,048,576 floats,
+ *     see dora_compose_bwd_workspace_size) are rejected with
+ *     DORA_ERR_UNSUPPORTED before anything is launched; dora_last_error()
+ *     then says how much scratch the shape needs.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream
+ *     capture.
+ *   - All calls share the one array: calls that overlap on the GPU (other
+ *     streams, other host threads) race and give wrong results.  Nothing in
+ *     the array needs to start at zero: each call writes every slot it
+ *     reads before reading it.
+ * ---------------------------------------------------------------------- */
+dora_status_t dora_compose_bwd_static(const void *dy, const void *base, const void *lora,
+                                      const float *m, const float *n, float s, float eps,
+                                      dora_dtype_t dt, int64_t T, int64_t d_out, void *d_base,
+                                      void *d_lora, float *dm, dora_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Status and diagnostics
  * ---------------------------------------------------------------------- */
 /* Synchronises `stream`, returns the first error any kernel of this library
