@@ -34,13 +34,22 @@ thread_local cudaEvent_t t_ev_before = nullptr;
 unsigned long long* g_trace = nullptr;  // optional norm-kernel trace (diagnostics)
 thread_local cudaEvent_t t_ev_after = nullptr;
 
+// While the stream is being captured into a graph, the events become event
+// record nodes of the graph (so they time the kernel at each replay).
+cudaError_t record_timing_event(cudaEvent_t ev, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    return cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
+  return cudaEventRecord(ev, st);
+}
+
 struct TimedLaunch {
   cudaStream_t st;
   explicit TimedLaunch(cudaStream_t s) : st(s) {
-    if (t_ev_before != nullptr) cudaEventRecord(t_ev_before, st);
+    if (t_ev_before != nullptr) record_timing_event(t_ev_before, st);
   }
   ~TimedLaunch() {
-    if (t_ev_after != nullptr) cudaEventRecord(t_ev_after, st);
+    if (t_ev_after != nullptr) record_timing_event(t_ev_after, st);
     t_ev_before = t_ev_after = nullptr;
   }
 };

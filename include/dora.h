@@ -211,7 +211,9 @@ void dora_set_wait_timeout_ns(uint64_t ns);
  * compose kernel of the compose calls) on that call's stream; the hook then
  * clears itself.  Both are cudaEvent_t handles created by the caller (NULL,
  * NULL clears the hook).  Lets a caller time that one kernel with CUDA events
- * on the stream it runs on. */
+ * on the stream it runs on.  While that stream is being captured into a CUDA
+ * graph, the events are recorded as event-record nodes of the graph, so each
+ * replay re-records them around the kernel. */
 void dora_set_timing_events(void *before, void *after);
 /* Diagnostics: when `buf` is non-NULL, later norm calls record 8 uint64 words
  * per CTA of the fused norm GEMM into it (device memory, 8 * 148 words for
