@@ -168,6 +168,22 @@ PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
   return fn;
 }
 
+// Row-major bf16 matrix [nblk * blk_rows, cols] viewed as 3-D {cols, blk_rows,
+// nblk}, loaded as one box {box_cols, blk_rows, nblk} (128-byte swizzle).  The
+// caller guarantees nblk * blk_rows equals the matrix's row count.
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* ptr, uint64_t blk_rows, uint64_t nblk,
+                       uint64_t cols, uint64_t ld, uint32_t box_cols) {
+  auto enc = tmap_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {cols, blk_rows, nblk};
+  cuuint64_t strides[2] = {ld * 2, blk_rows * ld * 2};
+  cuuint32_t box[3] = {box_cols, static_cast<cuuint32_t>(blk_rows), static_cast<cuuint32_t>(nblk)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Row-major bf16 matrix [rows, cols] with `ld` elements per row, loaded in
 // boxes of box_cols x box_rows with 128-byte swizzle; out-of-range elements
 // read as zero.
@@ -341,10 +357,20 @@ bool fill_descriptors(const dora_norm_problem_t& pr, const ModulePlan& p, uint8_
   uint16_t* gprime_lo = gprime + static_cast<size_t>(p.n_pad) * p.r8;
   bool ok = true;
   ok &= make_tmap_bf16(&nd.tm_w0, pr.W0, pr.d_out, pr.d_in, pr.d_in, kBlockK, kTileM);
-  ok &= make_tmap_bf16(&nd.tm_a, pr.A, pr.r, pr.d_in, pr.d_in, kBlockK, p.box_rows);
+  // The N-side slab in one 3-D box when its chunks are equal and cover r
+  // exactly (no dimension of the view can then reach past the matrix).
+  const bool slab3d = p.nbox == 2 && p.n0 == p.n1 && 2 * p.n0 == pr.r;
+  nd.slab3d = slab3d ? 1 : 0;
+  if (slab3d) {
+    ok &= make_tmap_bf16_3d(&nd.tm_a, pr.A, p.n0, 2, pr.d_in, pr.d_in, kBlockK);
+    ok &= make_tmap_bf16_3d(&nd.tm_g, gprime, p.n0, 2, pr.r, p.r8, kBlockK);
+    ok &= make_tmap_bf16_3d(&nd.tm_glo, gprime_lo, p.n0, 2, pr.r, p.r8, kBlockK);
+  } else {
+    ok &= make_tmap_bf16(&nd.tm_a, pr.A, pr.r, pr.d_in, pr.d_in, kBlockK, p.box_rows);
+    ok &= make_tmap_bf16(&nd.tm_g, gprime, pr.r, pr.r, p.r8, kBlockK, p.box_rows);
+    ok &= make_tmap_bf16(&nd.tm_glo, gprime_lo, pr.r, pr.r, p.r8, kBlockK, p.box_rows);
+  }
   ok &= make_tmap_bf16(&nd.tm_b, pr.B, pr.d_out, pr.r, pr.r, kBlockK, kTileM);
-  ok &= make_tmap_bf16(&nd.tm_g, gprime, pr.r, pr.r, p.r8, kBlockK, p.box_rows);
-  ok &= make_tmap_bf16(&nd.tm_glo, gprime_lo, pr.r, pr.r, p.r8, kBlockK, p.box_rows);
   ok &= make_tmap_bf16(&gd.tm_a, pr.A, pr.r, pr.d_in, pr.d_in, kBlockK, kTileM);
   nd.B = static_cast<const uint16_t*>(pr.B);
   nd.partial = reinterpret_cast<float*>(ws_base + p.off_np);

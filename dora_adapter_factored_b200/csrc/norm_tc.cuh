@@ -67,6 +67,7 @@ struct alignas(64) NormProblemDev {
   int d_out, r;
   int n0, n1;            // N of the two accumulator chunks (n1 = 0: single chunk)
   int box_rows, nbox;    // N-side operand: boxes per stage and rows per box
+  int slab3d;            // tm_a / tm_g / tm_glo are 3-D {64, box_rows, nbox}: one box per slab
   int kb_w, kb_r, kb_tile, tiles, seg_slots;  // kb_tile = kb_w + 2 kb_r (hi, then lo)
   uint32_t stage_tx;     // bytes landing per stage
   uint32_t idesc0, idesc1;
@@ -260,9 +261,12 @@ __global__ void __maxnreg__(kNormMaxRegs)
           mbar_arrive_expect_tx(&full[stage], P->stage_tx);
           tma_load_2d(sa, &P->tm_w0, &full[stage], kb * kBlockK, t * kTileM, pol_stream);
 
-          for (int j = 0; j < P->nbox; ++j)
-            tma_load_2d(sb + j * P->box_rows * 128, &P->tm_a, &full[stage], kb * kBlockK,
-                        j * P->box_rows, pol_keep);
+          if (P->slab3d)
+            tma_load_3d(sb, &P->tm_a, &full[stage], kb * kBlockK, 0, 0, pol_keep);
+          else
+            for (int j = 0; j < P->nbox; ++j)
+              tma_load_2d(sb + j * P->box_rows * 128, &P->tm_a, &full[stage], kb * kBlockK,
+                          j * P->box_rows, pol_keep);
         } else {
           if (!waited) {
             grid_dependency_wait();
@@ -274,9 +278,12 @@ __global__ void __maxnreg__(kNormMaxRegs)
           const CUtensorMap* gm = lo ? &P->tm_glo : &P->tm_g;
           mbar_arrive_expect_tx(&full[stage], P->stage_tx);
           tma_load_2d(sa, &P->tm_b, &full[stage], kr * kBlockK, t * kTileM, pol_keep);
-          for (int j = 0; j < P->nbox; ++j)
-            tma_load_2d(sb + j * P->box_rows * 128, gm, &full[stage], kr * kBlockK,
-                        j * P->box_rows, pol_keep);
+          if (P->slab3d)
+            tma_load_3d(sb, gm, &full[stage], kr * kBlockK, 0, 0, pol_keep);
+          else
+            for (int j = 0; j < P->nbox; ++j)
+              tma_load_2d(sb + j * P->box_rows * 128, gm, &full[stage], kr * kBlockK,
+                          j * P->box_rows, pol_keep);
         }
         ++issued;
         if (++stage == stages) {
