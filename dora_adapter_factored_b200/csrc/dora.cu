@@ -212,7 +212,7 @@ struct ModulePlan {
   // Gram
   int r8, tiles_r, pairs, kb_gram, S;
   // workspace (relative offsets inside the module's region)
-  size_t off_g, off_gp, off_np, bytes;
+  size_t off_g, off_gp, off_np, off_cnt, bytes;
   int seg_slots;
 };
 
@@ -277,7 +277,6 @@ struct GroupLayout {
   size_t smem_bytes = 0;
   int gram_jobs = 0;
   int max_pairs = 0;
-  int max_d_out = 0;
   size_t table_bytes = 0;  // descriptor tables at the start of the workspace (grouped)
   size_t total_bytes = 0;
 };
@@ -293,7 +292,6 @@ bool layout_group(const int64_t* d_out, const int64_t* d_in, const int64_t* r, i
     L.tmem_cols = std::max(L.tmem_cols, L.plans[i].tmem_cols);
     L.gram_jobs += L.plans[i].pairs * L.plans[i].S;
     L.max_pairs = std::max(L.max_pairs, L.plans[i].pairs);
-    L.max_d_out = std::max(L.max_d_out, static_cast<int>(d_out[i]));
   }
   L.ctas = static_cast<int>(std::min<long long>(sms, L.total_units));
   if (L.ctas < 1) return false;
@@ -316,6 +314,8 @@ bool layout_group(const int64_t* d_out, const int64_t* d_in, const int64_t* r, i
     off += align_up(static_cast<size_t>(p.pairs) * p.S * kTileM * kTileM * 4, 256);
     p.off_np = off;
     off += align_up(static_cast<size_t>(p.tiles) * L.seg_slots * kTileM * 4, 256);
+    p.off_cnt = off;
+    off += align_up(static_cast<size_t>(p.tiles) * 4 * sizeof(int), 256);
   }
   L.total_bytes = off;
   return true;
@@ -374,6 +374,7 @@ bool fill_descriptors(const dora_norm_problem_t& pr, const ModulePlan& p, uint8_
   ok &= make_tmap_bf16(&gd.tm_a, pr.A, pr.r, pr.d_in, pr.d_in, kBlockK, kTileM);
   nd.B = static_cast<const uint16_t*>(pr.B);
   nd.partial = reinterpret_cast<float*>(ws_base + p.off_np);
+  nd.tile_cnt = reinterpret_cast<int*>(ws_base + p.off_cnt);
   nd.m = pr.m;
   nd.n_out = pr.n_out;
   nd.g_out = pr.g_out;
@@ -397,6 +398,8 @@ bool fill_descriptors(const dora_norm_problem_t& pr, const ModulePlan& p, uint8_
   gd.partial = reinterpret_cast<float*>(ws_base + p.off_gp);
   gd.g_out = gprime;
   gd.g_lo = gprime_lo;
+  gd.tile_cnt = nd.tile_cnt;
+  gd.cnt_len = p.tiles * 4;
   gd.r = static_cast<int>(pr.r);
   gd.r8 = p.r8;
   gd.kb = p.kb_gram;
@@ -455,7 +458,6 @@ dora_status_t run_tc_group(const dora_norm_problem_t* probs, int count, bool gro
   const unsigned long long tmo = g_timeout_ns.load();
   const int gram_smem = 1024 + kGramStages * kGramStageBytes + 256;
   dora_status_t s;
-  const unsigned fin_x = static_cast<unsigned>(ceil_div_ll(L.max_d_out, 256));
   const dim3 red_grid(kTileM * kTileM / 256, L.max_pairs, grouped ? count : 1);
   if (!grouped) {
     launch_pdl(gram_kernel<false>, dim3(L.gram_jobs), dim3(kTcThreads), gram_smem, st, gds[0],
@@ -468,12 +470,9 @@ dora_status_t run_tc_group(const dora_norm_problem_t* probs, int count, bool gro
       TimedLaunch tl(st);
       launch_pdl(norm_main_kernel<false>, dim3(L.ctas), dim3(kNormThreads), L.smem_bytes, st,
                  nds[0], static_cast<const NormProblemDev*>(nullptr), 1, L.total_units, L.stages,
-                 L.b_region, static_cast<uint32_t>(L.tmem_cols), tmo, g_trace);
-      if ((s = launch_status()) != DORA_OK) return s;
+                 L.b_region, static_cast<uint32_t>(L.tmem_cols), eps, tmo, g_trace);
+      return launch_status();
     }
-    launch_pdl(norm_finalize_kernel<false>, dim3(fin_x, 1), dim3(256), 0, st, nds[0],
-               static_cast<const NormProblemDev*>(nullptr), L.total_units, L.ctas, eps);
-    return launch_status();
   }
   NormProblemDev* ntab = reinterpret_cast<NormProblemDev*>(base);
   GramProblemDev* gtab =
@@ -493,12 +492,9 @@ dora_status_t run_tc_group(const dora_norm_problem_t* probs, int count, bool gro
     TimedLaunch tl(st);
     launch_pdl(norm_main_kernel<true>, dim3(L.ctas), dim3(kNormThreads), L.smem_bytes, st, nds[0],
                static_cast<const NormProblemDev*>(ntab), count, L.total_units, L.stages,
-               L.b_region, static_cast<uint32_t>(L.tmem_cols), tmo, g_trace);
-    if ((s = launch_status()) != DORA_OK) return s;
+               L.b_region, static_cast<uint32_t>(L.tmem_cols), eps, tmo, g_trace);
+    return launch_status();
   }
-  launch_pdl(norm_finalize_kernel<true>, dim3(fin_x, count), dim3(256), 0, st, nds[0],
-             static_cast<const NormProblemDev*>(ntab), L.total_units, L.ctas, eps);
-  return launch_status();
 }
 
 

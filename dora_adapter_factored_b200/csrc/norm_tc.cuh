@@ -11,7 +11,8 @@
 //                    bf16 matrices, G'_hi = bf16(G') and G'_lo = bf16(G' - G'_hi),
 //                    so that the Gram term keeps fp32-level accuracy (the pages'
 //                    norm accumulates in fp32 whatever the weight dtype);
-//                    mirrors the off-diagonal tiles.
+//                    mirrors the off-diagonal tiles; zeroes the norm GEMM's
+//                    arrival counters.
 //   norm_main_kernel one 128-row tile of W0 at a time, stream-K over the
 //                    (tile, k-block) sequence.  Per tile the accumulator in
 //                    TMEM collects  W0_tile A^T  (k-blocks over d_in) and then
@@ -23,8 +24,10 @@
 //                    half of a row's columns, with B_i prefetched into registers
 //                    while the MMAs run) drains TMEM, dots each row with B_i
 //                    and writes the per-row partial ||W0_i||^2_part +
-//                    2 s B_i.acc_i for its k-range.
-//   norm_finalize    n_i = sqrt(max(sum of partials, 0)) in a fixed order,
+//                    2 s B_i.acc_i for its k-range.  The segment that posts a
+//                    tile's partials last (an arrival counter per 32 rows)
+//                    finalises those rows: n_i = sqrt(max(sum of partials, 0))
+//                    with the partials summed in slot order, and
 //                    g_i = m_i / max(n_i, eps)  (section 4, precision bullet).
 #pragma once
 
@@ -60,6 +63,7 @@ struct alignas(64) NormProblemDev {
   CUtensorMap tm_glo;    // G'_lo [r, r],     box 64 x box_rows
   const uint16_t* B;     // bf16 bits of B, for the epilogue dot
   float* partial;        // [tiles * seg_slots][128] per-row partials
+  int* tile_cnt;         // [tiles * 4] segments posted per 32-row quarter of a tile
   const float* m;        // [d_out] or null
   float* n_out;          // [d_out]
   float* g_out;          // [d_out] or null
@@ -79,6 +83,8 @@ struct alignas(64) GramProblemDev {
   float* partial;        // [pairs * S][128 * 128]
   uint16_t* g_out;       // G'_hi [r][r8] bf16 bits
   uint16_t* g_lo;        // G'_lo [r][r8] bf16 bits
+  int* tile_cnt;         // the norm GEMM's arrival counters, zeroed by the reduce
+  int cnt_len;
   int r, r8, kb, tiles_r, pairs, S, job_begin;
   float half_s;
 };
@@ -182,7 +188,7 @@ template <bool kGrouped>
 __global__ void __maxnreg__(kNormMaxRegs)
     norm_main_kernel(const __grid_constant__ NormProblemDev single,
                      const NormProblemDev* __restrict__ table, int nprob, long long total_units,
-                     int stages, uint32_t b_region, uint32_t tmem_cols,
+                     int stages, uint32_t b_region, uint32_t tmem_cols, float eps,
                      unsigned long long timeout_ns, unsigned long long* __restrict__ trace) {
   // trace (optional, diagnostics): per CTA 8 words -- entry and exit global
   // time, MMA-issuer cycles waiting for data / for the accumulator, issued
@@ -381,6 +387,7 @@ __global__ void __maxnreg__(kNormMaxRegs)
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     int stage = 0;
     uint32_t phase = 0, acc_phase = 0, seg_count = 0;
+    bool dep_waited = false;
     if (u_begin < u_end) {
       cur.start(u_begin);
       long long u = u_begin;
@@ -472,18 +479,40 @@ __global__ void __maxnreg__(kNormMaxRegs)
           mbar_arrive(&tail->half_ready);
           mbar_arrive(&tail->acc_empty);
         } else {
-          const bool got = mbar_wait(&tail->half_ready, seg_count & 1u, timeout_ns, abort_flag);
+          const bool got_one =
+              mbar_wait(&tail->half_ready, seg_count & 1u, timeout_ns, abort_flag);
           const float other = tail->half_part[buf][row];
           mbar_arrive(&tail->acc_empty);
-          if (!got) {
+          if (!__all_sync(0xffffffffu, got_one)) {
             give_up(abort_flag);
             break;
           }
-          if (valid) {
-            const long long x0 = P->unit_begin + static_cast<long long>(t) * P->kb_tile;
-            const int slot = cta - first_cta_of_unit(x0, total_units, C);
-            P->partial[(static_cast<size_t>(t) * P->seg_slots + slot) * kTileM + row] =
-                part + other;
+          const long long x0 = P->unit_begin + static_cast<long long>(t) * P->kb_tile;
+          const int c0 = first_cta_of_unit(x0, total_units, C);
+          const int nseg = first_cta_of_unit(x0 + P->kb_tile - 1, total_units, C) - c0 + 1;
+          float* part_t = P->partial + static_cast<size_t>(t) * P->seg_slots * kTileM + row;
+          if (valid) part_t[static_cast<size_t>(cta - c0) * kTileM] = part + other;
+          // The last of the tile's segments to post its partials (per warp:
+          // 32 rows) sums every slot in slot order and writes n and g.
+          __threadfence();
+          __syncwarp();
+          if (!dep_waited) {  // the counters are zeroed by the preceding kernel
+            grid_dependency_wait();
+            dep_waited = true;
+          }
+          int prev = 0;
+          if (lane == 0) prev = atomicAdd(P->tile_cnt + t * 4 + warp, 1);
+          prev = __shfl_sync(0xffffffffu, prev, 0);
+          if (prev == nseg - 1) {
+            __threadfence();
+            if (valid) {
+              float sum = 0.f;
+              for (int c = 0; c < nseg; ++c) sum += __ldcg(part_t + static_cast<size_t>(c) * kTileM);
+              const float n = __fsqrt_rn(fmaxf(sum, 0.f));
+              P->n_out[grow] = n;
+              if (P->m != nullptr && P->g_out != nullptr)
+                P->g_out[grow] = __fdiv_rn(__ldg(P->m + grow), fmaxf(n, eps));
+            }
           }
         }
         ++seg_count;
@@ -506,29 +535,6 @@ __global__ void __maxnreg__(kNormMaxRegs)
     tr[1] = global_timer_ns();
     tr[6] = smid;
   }
-}
-
-// n_i = sqrt(max(sum_slots p_i, 0)) in slot order; g_i = m_i / max(n_i, eps).
-template <bool kGrouped>
-__global__ void __launch_bounds__(256)
-    norm_finalize_kernel(const __grid_constant__ NormProblemDev single,
-                         const NormProblemDev* __restrict__ table, long long total_units, int ctas,
-                         float eps) {
-  grid_dependency_wait();
-  grid_dependency_trigger();
-  const NormProblemDev* P = kGrouped ? &table[blockIdx.y] : &single;
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= P->d_out) return;
-  const int t = i / kTileM;
-  const long long x0 = P->unit_begin + static_cast<long long>(t) * P->kb_tile;
-  const int c0 = first_cta_of_unit(x0, total_units, ctas);
-  const int c1 = first_cta_of_unit(x0 + P->kb_tile - 1, total_units, ctas);
-  const float* part = P->partial + static_cast<size_t>(t) * P->seg_slots * kTileM + (i % kTileM);
-  float sum = 0.f;
-  for (int c = c0; c <= c1; ++c) sum += part[static_cast<size_t>(c - c0) * kTileM];
-  const float n = __fsqrt_rn(fmaxf(sum, 0.f));
-  P->n_out[i] = n;
-  if (P->m != nullptr && P->g_out != nullptr) P->g_out[i] = __fdiv_rn(P->m[i], fmaxf(n, eps));
 }
 
 // ---------------------------------------------------------------------------
@@ -696,6 +702,8 @@ __global__ void __launch_bounds__(256)
   grid_dependency_wait();
   grid_dependency_trigger();
   const GramProblemDev* P = kGrouped ? &table[blockIdx.z] : &single;
+  if (blockIdx.x == 0 && blockIdx.y == 0)
+    for (int k = threadIdx.x; k < P->cnt_len; k += blockDim.x) P->tile_cnt[k] = 0;
   const int pair = blockIdx.y;
   if (pair >= P->pairs) return;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;  // element of the 128x128 tile
