@@ -57,6 +57,9 @@ __all__ = [
     "magnitude_scale",
     "compose_fwd",
     "compose_bwd",
+    "compose_inner",
+    "compose_bwd_from_inner",
+    "compose_bwd_frozen",
     "dora_linear_forward",
     "merged_weight",
     "rows_dense_row_norm",
@@ -190,6 +193,36 @@ def compose_bwd(dy, base, lora, m, n, s: float, eps: float):
     d_lora = (g * s) * dy
     dm = np.sum(dy * (base + s * lora), axis=0) / nc
     return d_base, d_lora, dm
+
+
+# --------------------------------------------------------------------------
+# Training-forward second output and the backward variants  [ScalingDoRA,
+# section 4 "Tier 1: Fused Backward" and section 6]
+# --------------------------------------------------------------------------
+
+def compose_inner(base, lora, s: float) -> np.ndarray:
+    """inner = base + s lora, the second output of the dual-output training
+    forward: y = g * inner, so the backward's dm needs inner and dy only
+    [ScalingDoRA, section 4, tier 1: output and inner computed together]."""
+    return _f64(base) + s * _f64(lora)
+
+
+def compose_bwd_from_inner(dy, inner, m, n, s: float, eps: float):
+    """Gradients of y = g * inner (n detached) from dy and inner alone:
+    d_base = g dy, d_lora = g s dy, dm_j = sum_t dy_tj inner_tj / n_c,j
+    [ScalingDoRA, section 4, tier 1; section 3, backward kernel]."""
+    dy, inner = _f64(dy), _f64(inner)
+    g, _, nc = magnitude_scale(m, n, eps)
+    return g * dy, (g * s) * dy, np.sum(dy * inner, axis=0) / nc
+
+
+def compose_bwd_frozen(dy, m, n, s: float, eps: float):
+    """d_base = g dy and d_lora = g s dy with the magnitude frozen: no dm and
+    no inner [ScalingDoRA, section 4, tier 1 and section 6: with frozen
+    magnitude the inner tensor is skipped]."""
+    dy = _f64(dy)
+    g, _, _ = magnitude_scale(m, n, eps)
+    return g * dy, (g * s) * dy
 
 
 # --------------------------------------------------------------------------

@@ -281,6 +281,50 @@ def test_dm_is_linear_in_dy():
     np.testing.assert_allclose(c, 2 * a - 3 * b, rtol=1e-12, atol=1e-12)
 
 
+# ---------------------------------------------------------------- training variants
+
+def test_inner_worked_example_and_forward_relation():
+    # inner = base + s lora by hand; and y = g * inner (the forward is the
+    # magnitude scale applied to inner, whatever the split of y into base and
+    # correction).
+    inner = oracle.compose_inner(np.array([[1.0, 2.0]]), np.array([[3.0, 4.0]]), 0.5)
+    np.testing.assert_array_equal(inner, [[2.5, 4.0]])
+    rng = np.random.default_rng(12)
+    T, d_out, s, eps = 5, 4, 1.5, 1e-12
+    base = rng.standard_normal((T, d_out)); lora = rng.standard_normal((T, d_out))
+    n = rng.uniform(0.5, 2.0, d_out); m = rng.uniform(0.5, 2.0, d_out)
+    y = oracle.compose_fwd(base, lora, m, n, s, eps)
+    np.testing.assert_allclose(y, (m / n) * oracle.compose_inner(base, lora, s), rtol=1e-14)
+
+
+def test_backward_from_inner_matches_finite_differences():
+    # L(inner, m) = sum dy * g(m) * inner; dm by finite differences in m, and
+    # d_base / d_lora by finite differences of the full forward in base / lora.
+    rng = np.random.default_rng(13)
+    T, d_out, s, eps = 4, 5, 2.0, 1e-12
+    base = rng.standard_normal((T, d_out)); lora = rng.standard_normal((T, d_out))
+    dy = rng.standard_normal((T, d_out))
+    n = rng.uniform(0.5, 2.0, d_out); m = n * rng.uniform(0.9, 1.1, d_out)
+    inner = base + s * lora
+    d_base, d_lora, dm = oracle.compose_bwd_from_inner(dy, inner, m, n, s, eps)
+    L = lambda b, l, mm: float(np.sum(dy * oracle.compose_fwd(b, l, mm, n, s, eps)))
+    np.testing.assert_allclose(d_base, _fd(lambda b: L(b, lora, m), base), rtol=1e-7, atol=1e-9)
+    np.testing.assert_allclose(d_lora, _fd(lambda l: L(base, l, m), lora), rtol=1e-7, atol=1e-9)
+    np.testing.assert_allclose(dm, _fd(lambda mm: L(base, lora, mm), m), rtol=1e-7, atol=1e-9)
+
+
+def test_frozen_backward_matches_finite_differences():
+    rng = np.random.default_rng(14)
+    T, d_out, s, eps = 3, 4, 0.75, 1e-12
+    base = rng.standard_normal((T, d_out)); lora = rng.standard_normal((T, d_out))
+    dy = rng.standard_normal((T, d_out))
+    n = rng.uniform(0.5, 2.0, d_out); m = rng.uniform(0.5, 2.0, d_out)
+    d_base, d_lora = oracle.compose_bwd_frozen(dy, m, n, s, eps)
+    L = lambda b, l: float(np.sum(dy * oracle.compose_fwd(b, l, m, n, s, eps)))
+    np.testing.assert_allclose(d_base, _fd(lambda b: L(b, lora), base), rtol=1e-7, atol=1e-9)
+    np.testing.assert_allclose(d_lora, _fd(lambda l: L(base, l), lora), rtol=1e-7, atol=1e-9)
+
+
 # ---------------------------------------------------------------- planted mistakes
 
 def test_pins_catch_planted_mistakes():
