@@ -24,6 +24,7 @@ DORA_OK, DORA_ERR_INVALID_ARG, DORA_ERR_UNSUPPORTED, DORA_ERR_WORKSPACE, DORA_ER
 DORA_F32, DORA_BF16 = 0, 1
 DORA_MAX_RANK = 512
 DORA_MAX_GROUP = 1024
+DORA_MAX_COMPOSE_GROUP = 64
 
 # Symbols include/dora.h declares (the ABI test checks the library exports each).
 EXPORTED = (
@@ -33,6 +34,9 @@ EXPORTED = (
     "dora_get_device_status", "dora_status_string", "dora_version", "dora_launch_count",
     "dora_set_wait_timeout_ns", "dora_debug_unsignalled_wait", "dora_set_timing_events",
     "dora_last_error", "dora_set_trace_buffer", "dora_compose_bwd_static",
+    "dora_compose_fwd_train", "dora_compose_bwd_inner", "dora_compose_bwd_frozen",
+    "dora_compose_fwd_grouped", "dora_compose_bwd_grouped_workspace_size",
+    "dora_compose_bwd_grouped",
 )
 
 
@@ -50,6 +54,16 @@ class NormProblem(ctypes.Structure):
         ("W0", ctypes.c_void_p), ("A", ctypes.c_void_p), ("B", ctypes.c_void_p),
         ("m", ctypes.c_void_p), ("n_out", ctypes.c_void_p), ("g_out", ctypes.c_void_p),
         ("d_out", ctypes.c_int64), ("d_in", ctypes.c_int64), ("r", ctypes.c_int64),
+        ("s", ctypes.c_float),
+    ]
+
+
+class ComposeProblem(ctypes.Structure):
+    _fields_ = [
+        ("base", ctypes.c_void_p), ("lora", ctypes.c_void_p), ("inner", ctypes.c_void_p),
+        ("m", ctypes.c_void_p), ("n", ctypes.c_void_p), ("y", ctypes.c_void_p),
+        ("dy", ctypes.c_void_p), ("d_base", ctypes.c_void_p), ("d_lora", ctypes.c_void_p),
+        ("dm", ctypes.c_void_p), ("T", ctypes.c_int64), ("d_out", ctypes.c_int64),
         ("s", ctypes.c_float),
     ]
 
@@ -111,6 +125,22 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.dora_compose_bwd_static.argtypes = [c_vp, c_vp, c_vp, c_vp, c_vp, c_f, c_f, c_i,
                                                 c_i64, c_i64, c_vp, c_vp, c_vp, c_vp]
         lib.dora_compose_bwd_static.restype = c_i
+        lib.dora_compose_fwd_train.argtypes = [c_vp, c_vp, c_vp, c_vp, c_f, c_f, c_i, c_i64, c_i64,
+                                               c_vp, c_vp, c_vp]
+        lib.dora_compose_fwd_train.restype = c_i
+        lib.dora_compose_bwd_inner.argtypes = [c_vp, c_vp, c_vp, c_vp, c_f, c_f, c_i, c_i64, c_i64,
+                                               c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]
+        lib.dora_compose_bwd_inner.restype = c_i
+        lib.dora_compose_bwd_frozen.argtypes = [c_vp, c_vp, c_vp, c_f, c_f, c_i, c_i64, c_i64,
+                                                c_vp, c_vp, c_vp]
+        lib.dora_compose_bwd_frozen.restype = c_i
+        cp = ctypes.POINTER(ComposeProblem)
+        lib.dora_compose_fwd_grouped.argtypes = [cp, c_i, c_i, c_f, c_vp]
+        lib.dora_compose_fwd_grouped.restype = c_i
+        lib.dora_compose_bwd_grouped_workspace_size.argtypes = [cp, c_i, c_i]
+        lib.dora_compose_bwd_grouped_workspace_size.restype = c_sz
+        lib.dora_compose_bwd_grouped.argtypes = [cp, c_i, c_i, c_f, c_vp, c_sz, c_vp]
+        lib.dora_compose_bwd_grouped.restype = c_i
         _lib = lib
         return lib
 
@@ -336,3 +366,114 @@ def dora_compose_bwd_static(dy: torch.Tensor, base: torch.Tensor, lora: torch.Te
         _dev(d_base, "d_base", dy.dtype, (T, d_out)), _dev(d_lora, "d_lora", dy.dtype, (T, d_out)),
         _dev(dm, "dm", torch.float32, (d_out,)), _stream(stream)), "dora_compose_bwd_static")
     return d_base, d_lora, dm
+
+
+def dora_compose_fwd_train(base: torch.Tensor, lora: torch.Tensor, m: torch.Tensor,
+                           n: torch.Tensor, s: float, eps: float = 0.0,
+                           y: Optional[torch.Tensor] = None, inner: Optional[torch.Tensor] = None,
+                           stream=None):
+    """Training forward: returns (y, inner) with inner = base + s lora."""
+    lib = load_library()
+    dt = _dtype_code(base)
+    T, d_out = base.shape
+    y = torch.empty_like(base) if y is None else y
+    inner = torch.empty_like(base) if inner is None else inner
+    _check(lib.dora_compose_fwd_train(
+        _dev(base, "base", base.dtype), _dev(lora, "lora", base.dtype, (T, d_out)),
+        _dev(m, "m", torch.float32, (d_out,)), _dev(n, "n", torch.float32, (d_out,)), float(s),
+        float(eps), dt, T, d_out, _dev(y, "y", base.dtype, (T, d_out)),
+        _dev(inner, "inner", base.dtype, (T, d_out)), _stream(stream)), "dora_compose_fwd_train")
+    return y, inner
+
+
+def dora_compose_bwd_inner(dy: torch.Tensor, inner: torch.Tensor, m: torch.Tensor,
+                           n: torch.Tensor, s: float, eps: float = 0.0,
+                           d_base: Optional[torch.Tensor] = None,
+                           d_lora: Optional[torch.Tensor] = None,
+                           dm: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                           stream=None):
+    """Backward from inner = base + s lora.  Returns (d_base, d_lora, dm)."""
+    lib = load_library()
+    dt = _dtype_code(dy)
+    T, d_out = dy.shape
+    dev = dy.device
+    d_base = torch.empty_like(dy) if d_base is None else d_base
+    d_lora = torch.empty_like(dy) if d_lora is None else d_lora
+    dm = torch.empty(d_out, dtype=torch.float32, device=dev) if dm is None else dm
+    ws = _workspace(lib.dora_compose_bwd_workspace_size(T, d_out, dt), dev, ws)
+    _check(lib.dora_compose_bwd_inner(
+        _dev(dy, "dy", dy.dtype), _dev(inner, "inner", dy.dtype, (T, d_out)),
+        _dev(m, "m", torch.float32, (d_out,)), _dev(n, "n", torch.float32, (d_out,)), float(s),
+        float(eps), dt, T, d_out, _dev(d_base, "d_base", dy.dtype, (T, d_out)),
+        _dev(d_lora, "d_lora", dy.dtype, (T, d_out)), _dev(dm, "dm", torch.float32, (d_out,)),
+        _dev(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream)),
+        "dora_compose_bwd_inner")
+    return d_base, d_lora, dm
+
+
+def dora_compose_bwd_frozen(dy: torch.Tensor, m: torch.Tensor, n: torch.Tensor, s: float,
+                            eps: float = 0.0, d_base: Optional[torch.Tensor] = None,
+                            d_lora: Optional[torch.Tensor] = None, stream=None):
+    """Backward with the magnitude frozen.  Returns (d_base, d_lora)."""
+    lib = load_library()
+    dt = _dtype_code(dy)
+    T, d_out = dy.shape
+    d_base = torch.empty_like(dy) if d_base is None else d_base
+    d_lora = torch.empty_like(dy) if d_lora is None else d_lora
+    _check(lib.dora_compose_bwd_frozen(
+        _dev(dy, "dy", dy.dtype), _dev(m, "m", torch.float32, (d_out,)),
+        _dev(n, "n", torch.float32, (d_out,)), float(s), float(eps), dt, T, d_out,
+        _dev(d_base, "d_base", dy.dtype, (T, d_out)), _dev(d_lora, "d_lora", dy.dtype, (T, d_out)),
+        _stream(stream)), "dora_compose_bwd_frozen")
+    return d_base, d_lora
+
+
+_COMPOSE_ACT = ("base", "lora", "inner", "y", "dy", "d_base", "d_lora")
+
+
+def _compose_problems(items: Sequence[dict]):
+    """ComposeProblem array from dicts: any of base, lora, inner, y, dy,
+    d_base, d_lora ([T, d_out], one dtype), m, n, dm ([d_out] fp32), s."""
+    arr = (ComposeProblem * len(items))()
+    dtype = None
+    for i, p in enumerate(items):
+        ref = next(p[k] for k in _COMPOSE_ACT if p.get(k) is not None)
+        T, d_out = ref.shape
+        dtype = dtype or ref.dtype
+        for k in _COMPOSE_ACT:
+            setattr(arr[i], k, _dev(p.get(k), f"{k}[{i}]", dtype, (T, d_out)))
+        arr[i].m = _dev(p["m"], f"m[{i}]", torch.float32, (d_out,))
+        arr[i].n = _dev(p["n"], f"n[{i}]", torch.float32, (d_out,))
+        arr[i].dm = _dev(p.get("dm"), f"dm[{i}]", torch.float32, (d_out,))
+        arr[i].T, arr[i].d_out = T, d_out
+        arr[i].s = float(p["s"])
+    if dtype not in _DT:
+        raise TypeError(f"unsupported dtype {dtype}: the library takes float32 or bfloat16")
+    return arr, _DT[dtype]
+
+
+def dora_compose_fwd_grouped(items: Sequence[dict], eps: float = 0.0, stream=None) -> None:
+    """One launch over several modules (dicts with base, lora, m, n, s, y and
+    optionally inner), written in place."""
+    arr, dt = _compose_problems(items)
+    _check(load_library().dora_compose_fwd_grouped(arr, len(items), dt, float(eps),
+                                                   _stream(stream)), "dora_compose_fwd_grouped")
+
+
+def dora_compose_bwd_grouped_workspace_size(items: Sequence[dict]) -> int:
+    arr, dt = _compose_problems(items)
+    return int(load_library().dora_compose_bwd_grouped_workspace_size(arr, len(items), dt))
+
+
+def dora_compose_bwd_grouped(items: Sequence[dict], eps: float = 0.0,
+                             ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Backward of several modules (dicts with dy, m, n, s, d_base, d_lora and
+    dm plus inner, or base and lora; no dm: frozen magnitude), in place."""
+    lib = load_library()
+    arr, dt = _compose_problems(items)
+    need = lib.dora_compose_bwd_grouped_workspace_size(arr, len(items), dt)
+    dev = next(p[k] for k in _COMPOSE_ACT for p in items if p.get(k) is not None).device
+    ws = _workspace(need, dev, ws) if need > 0 else None
+    _check(lib.dora_compose_bwd_grouped(arr, len(items), dt, float(eps), _dev(ws, "ws"),
+                                        0 if ws is None else ws.numel() * ws.element_size(),
+                                        _stream(stream)), "dora_compose_bwd_grouped")

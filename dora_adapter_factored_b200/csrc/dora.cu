@@ -517,34 +517,74 @@ namespace dora {
 namespace {
 template <typename E, int VEC>
 void launch_fwd(bool small, int64_t rows, int64_t d_out, const void* base, const void* lora,
-                const float* m, const float* n, float s, float eps, void* y, cudaStream_t cs) {
+                const float* m, const float* n, float s, float eps, void* y, void* inner,
+                cudaStream_t cs) {
   const StreamGrid g = stream_grid(rows, static_cast<int>(d_out / VEC), kFwdRowUnroll);
   const dim3 grid(g.gx, g.gy), block(g.bx, g.by);
-  if (small)
-    launch_pdl(compose_fwd_kernel<E, VEC, uint32_t>, grid, block, 0, cs,
-               static_cast<const E*>(base), static_cast<const E*>(lora), m, n, s, eps,
-               static_cast<long long>(rows), (int)d_out, static_cast<E*>(y));
-  else
-    launch_pdl(compose_fwd_kernel<E, VEC, uint64_t>, grid, block, 0, cs,
-               static_cast<const E*>(base), static_cast<const E*>(lora), m, n, s, eps,
-               static_cast<long long>(rows), (int)d_out, static_cast<E*>(y));
+  const E* b = static_cast<const E*>(base);
+  const E* l = static_cast<const E*>(lora);
+  E* yo = static_cast<E*>(y);
+  E* io = static_cast<E*>(inner);
+  const long long R = rows;
+  const int D = static_cast<int>(d_out);
+  if (inner != nullptr) {
+    if (small)
+      launch_pdl(compose_fwd_kernel<E, VEC, uint32_t, true>, grid, block, 0, cs, b, l, m, n, s,
+                 eps, R, D, yo, io);
+    else
+      launch_pdl(compose_fwd_kernel<E, VEC, uint64_t, true>, grid, block, 0, cs, b, l, m, n, s,
+                 eps, R, D, yo, io);
+  } else {
+    if (small)
+      launch_pdl(compose_fwd_kernel<E, VEC, uint32_t, false>, grid, block, 0, cs, b, l, m, n, s,
+                 eps, R, D, yo, io);
+    else
+      launch_pdl(compose_fwd_kernel<E, VEC, uint64_t, false>, grid, block, 0, cs, b, l, m, n, s,
+                 eps, R, D, yo, io);
+  }
 }
 
-template <typename E, int VEC>
+template <typename E, int VEC, int kMode>
 void launch_bwd(bool small, const StreamGrid& g, int64_t rows, int64_t d_out, const void* dy,
-                const void* base, const void* lora, const float* m, const float* n, float s,
+                const void* x1, const void* x2, const float* m, const float* n, float s,
                 float eps, void* d_base, void* d_lora, float* partial, cudaStream_t cs) {
   const dim3 grid(g.gx, g.gy), block(g.bx, g.by);
+  const E* d = static_cast<const E*>(dy);
+  const E* a1 = static_cast<const E*>(x1);
+  const E* a2 = static_cast<const E*>(x2);
+  E* ob = static_cast<E*>(d_base);
+  E* ol = static_cast<E*>(d_lora);
+  const long long R = rows;
+  const int D = static_cast<int>(d_out);
   if (small)
-    launch_pdl(compose_bwd_kernel<E, VEC, uint32_t>, grid, block, 0, cs,
-               static_cast<const E*>(dy), static_cast<const E*>(base),
-               static_cast<const E*>(lora), m, n, s, eps, static_cast<long long>(rows),
-               (int)d_out, static_cast<E*>(d_base), static_cast<E*>(d_lora), partial);
+    launch_pdl(compose_bwd_kernel<E, VEC, uint32_t, kMode>, grid, block, 0, cs, d, a1, a2, m, n,
+               s, eps, R, D, ob, ol, partial);
   else
-    launch_pdl(compose_bwd_kernel<E, VEC, uint64_t>, grid, block, 0, cs,
-               static_cast<const E*>(dy), static_cast<const E*>(base),
-               static_cast<const E*>(lora), m, n, s, eps, static_cast<long long>(rows),
-               (int)d_out, static_cast<E*>(d_base), static_cast<E*>(d_lora), partial);
+    launch_pdl(compose_bwd_kernel<E, VEC, uint64_t, kMode>, grid, block, 0, cs, d, a1, a2, m, n,
+               s, eps, R, D, ob, ol, partial);
+}
+
+template <int kMode>
+void launch_bwd_dt(dora_dtype_t dt, int vec, bool small, const StreamGrid& g, int64_t rows,
+                   int64_t d_out, const void* dy, const void* x1, const void* x2, const float* m,
+                   const float* n, float s, float eps, void* d_base, void* d_lora,
+                   float* partial, cudaStream_t cs) {
+  using B16 = __nv_bfloat16;
+  if (dt == DORA_BF16) {
+    if (vec == 8)
+      launch_bwd<B16, 8, kMode>(small, g, rows, d_out, dy, x1, x2, m, n, s, eps, d_base, d_lora,
+                                partial, cs);
+    else
+      launch_bwd<B16, 1, kMode>(small, g, rows, d_out, dy, x1, x2, m, n, s, eps, d_base, d_lora,
+                                partial, cs);
+  } else {
+    if (vec == 4)
+      launch_bwd<float, 4, kMode>(small, g, rows, d_out, dy, x1, x2, m, n, s, eps, d_base,
+                                  d_lora, partial, cs);
+    else
+      launch_bwd<float, 1, kMode>(small, g, rows, d_out, dy, x1, x2, m, n, s, eps, d_base,
+                                  d_lora, partial, cs);
+  }
 }
 }  // namespace
 }  // namespace dora
@@ -637,63 +677,147 @@ dora_status_t dora_factored_norm_grouped(const dora_norm_problem_t* problems, in
                       reinterpret_cast<cudaStream_t>(stream));
 }
 
-dora_status_t dora_compose_fwd(const void* base, const void* lora, const float* m, const float* n,
+}  // extern "C"
+
+namespace {
+
+// Forward with an optional second output.  Validation, then one launch.
+dora_status_t compose_fwd_impl(const void* base, const void* lora, const float* m, const float* n,
                                float s, float eps, dora_dtype_t dt, int64_t T, int64_t d_out,
-                               void* y, dora_stream_t stream) {
+                               void* y, void* inner, bool want_inner, dora_stream_t stream) {
   if (dt != DORA_F32 && dt != DORA_BF16) return DORA_ERR_INVALID_ARG;
   if (T < 0 || d_out < 1) return DORA_ERR_INVALID_ARG;
   if (m == nullptr || n == nullptr) return DORA_ERR_INVALID_ARG;
   if (T > 0 && (base == nullptr || lora == nullptr || y == nullptr)) return DORA_ERR_INVALID_ARG;
+  if (want_inner && T > 0 && inner == nullptr) return DORA_ERR_INVALID_ARG;
   if (d_out > (1ll << 31) - 1) return DORA_ERR_UNSUPPORTED;
   if (!(eps >= 0.f)) return DORA_ERR_INVALID_ARG;
   const size_t es = dt == DORA_BF16 ? 2 : 4;
   const size_t nbytes = static_cast<size_t>(T) * d_out * es;
   if (y != base && overlaps(y, nbytes, base, nbytes)) return DORA_ERR_INVALID_ARG;
   if (overlaps(y, nbytes, lora, nbytes)) return DORA_ERR_INVALID_ARG;
+  if (want_inner) {
+    if (inner != lora && overlaps(inner, nbytes, lora, nbytes)) return DORA_ERR_INVALID_ARG;
+    if (overlaps(inner, nbytes, base, nbytes) || overlaps(inner, nbytes, y, nbytes))
+      return DORA_ERR_INVALID_ARG;
+  }
   const DeviceInfo* di = device_info();
   if (di == nullptr) return DORA_ERR_CUDA;
   if (!di->supported) return DORA_ERR_UNSUPPORTED;
   if (T == 0) return DORA_OK;
+  void* in_out = want_inner ? inner : nullptr;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   TimedLaunch tl(cs);
-  const bool al = aligned16(base) && aligned16(lora) && aligned16(y);
+  const bool al = aligned16(base) && aligned16(lora) && aligned16(y) &&
+                  (in_out == nullptr || aligned16(in_out));
   const bool small = static_cast<unsigned long long>(T) * static_cast<unsigned long long>(d_out) <
                      (1ull << 31);
   if (dt == DORA_BF16) {
     using B16 = __nv_bfloat16;
     if (al && d_out % 8 == 0)
-      launch_fwd<B16, 8>(small, T, d_out, base, lora, m, n, s, eps, y, cs);
+      launch_fwd<B16, 8>(small, T, d_out, base, lora, m, n, s, eps, y, in_out, cs);
     else
-      launch_fwd<B16, 1>(small, T, d_out, base, lora, m, n, s, eps, y, cs);
+      launch_fwd<B16, 1>(small, T, d_out, base, lora, m, n, s, eps, y, in_out, cs);
   } else {
     if (al && d_out % 4 == 0)
-      launch_fwd<float, 4>(small, T, d_out, base, lora, m, n, s, eps, y, cs);
+      launch_fwd<float, 4>(small, T, d_out, base, lora, m, n, s, eps, y, in_out, cs);
     else
-      launch_fwd<float, 1>(small, T, d_out, base, lora, m, n, s, eps, y, cs);
+      launch_fwd<float, 1>(small, T, d_out, base, lora, m, n, s, eps, y, in_out, cs);
   }
   return launch_status();
 }
 
-namespace {
 struct BwdShape {
   int vec;
   StreamGrid g;
 };
-BwdShape bwd_shape(int64_t T, int64_t d_out, dora_dtype_t dt, bool aligned) {
+BwdShape bwd_shape(int64_t T, int64_t d_out, dora_dtype_t dt, bool aligned, int unroll) {
   BwdShape b;
   const int v = dt == DORA_BF16 ? 8 : 4;
   b.vec = (aligned && d_out % v == 0) ? v : 1;
-  b.g = stream_grid(T, static_cast<int>(d_out / b.vec), kBwdRowUnroll);
+  b.g = stream_grid(T, static_cast<int>(d_out / b.vec), unroll);
   return b;
 }
+
+// The three backward variants after their own validation: x1 / x2 are base /
+// lora, inner / unused, or unused / unused.
+dora_status_t compose_bwd_impl(int mode, const void* dy, const void* x1, const void* x2,
+                               const float* m, const float* n, float s, float eps,
+                               dora_dtype_t dt, int64_t T, int64_t d_out, void* d_base,
+                               void* d_lora, float* dm, void* ws, size_t ws_bytes,
+                               dora_stream_t stream) {
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return DORA_ERR_CUDA;
+  if (!di->supported) return DORA_ERR_UNSUPPORTED;
+  if (mode == kBwdFrozen && T == 0) return DORA_OK;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const bool al = aligned16(dy) && (mode == kBwdFrozen || aligned16(x1)) &&
+                  (mode != kBwdFromBaseLora || aligned16(x2)) && aligned16(d_base) &&
+                  aligned16(d_lora);
+  const BwdShape b = bwd_shape(T, d_out, dt, al, bwd_row_unroll(mode));
+  float* partial = nullptr;
+  if (mode != kBwdFrozen) {
+    const size_t need = static_cast<size_t>(b.g.gy) * d_out * 4;
+    if (ws == nullptr || ws_bytes < need || !aligned256(ws)) return DORA_ERR_WORKSPACE;
+    partial = static_cast<float*>(ws);
+  }
+  const bool small = static_cast<unsigned long long>(T) * static_cast<unsigned long long>(d_out) <
+                     (1ull << 31);
+  dora_status_t st;
+  {
+    TimedLaunch tl(cs);
+    if (mode == kBwdFromBaseLora)
+      launch_bwd_dt<kBwdFromBaseLora>(dt, b.vec, small, b.g, T, d_out, dy, x1, x2, m, n, s, eps,
+                                      d_base, d_lora, partial, cs);
+    else if (mode == kBwdFromInner)
+      launch_bwd_dt<kBwdFromInner>(dt, b.vec, small, b.g, T, d_out, dy, x1, x2, m, n, s, eps,
+                                   d_base, d_lora, partial, cs);
+    else
+      launch_bwd_dt<kBwdFrozen>(dt, b.vec, small, b.g, T, d_out, dy, x1, x2, m, n, s, eps,
+                                d_base, d_lora, partial, cs);
+    st = launch_status();
+  }
+  if (st != DORA_OK || mode == kBwdFrozen) return st;
+  launch_pdl(colsum_finalize_kernel, dim3((unsigned)ceil_div_ll(d_out, 32)), dim3(32, 8), 0, cs,
+             static_cast<const float*>(partial), b.g.gy, (int)d_out, n, eps, dm);
+  return launch_status();
+}
+
+// Arguments shared by every backward variant.
+dora_status_t check_bwd_common(const float* m, const float* n, float eps, dora_dtype_t dt,
+                               int64_t T, int64_t d_out) {
+  if (dt != DORA_F32 && dt != DORA_BF16) return DORA_ERR_INVALID_ARG;
+  if (T < 0 || d_out < 1) return DORA_ERR_INVALID_ARG;
+  if (m == nullptr || n == nullptr) return DORA_ERR_INVALID_ARG;
+  if (d_out > (1ll << 31) - 1) return DORA_ERR_UNSUPPORTED;
+  if (!(eps >= 0.f)) return DORA_ERR_INVALID_ARG;
+  return DORA_OK;
+}
+
 }  // namespace
+
+extern "C" {
+
+dora_status_t dora_compose_fwd(const void* base, const void* lora, const float* m, const float* n,
+                               float s, float eps, dora_dtype_t dt, int64_t T, int64_t d_out,
+                               void* y, dora_stream_t stream) {
+  return compose_fwd_impl(base, lora, m, n, s, eps, dt, T, d_out, y, nullptr, false, stream);
+}
+
+dora_status_t dora_compose_fwd_train(const void* base, const void* lora, const float* m,
+                                     const float* n, float s, float eps, dora_dtype_t dt,
+                                     int64_t T, int64_t d_out, void* y, void* inner,
+                                     dora_stream_t stream) {
+  return compose_fwd_impl(base, lora, m, n, s, eps, dt, T, d_out, y, inner, true, stream);
+}
 
 size_t dora_compose_bwd_workspace_size(int64_t T, int64_t d_out, dora_dtype_t dt) {
   if (T < 0 || d_out < 1) return 0;
   // The chunk count does not depend on the vector width chosen at call time:
-  // take the larger of the two layouts.
-  const BwdShape a = bwd_shape(T, d_out, dt, true);
-  const BwdShape b = bwd_shape(T, d_out, dt, false);
+  // take the larger of the two layouts.  The variants that read fewer
+  // streams keep more rows in flight per thread, so they need no more.
+  const BwdShape a = bwd_shape(T, d_out, dt, true, kBwdRowUnroll);
+  const BwdShape b = bwd_shape(T, d_out, dt, false, kBwdRowUnroll);
   const int chunks = std::max(a.g.gy, b.g.gy);
   return align_up(static_cast<size_t>(chunks) * d_out * 4, 256);
 }
@@ -702,14 +826,12 @@ dora_status_t dora_compose_bwd(const void* dy, const void* base, const void* lor
                                const float* n, float s, float eps, dora_dtype_t dt, int64_t T,
                                int64_t d_out, void* d_base, void* d_lora, float* dm, void* ws,
                                size_t ws_bytes, dora_stream_t stream) {
-  if (dt != DORA_F32 && dt != DORA_BF16) return DORA_ERR_INVALID_ARG;
-  if (T < 0 || d_out < 1) return DORA_ERR_INVALID_ARG;
-  if (m == nullptr || n == nullptr || dm == nullptr) return DORA_ERR_INVALID_ARG;
+  dora_status_t c = check_bwd_common(m, n, eps, dt, T, d_out);
+  if (c != DORA_OK) return c;
+  if (dm == nullptr) return DORA_ERR_INVALID_ARG;
   if (T > 0 && (dy == nullptr || base == nullptr || lora == nullptr || d_base == nullptr ||
                 d_lora == nullptr))
     return DORA_ERR_INVALID_ARG;
-  if (d_out > (1ll << 31) - 1) return DORA_ERR_UNSUPPORTED;
-  if (!(eps >= 0.f)) return DORA_ERR_INVALID_ARG;
   const size_t es = dt == DORA_BF16 ? 2 : 4;
   const size_t nbytes = static_cast<size_t>(T) * d_out * es;
   const size_t vb = static_cast<size_t>(d_out) * 4;
@@ -719,41 +841,326 @@ dora_status_t dora_compose_bwd(const void* dy, const void* base, const void* lor
       overlaps(d_lora, nbytes, base, nbytes) || overlaps(d_lora, nbytes, lora, nbytes))
     return DORA_ERR_INVALID_ARG;
   if (overlaps(dm, vb, m, vb) || overlaps(dm, vb, n, vb)) return DORA_ERR_INVALID_ARG;
+  return compose_bwd_impl(kBwdFromBaseLora, dy, base, lora, m, n, s, eps, dt, T, d_out, d_base,
+                          d_lora, dm, ws, ws_bytes, stream);
+}
+
+dora_status_t dora_compose_bwd_inner(const void* dy, const void* inner, const float* m,
+                                     const float* n, float s, float eps, dora_dtype_t dt,
+                                     int64_t T, int64_t d_out, void* d_base, void* d_lora,
+                                     float* dm, void* ws, size_t ws_bytes, dora_stream_t stream) {
+  dora_status_t c = check_bwd_common(m, n, eps, dt, T, d_out);
+  if (c != DORA_OK) return c;
+  if (dm == nullptr) return DORA_ERR_INVALID_ARG;
+  if (T > 0 && (dy == nullptr || inner == nullptr || d_base == nullptr || d_lora == nullptr))
+    return DORA_ERR_INVALID_ARG;
+  const size_t es = dt == DORA_BF16 ? 2 : 4;
+  const size_t nbytes = static_cast<size_t>(T) * d_out * es;
+  const size_t vb = static_cast<size_t>(d_out) * 4;
+  if (d_base != dy && overlaps(d_base, nbytes, dy, nbytes)) return DORA_ERR_INVALID_ARG;
+  if (overlaps(d_base, nbytes, inner, nbytes) || overlaps(d_base, nbytes, d_lora, nbytes) ||
+      overlaps(d_lora, nbytes, dy, nbytes) || overlaps(d_lora, nbytes, inner, nbytes))
+    return DORA_ERR_INVALID_ARG;
+  if (overlaps(dm, vb, m, vb) || overlaps(dm, vb, n, vb)) return DORA_ERR_INVALID_ARG;
+  return compose_bwd_impl(kBwdFromInner, dy, inner, nullptr, m, n, s, eps, dt, T, d_out, d_base,
+                          d_lora, dm, ws, ws_bytes, stream);
+}
+
+dora_status_t dora_compose_bwd_frozen(const void* dy, const float* m, const float* n, float s,
+                                      float eps, dora_dtype_t dt, int64_t T, int64_t d_out,
+                                      void* d_base, void* d_lora, dora_stream_t stream) {
+  dora_status_t c = check_bwd_common(m, n, eps, dt, T, d_out);
+  if (c != DORA_OK) return c;
+  if (T > 0 && (dy == nullptr || d_base == nullptr || d_lora == nullptr))
+    return DORA_ERR_INVALID_ARG;
+  const size_t es = dt == DORA_BF16 ? 2 : 4;
+  const size_t nbytes = static_cast<size_t>(T) * d_out * es;
+  if (d_base != dy && overlaps(d_base, nbytes, dy, nbytes)) return DORA_ERR_INVALID_ARG;
+  if (overlaps(d_base, nbytes, d_lora, nbytes) || overlaps(d_lora, nbytes, dy, nbytes))
+    return DORA_ERR_INVALID_ARG;
+  return compose_bwd_impl(kBwdFrozen, dy, nullptr, nullptr, m, n, s, eps, dt, T, d_out, d_base,
+                          d_lora, nullptr, nullptr, 0, stream);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Grouped compose: the modules of a layer in one launch.
+// ---------------------------------------------------------------------------
+namespace dora {
+namespace {
+static_assert(kMaxComposeGroup == DORA_MAX_COMPOSE_GROUP, "group capacity");
+
+struct ComposePlan {
+  ComposeGroup grp;
+  int blocks = 0, cblocks = 0;
+  bool small = true;
+  size_t ws_bytes = 0;
+};
+
+// Each module's grid is stream_grid() with its share of the launch's slots
+// (by activation elements); its dm partial table follows the previous
+// module's at a 256-byte boundary of the workspace.  Depends on the shapes,
+// the vector width and the variant only, so dm's summation order is fixed.
+void plan_compose_group(const dora_compose_problem_t* pr, int count, int vec, int unroll,
+                        bool partials, uint8_t* ws, float eps, ComposePlan& P) {
+  std::memset(&P.grp, 0, sizeof(P.grp));
+  P.grp.count = count;
+  P.grp.eps = eps;
+  double total = 0.0;
+  for (int p = 0; p < count; ++p) total += static_cast<double>(pr[p].T) * pr[p].d_out;
+  int blk = 0, cblk = 0;
+  size_t off = 0;
+  P.small = true;
+  for (int p = 0; p < count; ++p) {
+    ComposeItem& it = P.grp.it[p];
+    const double share = total > 0.0 ? static_cast<double>(pr[p].T) * pr[p].d_out / total : 0.0;
+    const long long slots = std::max(1ll, std::llround(kStreamSlots * share));
+    const StreamGrid g = stream_grid(pr[p].T, static_cast<int>(pr[p].d_out / vec), unroll, slots);
+    it.T = pr[p].T;
+    it.d_out = static_cast<int>(pr[p].d_out);
+    it.s = pr[p].s;
+    it.m = pr[p].m;
+    it.n = pr[p].n;
+    it.bx = g.bx;
+    it.gx = g.gx;
+    it.gy = g.gy;
+    it.blk_begin = blk;
+    it.cblk_begin = cblk;
+    blk += g.gx * g.gy;
+    cblk += static_cast<int>(ceil_div_ll(pr[p].d_out, 32));
+    if (partials) {
+      it.partial = ws != nullptr ? reinterpret_cast<float*>(ws + off) : nullptr;
+      off += align_up(static_cast<size_t>(g.gy) * pr[p].d_out * 4, 256);
+    }
+    if (static_cast<unsigned long long>(pr[p].T) * static_cast<unsigned long long>(pr[p].d_out) >=
+        (1ull << 31))
+      P.small = false;
+  }
+  P.blocks = blk;
+  P.cblocks = cblk;
+  P.ws_bytes = off;
+}
+
+// Backward variant of a record list, or -1 if the records disagree.  dm
+// (never empty) tells frozen from not; inner vs base and lora is read from the
+// records with T > 0 (an empty record reads nothing and may leave them NULL).
+int compose_group_mode(const dora_compose_problem_t* pr, int count) {
+  const bool frozen = pr[0].dm == nullptr;
+  for (int p = 1; p < count; ++p)
+    if ((pr[p].dm == nullptr) != frozen) return -1;
+  if (frozen) return kBwdFrozen;
+  int mode = -1;
+  for (int p = 0; p < count; ++p) {
+    if (pr[p].T == 0) continue;
+    const int mp = pr[p].inner != nullptr ? kBwdFromInner : kBwdFromBaseLora;
+    if (mode >= 0 && mp != mode) return -1;
+    mode = mp;
+  }
+  return mode >= 0 ? mode : kBwdFromBaseLora;
+}
+
+dora_status_t check_compose_record(const dora_compose_problem_t& q, dora_dtype_t dt, bool bwd,
+                                   int mode) {
+  if (q.T < 0 || q.d_out < 1) return DORA_ERR_INVALID_ARG;
+  if (q.d_out > (1ll << 31) - 1) return DORA_ERR_UNSUPPORTED;
+  if (q.m == nullptr || q.n == nullptr) return DORA_ERR_INVALID_ARG;
+  const size_t es = dt == DORA_BF16 ? 2 : 4;
+  const size_t nb = static_cast<size_t>(q.T) * q.d_out * es;
+  const size_t vb = static_cast<size_t>(q.d_out) * 4;
+  if (!bwd) {
+    if (q.T > 0 && (q.base == nullptr || q.lora == nullptr || q.y == nullptr))
+      return DORA_ERR_INVALID_ARG;
+    if (q.y != q.base && overlaps(q.y, nb, q.base, nb)) return DORA_ERR_INVALID_ARG;
+    if (overlaps(q.y, nb, q.lora, nb)) return DORA_ERR_INVALID_ARG;
+    if (q.inner != nullptr) {
+      if (q.inner != q.lora && overlaps(q.inner, nb, q.lora, nb)) return DORA_ERR_INVALID_ARG;
+      if (overlaps(q.inner, nb, q.base, nb) || overlaps(q.inner, nb, q.y, nb))
+        return DORA_ERR_INVALID_ARG;
+    }
+    return DORA_OK;
+  }
+  if (q.T > 0 && (q.dy == nullptr || q.d_base == nullptr || q.d_lora == nullptr))
+    return DORA_ERR_INVALID_ARG;
+  if (q.d_base != q.dy && overlaps(q.d_base, nb, q.dy, nb)) return DORA_ERR_INVALID_ARG;
+  if (overlaps(q.d_base, nb, q.d_lora, nb) || overlaps(q.d_lora, nb, q.dy, nb))
+    return DORA_ERR_INVALID_ARG;
+  if (mode == kBwdFrozen) return DORA_OK;
+  if (overlaps(q.dm, vb, q.m, vb) || overlaps(q.dm, vb, q.n, vb)) return DORA_ERR_INVALID_ARG;
+  // The streams this variant reads besides dy: inner, or base and lora.
+  const void* ins[2] = {mode == kBwdFromInner ? q.inner : q.base, q.lora};
+  const int nin = mode == kBwdFromInner ? 1 : 2;
+  for (int k = 0; k < nin; ++k) {
+    if (q.T > 0 && ins[k] == nullptr) return DORA_ERR_INVALID_ARG;
+    if (overlaps(q.d_base, nb, ins[k], nb) || overlaps(q.d_lora, nb, ins[k], nb))
+      return DORA_ERR_INVALID_ARG;
+  }
+  return DORA_OK;
+}
+
+// Vector width usable by every record of the group.
+int compose_group_vec(const dora_compose_problem_t* pr, int count, dora_dtype_t dt, bool bwd,
+                      int mode) {
+  const int v = dt == DORA_BF16 ? 8 : 4;
+  for (int p = 0; p < count; ++p) {
+    const dora_compose_problem_t& q = pr[p];
+    if (q.d_out % v != 0) return 1;
+    bool al;
+    if (!bwd)
+      al = aligned16(q.base) && aligned16(q.lora) && aligned16(q.y) &&
+           (q.inner == nullptr || aligned16(q.inner));
+    else
+      al = aligned16(q.dy) && aligned16(q.d_base) && aligned16(q.d_lora) &&
+           (mode != kBwdFromInner || aligned16(q.inner)) &&
+           (mode != kBwdFromBaseLora || (aligned16(q.base) && aligned16(q.lora)));
+    if (!al) return 1;
+  }
+  return v;
+}
+
+template <typename E, int VEC>
+void launch_fwd_grouped(const ComposePlan& P, cudaStream_t cs) {
+  if (P.small)
+    launch_pdl(compose_fwd_grouped_kernel<E, VEC, uint32_t>, dim3(P.blocks), dim3(kStreamThreads),
+               0, cs, P.grp);
+  else
+    launch_pdl(compose_fwd_grouped_kernel<E, VEC, uint64_t>, dim3(P.blocks), dim3(kStreamThreads),
+               0, cs, P.grp);
+}
+
+template <typename E, int VEC, int kMode>
+void launch_bwd_grouped(const ComposePlan& P, cudaStream_t cs) {
+  if (P.small)
+    launch_pdl(compose_bwd_grouped_kernel<E, VEC, uint32_t, kMode>, dim3(P.blocks),
+               dim3(kStreamThreads), 0, cs, P.grp);
+  else
+    launch_pdl(compose_bwd_grouped_kernel<E, VEC, uint64_t, kMode>, dim3(P.blocks),
+               dim3(kStreamThreads), 0, cs, P.grp);
+}
+
+template <int kMode>
+void launch_bwd_grouped_dt(dora_dtype_t dt, int vec, const ComposePlan& P, cudaStream_t cs) {
+  if (dt == DORA_BF16) {
+    if (vec == 8)
+      launch_bwd_grouped<__nv_bfloat16, 8, kMode>(P, cs);
+    else
+      launch_bwd_grouped<__nv_bfloat16, 1, kMode>(P, cs);
+  } else {
+    if (vec == 4)
+      launch_bwd_grouped<float, 4, kMode>(P, cs);
+    else
+      launch_bwd_grouped<float, 1, kMode>(P, cs);
+  }
+}
+}  // namespace
+}  // namespace dora
+
+extern "C" {
+
+dora_status_t dora_compose_fwd_grouped(const dora_compose_problem_t* problems, int count,
+                                       dora_dtype_t dt, float eps, dora_stream_t stream) {
+  if (dt != DORA_F32 && dt != DORA_BF16) return DORA_ERR_INVALID_ARG;
+  if (problems == nullptr || count < 1) return DORA_ERR_INVALID_ARG;
+  if (count > DORA_MAX_COMPOSE_GROUP) return DORA_ERR_UNSUPPORTED;
+  if (!(eps >= 0.f)) return DORA_ERR_INVALID_ARG;
+  for (int p = 0; p < count; ++p) {
+    const dora_status_t c = check_compose_record(problems[p], dt, false, 0);
+    if (c != DORA_OK) return c;
+  }
   const DeviceInfo* di = device_info();
   if (di == nullptr) return DORA_ERR_CUDA;
   if (!di->supported) return DORA_ERR_UNSUPPORTED;
+  const int vec = compose_group_vec(problems, count, dt, false, 0);
+  static thread_local ComposePlan P;
+  plan_compose_group(problems, count, vec, kFwdRowUnroll, false, nullptr, eps, P);
+  for (int p = 0; p < count; ++p) {
+    ComposeItem& it = P.grp.it[p];
+    it.in0 = problems[p].base;
+    it.in1 = problems[p].lora;
+    it.out0 = problems[p].y;
+    it.out1 = problems[p].inner;
+  }
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  const bool al = aligned16(dy) && aligned16(base) && aligned16(lora) && aligned16(d_base) &&
-                  aligned16(d_lora);
-  const BwdShape b = bwd_shape(T, d_out, dt, al);
-  const size_t need = static_cast<size_t>(b.g.gy) * d_out * 4;
-  if (ws == nullptr || ws_bytes < need || !aligned256(ws)) return DORA_ERR_WORKSPACE;
-  float* partial = static_cast<float*>(ws);
-  const bool small = static_cast<unsigned long long>(T) * static_cast<unsigned long long>(d_out) <
-                     (1ull << 31);
+  TimedLaunch tl(cs);
+  if (dt == DORA_BF16) {
+    if (vec == 8)
+      launch_fwd_grouped<__nv_bfloat16, 8>(P, cs);
+    else
+      launch_fwd_grouped<__nv_bfloat16, 1>(P, cs);
+  } else {
+    if (vec == 4)
+      launch_fwd_grouped<float, 4>(P, cs);
+    else
+      launch_fwd_grouped<float, 1>(P, cs);
+  }
+  return launch_status();
+}
+
+size_t dora_compose_bwd_grouped_workspace_size(const dora_compose_problem_t* problems, int count,
+                                               dora_dtype_t dt) {
+  if (problems == nullptr || count < 1 || count > DORA_MAX_COMPOSE_GROUP) return 0;
+  const int mode = compose_group_mode(problems, count);
+  if (mode < 0 || mode == kBwdFrozen) return 0;
+  for (int p = 0; p < count; ++p)
+    if (problems[p].T < 0 || problems[p].d_out < 1) return 0;
+  static thread_local ComposePlan P;
+  size_t best = 0;
+  for (int vec : {dt == DORA_BF16 ? 8 : 4, 1}) {
+    bool ok = true;
+    for (int p = 0; p < count; ++p) ok = ok && problems[p].d_out % vec == 0;
+    if (!ok) continue;
+    plan_compose_group(problems, count, vec, bwd_row_unroll(mode), true, nullptr, 0.f, P);
+    best = std::max(best, P.ws_bytes);
+  }
+  return best;
+}
+
+dora_status_t dora_compose_bwd_grouped(const dora_compose_problem_t* problems, int count,
+                                       dora_dtype_t dt, float eps, void* ws, size_t ws_bytes,
+                                       dora_stream_t stream) {
+  if (dt != DORA_F32 && dt != DORA_BF16) return DORA_ERR_INVALID_ARG;
+  if (problems == nullptr || count < 1) return DORA_ERR_INVALID_ARG;
+  if (count > DORA_MAX_COMPOSE_GROUP) return DORA_ERR_UNSUPPORTED;
+  if (!(eps >= 0.f)) return DORA_ERR_INVALID_ARG;
+  const int mode = compose_group_mode(problems, count);
+  if (mode < 0) return DORA_ERR_INVALID_ARG;
+  for (int p = 0; p < count; ++p) {
+    const dora_status_t c = check_compose_record(problems[p], dt, true, mode);
+    if (c != DORA_OK) return c;
+  }
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return DORA_ERR_CUDA;
+  if (!di->supported) return DORA_ERR_UNSUPPORTED;
+  const int vec = compose_group_vec(problems, count, dt, true, mode);
+  static thread_local ComposePlan P;
+  const bool partials = mode != kBwdFrozen;
+  plan_compose_group(problems, count, vec, bwd_row_unroll(mode), partials,
+                     static_cast<uint8_t*>(ws), eps, P);
+  if (partials && (ws == nullptr || ws_bytes < P.ws_bytes || !aligned256(ws)))
+    return DORA_ERR_WORKSPACE;
+  for (int p = 0; p < count; ++p) {
+    ComposeItem& it = P.grp.it[p];
+    it.in0 = problems[p].dy;
+    it.in1 = mode == kBwdFromInner ? problems[p].inner : problems[p].base;
+    it.in2 = mode == kBwdFromBaseLora ? problems[p].lora : nullptr;
+    it.out0 = problems[p].d_base;
+    it.out1 = problems[p].d_lora;
+    it.dm = problems[p].dm;
+  }
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   dora_status_t st;
   {
     TimedLaunch tl(cs);
-    if (dt == DORA_BF16) {
-      if (b.vec == 8)
-        launch_bwd<__nv_bfloat16, 8>(small, b.g, T, d_out, dy, base, lora, m, n, s, eps, d_base,
-                                     d_lora, partial, cs);
-      else
-        launch_bwd<__nv_bfloat16, 1>(small, b.g, T, d_out, dy, base, lora, m, n, s, eps, d_base,
-                                     d_lora, partial, cs);
-    } else {
-      if (b.vec == 4)
-        launch_bwd<float, 4>(small, b.g, T, d_out, dy, base, lora, m, n, s, eps, d_base, d_lora,
-                             partial, cs);
-      else
-        launch_bwd<float, 1>(small, b.g, T, d_out, dy, base, lora, m, n, s, eps, d_base, d_lora,
-                             partial, cs);
-    }
+    if (mode == kBwdFromBaseLora)
+      launch_bwd_grouped_dt<kBwdFromBaseLora>(dt, vec, P, cs);
+    else if (mode == kBwdFromInner)
+      launch_bwd_grouped_dt<kBwdFromInner>(dt, vec, P, cs);
+    else
+      launch_bwd_grouped_dt<kBwdFrozen>(dt, vec, P, cs);
     st = launch_status();
   }
-  if (st != DORA_OK) return st;
-  launch_pdl(colsum_finalize_kernel, dim3((unsigned)ceil_div_ll(d_out, 32)), dim3(32, 8), 0, cs,
-             static_cast<const float*>(partial), b.g.gy, (int)d_out, n, eps, dm);
+  if (st != DORA_OK || !partials) return st;
+  launch_pdl(colsum_grouped_kernel, dim3(P.cblocks), dim3(32, 8), 0, cs, P.grp);
   return launch_status();
 }
 

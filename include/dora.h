@@ -155,6 +155,100 @@ dora_status_t dora_compose_bwd(const void *dy, const void *base, const void *lor
                                size_t ws_bytes, dora_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Training forward with a second output  ["Scaling DoRA ...", section 4,
+ * tier 1: the dual-output kernel computes the output and `inner` together]
+ *
+ * Writes y exactly as dora_compose_fwd does and, in the same pass,
+ *   inner[t, j] = base[t, j] + s lora[t, j]
+ * in fp32, rounded once to `dt`.  inner is what the backward needs for dm
+ * (dora_compose_bwd_inner), so a training step can keep one activation
+ * tensor for the backward instead of base and lora.  y may equal base and
+ * inner may equal lora (same element, same thread); no other overlap.
+ * One pass: two reads and two writes per element.  T == 0 launches nothing.
+ * ---------------------------------------------------------------------- */
+dora_status_t dora_compose_fwd_train(const void *base, const void *lora, const float *m,
+                                     const float *n, float s, float eps, dora_dtype_t dt,
+                                     int64_t T, int64_t d_out, void *y, void *inner,
+                                     dora_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Backward from `inner`  ["Scaling DoRA ...", section 4, tier 1]
+ *
+ *   d_base = g dy,  d_lora = (g s) dy,  dm[j] = (sum_t dy[t, j] inner[t, j]) / n_c,j
+ * with inner = base + s lora from dora_compose_fwd_train.  Same fixed-order
+ * dm reduction as dora_compose_bwd.  Four passes per element (dy and inner
+ * read, d_base and d_lora written) instead of five.  d_base may equal dy.
+ * Workspace: dora_compose_bwd_workspace_size(T, d_out, dt) bytes (the same
+ * table as dora_compose_bwd, of which this call uses at most all).
+ * ---------------------------------------------------------------------- */
+dora_status_t dora_compose_bwd_inner(const void *dy, const void *inner, const float *m,
+                                     const float *n, float s, float eps, dora_dtype_t dt,
+                                     int64_t T, int64_t d_out, void *d_base, void *d_lora,
+                                     float *dm, void *ws, size_t ws_bytes,
+                                     dora_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Backward with the magnitude frozen  ["Scaling DoRA ...", section 4, tier
+ * 1 and section 6: with frozen magnitude the inner tensor is skipped]
+ *
+ *   d_base = g dy,  d_lora = (g s) dy;  no dm, no inner, no workspace.
+ * Three passes per element.  d_base may equal dy.  The forward of a
+ * frozen-magnitude step is dora_compose_fwd.
+ * ---------------------------------------------------------------------- */
+dora_status_t dora_compose_bwd_frozen(const void *dy, const float *m, const float *n, float s,
+                                      float eps, dora_dtype_t dt, int64_t T, int64_t d_out,
+                                      void *d_base, void *d_lora, dora_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Grouped compose  ["Scaling DoRA ...", section 6: below about 2048 x 6144
+ * activations launch latency dominates; one launch covers every module of a
+ * layer]
+ *
+ * One record per module (host array, read during the call only).  Every
+ * module is computed exactly as by the single-module call named below; the
+ * modules may differ in T, d_out and s, and share dt and eps.
+ *   forward  (dora_compose_fwd_grouped): base, lora, m, n, y; inner NULL, or
+ *            the second output of dora_compose_fwd_train.  One launch.
+ *   backward (dora_compose_bwd_grouped): dy, m, n, d_base, d_lora and
+ *            - dm NULL in every record: frozen magnitude
+ *              (dora_compose_bwd_frozen), no workspace;
+ *            - else inner non-NULL in every record: dora_compose_bwd_inner;
+ *            - else base and lora: dora_compose_bwd.
+ *            (Records with T == 0 read nothing and may leave inner, base
+ *            and lora NULL whatever the variant.)
+ *            Mixed records are DORA_ERR_INVALID_ARG.  Two launches (one when
+ *            frozen): the stream pass and one fixed-order dm reduction for
+ *            all modules.
+ * Aliasing inside a record as for the single-module calls; records must not
+ * write memory that another record reads or writes.  1 <= count <= 64.
+ * Workspace (backward): dora_compose_bwd_grouped_workspace_size() bytes,
+ * 256-byte aligned (0 for the frozen form).
+ * ---------------------------------------------------------------------- */
+#define DORA_MAX_COMPOSE_GROUP 64
+typedef struct {
+  const void *base;   /* [T, d_out] */
+  const void *lora;   /* [T, d_out] */
+  void *inner;        /* [T, d_out]: forward output (optional), backward input */
+  const float *m;     /* [d_out] */
+  const float *n;     /* [d_out] */
+  void *y;            /* [T, d_out] forward output */
+  const void *dy;     /* [T, d_out] backward input */
+  void *d_base;       /* [T, d_out] backward output */
+  void *d_lora;       /* [T, d_out] backward output */
+  float *dm;          /* [d_out] backward output; NULL = frozen magnitude */
+  int64_t T, d_out;
+  float s;
+} dora_compose_problem_t;
+
+dora_status_t dora_compose_fwd_grouped(const dora_compose_problem_t *problems, int count,
+                                       dora_dtype_t dt, float eps, dora_stream_t stream);
+size_t dora_compose_bwd_grouped_workspace_size(const dora_compose_problem_t *problems,
+                                               int count, dora_dtype_t dt);
+dora_status_t dora_compose_bwd_grouped(const dora_compose_problem_t *problems, int count,
+                                       dora_dtype_t dt, float eps, void *ws, size_t ws_bytes,
+                                       dora_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Compose backward without a workspace (no counterpart on the pages: it is
  * an interface convenience, not part of the method).
  *

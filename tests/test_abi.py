@@ -82,6 +82,59 @@ def test_host_validation_rejects_before_launch(built_library):
     assert dora.dora_launch_count() == before
 
 
+def test_training_and_grouped_validation(built_library):
+    lib = dora.load_library(built_library)
+    before = dora.dora_launch_count()
+    p = ctypes.c_void_p(0x10000)
+    vp = ctypes.c_void_p
+    # training forward: inner must be given, and may not overlap y
+    assert lib.dora_compose_fwd_train(p, vp(0x20000), p, p, 2.0, 0.0, _abi.DORA_BF16, 4, 8,
+                                      vp(0x30000), None, None) == _abi.DORA_ERR_INVALID_ARG
+    assert lib.dora_compose_fwd_train(p, vp(0x20000), p, p, 2.0, 0.0, _abi.DORA_BF16, 4, 8,
+                                      vp(0x30000), vp(0x30010), None) == _abi.DORA_ERR_INVALID_ARG
+    # backward from inner: d_lora aliasing inner; missing dm
+    assert lib.dora_compose_bwd_inner(p, vp(0x20000), p, p, 2.0, 0.0, _abi.DORA_BF16, 4, 8,
+                                      vp(0x40000), vp(0x20000), vp(0x50000), p, 1 << 20,
+                                      None) == _abi.DORA_ERR_INVALID_ARG
+    assert lib.dora_compose_bwd_inner(p, vp(0x20000), p, p, 2.0, 0.0, _abi.DORA_BF16, 4, 8,
+                                      vp(0x40000), vp(0x60000), None, p, 1 << 20,
+                                      None) == _abi.DORA_ERR_INVALID_ARG
+    # frozen backward: d_lora aliasing dy
+    assert lib.dora_compose_bwd_frozen(p, p, p, 2.0, 0.0, _abi.DORA_BF16, 4, 8, vp(0x40000), p,
+                                       None) == _abi.DORA_ERR_INVALID_ARG
+    # grouped: a record with dm next to one without (mixed variants)
+    arr = (_abi.ComposeProblem * 2)()
+    for i in range(2):
+        arr[i].dy, arr[i].d_base, arr[i].d_lora = 0x100000 * (i + 1), 0x110000 * (i + 1), \
+            0x120000 * (i + 1)
+        arr[i].m = arr[i].n = 0x10000
+        arr[i].T, arr[i].d_out, arr[i].s = 4, 8, 1.0
+    arr[0].dm, arr[0].inner = 0x900000, 0x910000
+    assert lib.dora_compose_bwd_grouped(arr, 2, _abi.DORA_BF16, 0.0, p, 1 << 20,
+                                        None) == _abi.DORA_ERR_INVALID_ARG
+    assert lib.dora_compose_bwd_grouped_workspace_size(arr, 2, _abi.DORA_BF16) == 0
+    big = (_abi.ComposeProblem * 65)()
+    assert lib.dora_compose_fwd_grouped(big, 65, _abi.DORA_BF16, 0.0,
+                                        None) == _abi.DORA_ERR_UNSUPPORTED
+    assert lib.dora_compose_fwd_grouped(arr, 0, _abi.DORA_BF16, 0.0,
+                                        None) == _abi.DORA_ERR_INVALID_ARG
+    assert dora.dora_launch_count() == before
+
+
+def test_grouped_workspace_sizes(built_library):
+    lib = dora.load_library(built_library)
+    arr = (_abi.ComposeProblem * 3)()
+    for i, (T, d) in enumerate([(512, 4096), (512, 1024), (7, 1000)]):
+        arr[i].dy = arr[i].base = arr[i].lora = arr[i].d_base = arr[i].d_lora = 0x10000
+        arr[i].m = arr[i].n = arr[i].dm = 0x10000
+        arr[i].T, arr[i].d_out, arr[i].s = T, d, 1.0
+    w = lib.dora_compose_bwd_grouped_workspace_size(arr, 3, _abi.DORA_BF16)
+    assert (4096 + 1024 + 1000) * 4 <= w < 64 << 20 and w % 256 == 0
+    for i in range(3):
+        arr[i].dm = None
+    assert lib.dora_compose_bwd_grouped_workspace_size(arr, 3, _abi.DORA_BF16) == 0
+
+
 def test_workspace_sizes_are_host_computable(built_library):
     lib = dora.load_library(built_library)
     # headline module: G' + Gram partials + norm partials, all modest
