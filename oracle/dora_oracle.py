@@ -62,6 +62,7 @@ __all__ = [
     "compose_bwd_frozen",
     "dora_linear_forward",
     "merged_weight",
+    "merge_weight_given_norm",
     "rows_dense_row_norm",
 ]
 
@@ -242,3 +243,12 @@ def dora_linear_forward(x, W0, A, B, m, s: float) -> np.ndarray:
     """y = x W'^T with the merged DoRA weight: the ``DoRALinear`` forward
     [DoRA-aiwiki]."""
     return _f64(x) @ merged_weight(W0, A, B, m, s).T
+
+
+def merge_weight_given_norm(W0, A, B, m, n, s: float, eps: float) -> np.ndarray:
+    """W' = g * (W0 + s B A) per output row with g = m / max(n, eps) for a
+    given row norm n: the merged inference weight [LoRA&DoRA, section 6],
+    with the magnitude scale of [ScalingDoRA, section 4 precision bullet]."""
+    W0, A, B = _f64(W0), _f64(A), _f64(B)
+    g, _, _ = magnitude_scale(m, n, eps)
+    return g[:, None] * (W0 + s * (B @ A))

@@ -325,6 +325,44 @@ def test_frozen_backward_matches_finite_differences():
     np.testing.assert_allclose(d_lora, _fd(lambda l: L(base, l), lora), rtol=1e-7, atol=1e-9)
 
 
+# ---------------------------------------------------------------- merged weight
+
+def test_merged_rows_have_the_magnitude_as_norm():
+    # With n the true row norm of W0 + sBA, every row of W' has norm m
+    # (numpy.linalg.norm), whatever the direction.
+    rng = np.random.default_rng(15)
+    W0, A, B = _rand_module(rng, 9, 7, 3)
+    m = rng.uniform(0.5, 2.0, 9)
+    n = np.linalg.norm(W0 + 2.0 * (B @ A), axis=1)
+    Wm = oracle.merge_weight_given_norm(W0, A, B, m, n, 2.0, 1e-12)
+    np.testing.assert_allclose(np.linalg.norm(Wm, axis=1), m, rtol=1e-13)
+    # ... and points along W0 + sBA (cosine 1 per row)
+    V = W0 + 2.0 * (B @ A)
+    cos = np.sum(Wm * V, axis=1) / (np.linalg.norm(Wm, axis=1) * np.linalg.norm(V, axis=1))
+    np.testing.assert_allclose(cos, 1.0, rtol=1e-13)
+
+
+def test_merged_init_is_w0_exactly():
+    # B = 0 and m = ||W0_i||: the merged weight is W0 (DoRA's initial weight).
+    rng = np.random.default_rng(16)
+    W0 = rng.standard_normal((6, 5)); A = rng.standard_normal((2, 5)); B = np.zeros((6, 2))
+    m = np.linalg.norm(W0, axis=1)
+    np.testing.assert_allclose(oracle.merge_weight_given_norm(W0, A, B, m, m, 3.0, 1e-12), W0,
+                               rtol=1e-15, atol=0)
+
+
+def test_merged_forward_equals_compose():
+    # x W'^T = compose(base = x W0^T, lora = x A^T B^T): merging is exact.
+    rng = np.random.default_rng(17)
+    d_out, d_in, r, T, s, eps = 7, 6, 3, 5, 1.5, 1e-12
+    W0, A, B = _rand_module(rng, d_out, d_in, r)
+    n = rng.uniform(0.5, 2.0, d_out); m = rng.uniform(0.5, 2.0, d_out)
+    x = rng.standard_normal((T, d_in))
+    y = x @ oracle.merge_weight_given_norm(W0, A, B, m, n, s, eps).T
+    ref = oracle.compose_fwd(x @ W0.T, (x @ A.T) @ B.T, m, n, s, eps)
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
 # ---------------------------------------------------------------- planted mistakes
 
 def test_pins_catch_planted_mistakes():
