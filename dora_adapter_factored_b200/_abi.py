@@ -36,7 +36,7 @@ EXPORTED = (
     "dora_last_error", "dora_set_trace_buffer", "dora_compose_bwd_static",
     "dora_compose_fwd_train", "dora_compose_bwd_inner", "dora_compose_bwd_frozen",
     "dora_compose_fwd_grouped", "dora_compose_bwd_grouped_workspace_size",
-    "dora_compose_bwd_grouped",
+    "dora_compose_bwd_grouped", "dora_merge_weight_workspace_size", "dora_merge_weight",
 )
 
 
@@ -141,6 +141,11 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.dora_compose_bwd_grouped_workspace_size.restype = c_sz
         lib.dora_compose_bwd_grouped.argtypes = [cp, c_i, c_i, c_f, c_vp, c_sz, c_vp]
         lib.dora_compose_bwd_grouped.restype = c_i
+        lib.dora_merge_weight_workspace_size.argtypes = [c_i64, c_i64, c_i64]
+        lib.dora_merge_weight_workspace_size.restype = c_sz
+        lib.dora_merge_weight.argtypes = [c_vp, c_vp, c_vp, c_vp, c_vp, c_f, c_f, c_i64, c_i64,
+                                          c_i64, c_vp, c_vp, c_sz, c_vp]
+        lib.dora_merge_weight.restype = c_i
         _lib = lib
         return lib
 
@@ -477,3 +482,27 @@ def dora_compose_bwd_grouped(items: Sequence[dict], eps: float = 0.0,
     _check(lib.dora_compose_bwd_grouped(arr, len(items), dt, float(eps), _dev(ws, "ws"),
                                         0 if ws is None else ws.numel() * ws.element_size(),
                                         _stream(stream)), "dora_compose_bwd_grouped")
+
+
+def dora_merge_weight_workspace_size(d_out: int, d_in: int, r: int) -> int:
+    return int(load_library().dora_merge_weight_workspace_size(d_out, d_in, r))
+
+
+def dora_merge_weight(W0: torch.Tensor, A: torch.Tensor, B: torch.Tensor, m: torch.Tensor,
+                      n: torch.Tensor, s: float, eps: float = 0.0,
+                      W_out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """W' = g (W0 + s B A), g = m / max(n, eps), bf16 [d_out, d_in].  W_out may
+    be W0 itself (in-place merge)."""
+    lib = load_library()
+    d_out, d_in = W0.shape
+    r = A.shape[0]
+    W_out = torch.empty_like(W0) if W_out is None else W_out
+    ws = _workspace(lib.dora_merge_weight_workspace_size(d_out, d_in, r), W0.device, ws)
+    _check(lib.dora_merge_weight(
+        _dev(W0, "W0", torch.bfloat16), _dev(A, "A", torch.bfloat16, (r, d_in)),
+        _dev(B, "B", torch.bfloat16, (d_out, r)), _dev(m, "m", torch.float32, (d_out,)),
+        _dev(n, "n", torch.float32, (d_out,)), float(s), float(eps), d_out, d_in, r,
+        _dev(W_out, "W_out", torch.bfloat16, (d_out, d_in)), _dev(ws, "ws"),
+        ws.numel() * ws.element_size(), _stream(stream)), "dora_merge_weight")
+    return W_out

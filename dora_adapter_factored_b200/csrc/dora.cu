@@ -16,6 +16,7 @@
 #include "dora.h"
 #include "common.cuh"
 #include "compose.cuh"
+#include "merge.cuh"
 #include "norm_simt.cuh"
 #include "norm_tc.cuh"
 
@@ -339,7 +340,9 @@ bool ensure_tc_attrs(int smem_norm) {
       (e = cudaFuncSetAttribute(gram_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 gram_smem)) != cudaSuccess ||
       (e = cudaFuncSetAttribute(gram_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                gram_smem)) != cudaSuccess) {
+                                gram_smem)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kMaxDynSmem)) != cudaSuccess) {
     note_error("cudaFuncSetAttribute", e);
     return false;
   }
@@ -880,6 +883,104 @@ dora_status_t dora_compose_bwd_frozen(const void* dy, const float* m, const floa
     return DORA_ERR_INVALID_ARG;
   return compose_bwd_impl(kBwdFrozen, dy, nullptr, nullptr, m, n, s, eps, dt, T, d_out, d_base,
                           d_lora, nullptr, nullptr, 0, stream);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Merged inference weight.
+// ---------------------------------------------------------------------------
+namespace dora {
+namespace {
+struct MergeLayout {
+  int kb, stages, tiles_m, tiles_n, r8;
+  size_t smem_bytes, ws_bytes;
+};
+
+bool merge_layout(int64_t d_out, int64_t d_in, int64_t r, MergeLayout& L) {
+  if (d_out < 1 || d_in < 1 || r < 1 || r > DORA_MAX_RANK) return false;
+  L.kb = static_cast<int>(ceil_div_ll(r, kMergeK));
+  L.r8 = round_up_int(static_cast<int>(r), 8);
+  L.tiles_m = static_cast<int>(ceil_div_ll(d_out, kMergeM));
+  L.tiles_n = static_cast<int>(ceil_div_ll(d_in, kMergeN));
+  const size_t tail = align_up(sizeof(MergeSmemTail), 128);
+  const size_t fixed = 1024 + 2 * kMergeTileBytes + static_cast<size_t>(L.kb) * kMergeOperandBytes + tail;
+  if (fixed + 2 * kMergeOperandBytes > static_cast<size_t>(kMaxDynSmem)) return false;
+  L.stages = static_cast<int>(std::min<size_t>(kMergeMaxStages,
+                                               (kMaxDynSmem - fixed) / kMergeOperandBytes));
+  L.smem_bytes = fixed + static_cast<size_t>(L.stages) * kMergeOperandBytes;
+  L.ws_bytes = align_up(static_cast<size_t>(d_in) * L.r8 * 2, 256);
+  return true;
+}
+}  // namespace
+}  // namespace dora
+
+extern "C" {
+
+size_t dora_merge_weight_workspace_size(int64_t d_out, int64_t d_in, int64_t r) {
+  MergeLayout L;
+  return merge_layout(d_out, d_in, r, L) ? L.ws_bytes : 0;
+}
+
+dora_status_t dora_merge_weight(const void* W0, const void* A, const void* B, const float* m,
+                                const float* n, float s, float eps, int64_t d_out, int64_t d_in,
+                                int64_t r, void* W_out, void* ws, size_t ws_bytes,
+                                dora_stream_t stream) {
+  if (W0 == nullptr || A == nullptr || B == nullptr || m == nullptr || n == nullptr ||
+      W_out == nullptr)
+    return DORA_ERR_INVALID_ARG;
+  if (d_out < 1 || d_in < 1 || r < 1) return DORA_ERR_INVALID_ARG;
+  if (!(eps >= 0.f)) return DORA_ERR_INVALID_ARG;
+  if (r > DORA_MAX_RANK || d_out > (1ll << 31) - 1 || d_in > (1ll << 31) - 1)
+    return DORA_ERR_UNSUPPORTED;
+  if (d_in % 8 != 0 || r % 8 != 0 || !aligned16(W0) || !aligned16(A) || !aligned16(B) ||
+      !aligned16(W_out))
+    return DORA_ERR_UNSUPPORTED;
+  const size_t wb = static_cast<size_t>(d_out) * d_in * 2;
+  if (W_out != W0 && overlaps(W_out, wb, W0, wb)) return DORA_ERR_INVALID_ARG;
+  if (overlaps(W_out, wb, A, static_cast<size_t>(r) * d_in * 2) ||
+      overlaps(W_out, wb, B, static_cast<size_t>(d_out) * r * 2) ||
+      overlaps(W_out, wb, m, d_out * 4) || overlaps(W_out, wb, n, d_out * 4))
+    return DORA_ERR_INVALID_ARG;
+  MergeLayout L;
+  if (!merge_layout(d_out, d_in, r, L)) return DORA_ERR_UNSUPPORTED;
+  if (ws == nullptr || ws_bytes < L.ws_bytes || !aligned256(ws)) return DORA_ERR_WORKSPACE;
+  if (overlaps(ws, L.ws_bytes, W_out, wb)) return DORA_ERR_INVALID_ARG;
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return DORA_ERR_CUDA;
+  if (!di->supported) return DORA_ERR_UNSUPPORTED;
+  if (!ensure_tc_attrs(0)) return DORA_ERR_CUDA;
+  static thread_local MergeDev P;
+  std::memset(&P, 0, sizeof(P));
+  uint16_t* At = static_cast<uint16_t*>(ws);
+  bool ok = true;
+  ok &= make_tmap_bf16(&P.tm_w0, W0, d_out, d_in, d_in, 64, kMergeM);
+  ok &= make_tmap_bf16(&P.tm_out, W_out, d_out, d_in, d_in, 64, kMergeM);
+  ok &= make_tmap_bf16(&P.tm_b, B, d_out, r, r, kMergeK, kMergeM);
+  ok &= make_tmap_bf16(&P.tm_at, At, d_in, r, L.r8, kMergeK, kMergeN);
+  if (!ok) return DORA_ERR_INVALID_ARG;
+  P.m = m;
+  P.n = n;
+  P.s = s;
+  P.eps = eps;
+  P.d_out = static_cast<int>(d_out);
+  P.d_in = static_cast<int>(d_in);
+  P.r = static_cast<int>(r);
+  P.kb = L.kb;
+  P.tiles_n = L.tiles_n;
+  P.tiles = L.tiles_m * L.tiles_n;
+  P.idesc = idesc_bf16_f32(kMergeM, kMergeN);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  launch_pdl(transpose_bf16_kernel, dim3((unsigned)ceil_div_ll(d_in, 32), (unsigned)ceil_div_ll(r, 32)),
+             dim3(32, 8), 0, cs, static_cast<const uint16_t*>(A), static_cast<int>(r),
+             static_cast<int>(d_in), At, L.r8);
+  dora_status_t st = launch_status();
+  if (st != DORA_OK) return st;
+  const int ctas = std::min(di->sms, P.tiles);
+  TimedLaunch tl(cs);
+  launch_pdl(merge_kernel, dim3(ctas), dim3(kMergeThreads), L.smem_bytes, cs, P, L.stages,
+             g_timeout_ns.load());
+  return launch_status();
 }
 
 }  // extern "C"

@@ -1,0 +1,358 @@
+// Merged DoRA weight W' = g (W0 + s B A), g = m / max(n, eps), for inference
+// without the adapter branch ("LoRA & DoRA: The Math, Memory, and
+// Trade-offs", section 6: the trained magnitude and direction fold into one
+// dense weight; "Scaling DoRA ...", section 4 precision bullet for g).  n is
+// the row norm the norm kernels produce; the merge does not recompute it.
+//
+// Two kernels:
+//   transpose_bf16_kernel  A [r, d_in] -> A^T [d_in, r8] in the workspace, so
+//                          that both MMA operands are K-major (K = r).
+//   merge_kernel           persistent, one CTA per SM over 128 x 128 tiles of
+//                          W' in row-major order.  Per tile the tensor cores
+//                          form acc = B_tile A^T_tile over K = r into one of two
+//                          TMEM accumulators (128 columns each); four epilogue
+//                          warps then read the W0 tile (staged by TMA into one
+//                          of two shared buffers), write g_i (W0_ij + s acc_ij)
+//                          rounded once to bf16 over it in place, and one thread
+//                          stores the tile with TMA.  The CTA keeps its row
+//                          block's B tile (128 x r) resident in shared memory
+//                          while it walks that block's column tiles, so only
+//                          A^T streams through the k-block stages.
+// HBM-bound: W0 is read once and W' written once (2 x 2 bytes per element);
+// the 2 d_out d_in r MMA FLOPs overlap with that traffic.
+#pragma once
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace dora {
+
+constexpr int kMergeM = 128;        // rows of W' per tile (TMEM lanes)
+constexpr int kMergeN = 128;        // columns of W' per tile (accumulator columns)
+constexpr int kMergeK = 64;         // r per k-block: one 128-byte swizzle row
+constexpr int kMergeThreads = 192;  // warps 0-3 epilogue, 4 TMA producer, 5 MMA issuer
+constexpr int kMergeMaxStages = 4;
+constexpr uint32_t kMergeOperandBytes = kMergeM * kMergeK * 2;  // 16 KiB: B or A^T k-block
+constexpr uint32_t kMergeTileBytes = kMergeM * kMergeN * 2;     // 32 KiB: W0 in, W' out
+constexpr uint32_t kMergeBoxBytes = kMergeM * 64 * 2;           // 16 KiB: one 64-column box
+
+struct alignas(64) MergeDev {
+  CUtensorMap tm_w0;   // W0 [d_out, d_in], box 64 x 128 (load)
+  CUtensorMap tm_out;  // W' [d_out, d_in], box 64 x 128 (store)
+  CUtensorMap tm_b;    // B  [d_out, r],    box 64 x 128
+  CUtensorMap tm_at;   // A^T [d_in, r],    box 64 x 128
+  const float* m;
+  const float* n;
+  float s, eps;
+  int d_out, d_in, r;
+  int kb;              // k-blocks over r
+  int tiles_n, tiles;  // column tiles per row block, all tiles
+  uint32_t idesc;
+};
+
+struct MergeSmemTail {
+  uint64_t full[kMergeMaxStages];   // A^T k-block landed
+  uint64_t empty[kMergeMaxStages];  // MMAs done with the k-block
+  uint64_t b_full, b_empty;         // resident B tile landed / no longer read
+  uint64_t w_full[2], w_empty[2];   // W0 tile landed / W' tile stored out of the buffer
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t epi_done[2];             // the four epilogue warps wrote the buffer
+  uint64_t drain;
+  uint32_t tmem_slot;
+  int abort_flag;
+};
+
+__device__ __forceinline__ void merge_give_up(volatile int* abort_flag) {
+  *abort_flag = 1;
+  record_error(DORA_ERR_TIMEOUT);
+}
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t x,
+                                             int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_addr(src)), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until the bulk stores committed so far have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_group0() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Makes this thread's generic-proxy shared-memory writes visible to TMA.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// At[j][k] = A[k][j]: 32 x 32 tiles through shared memory, block (32, 8).
+__global__ void __launch_bounds__(256)
+    transpose_bf16_kernel(const uint16_t* __restrict__ A, int rows, int cols,
+                          uint16_t* __restrict__ At, int ld_at) {
+  __shared__ uint16_t tile[32][33];
+  grid_dependency_wait();
+  grid_dependency_trigger();
+  const int x = blockIdx.x * 32 + threadIdx.x;  // column of A
+  const int y = blockIdx.y * 32 + threadIdx.y;  // row of A
+#pragma unroll
+  for (int j = 0; j < 32; j += 8)
+    if (x < cols && y + j < rows)
+      tile[threadIdx.y + j][threadIdx.x] = A[static_cast<size_t>(y + j) * cols + x];
+  __syncthreads();
+  const int tx = blockIdx.y * 32 + threadIdx.x;  // column of At (= row of A)
+  const int ty = blockIdx.x * 32 + threadIdx.y;  // row of At (= column of A)
+#pragma unroll
+  for (int j = 0; j < 32; j += 8)
+    if (tx < rows && ty + j < cols)
+      At[static_cast<size_t>(ty + j) * ld_at + tx] = tile[threadIdx.x][threadIdx.y + j];
+}
+
+__global__ void __launch_bounds__(kMergeThreads, 1)
+    merge_kernel(const __grid_constant__ MergeDev P, int stages, unsigned long long timeout_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* s_w = smem;                                        // 2 x 32 KiB W0 / W' tiles
+  uint8_t* s_b = s_w + 2 * kMergeTileBytes;                   // kb x 16 KiB resident B
+  uint8_t* s_at = s_b + P.kb * kMergeOperandBytes;            // stages x 16 KiB A^T
+  MergeSmemTail* tail =
+      reinterpret_cast<MergeSmemTail*>(s_at + stages * kMergeOperandBytes);
+  volatile int* abort_flag = &tail->abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int C = gridDim.x;
+  const int t_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * P.tiles / C);
+  const int t_end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * P.tiles / C);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&tail->full[s], 1);
+      mbar_init(&tail->empty[s], 1);
+    }
+    mbar_init(&tail->b_full, 1);
+    mbar_init(&tail->b_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tail->w_full[b], 1);
+      mbar_init(&tail->w_empty[b], 1);
+      mbar_init(&tail->acc_full[b], 1);
+      mbar_init(&tail->acc_empty[b], 4);
+      mbar_init(&tail->epi_done[b], 4);
+    }
+    mbar_init(&tail->drain, 1);
+    tail->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tail->tmem_slot, 2 * kMergeN);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tmap(&P.tm_w0);
+    prefetch_tmap(&P.tm_out);
+    prefetch_tmap(&P.tm_b);
+    prefetch_tmap(&P.tm_at);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = tail->tmem_slot;
+  // A^T is written by the transpose that precedes this kernel.
+  grid_dependency_wait();
+  grid_dependency_trigger();
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && t_begin < t_end) {
+      const uint64_t pol_stream = policy_evict_first();
+      const uint64_t pol_keep = policy_evict_last();
+      int stage = 0, cur_tm = -1, b_loads = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int t = t_begin, it = 0; ok && t < t_end; ++t, ++it) {
+        const int tm = t / P.tiles_n, tn = t % P.tiles_n;
+        if (tm != cur_tm) {
+          if (b_loads > 0 &&
+              !mbar_wait(&tail->b_empty, static_cast<uint32_t>((b_loads - 1) & 1), timeout_ns,
+                         abort_flag)) {
+            merge_give_up(abort_flag);
+            break;
+          }
+          mbar_arrive_expect_tx(&tail->b_full, P.kb * kMergeOperandBytes);
+          for (int k = 0; k < P.kb; ++k)
+            tma_load_2d(s_b + k * kMergeOperandBytes, &P.tm_b, &tail->b_full, k * kMergeK,
+                        tm * kMergeM, pol_keep);
+          cur_tm = tm;
+          ++b_loads;
+        }
+        const int wb = it & 1;
+        if (!mbar_wait(&tail->w_empty[wb], static_cast<uint32_t>(((it >> 1) & 1) ^ 1), timeout_ns,
+                       abort_flag)) {
+          merge_give_up(abort_flag);
+          break;
+        }
+        mbar_arrive_expect_tx(&tail->w_full[wb], kMergeTileBytes);
+        for (int h = 0; h < kMergeN / 64; ++h)
+          tma_load_2d(s_w + wb * kMergeTileBytes + h * kMergeBoxBytes, &P.tm_w0, &tail->w_full[wb],
+                      tn * kMergeN + h * 64, tm * kMergeM, pol_stream);
+        for (int k = 0; k < P.kb; ++k) {
+          if (!mbar_wait(&tail->empty[stage], phase ^ 1u, timeout_ns, abort_flag)) {
+            merge_give_up(abort_flag);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&tail->full[stage], kMergeOperandBytes);
+          tma_load_2d(s_at + stage * kMergeOperandBytes, &P.tm_at, &tail->full[stage],
+                      k * kMergeK, tn * kMergeN, pol_keep);
+          ++issued;
+          if (++stage == stages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Let every operand copy already issued land before the block can exit.
+      const long long first = issued > stages ? issued - stages : 0;
+      for (long long j = first; j < issued; ++j)
+        mbar_wait(&tail->full[j % stages], static_cast<uint32_t>((j / stages) & 1),
+                  kDrainTimeoutNs, nullptr);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && t_begin < t_end) {
+      int stage = 0, cur_tm = -1, b_loads = 0;
+      uint32_t phase = 0;
+      bool issued_any = false, ok = true;
+      for (int t = t_begin, it = 0; ok && t < t_end; ++t, ++it) {
+        const int tm = t / P.tiles_n;
+        if (tm != cur_tm) {
+          if (b_loads > 0) umma_commit(&tail->b_empty);  // previous row block's MMAs
+          if (!mbar_wait(&tail->b_full, static_cast<uint32_t>(b_loads & 1), timeout_ns,
+                         abort_flag)) {
+            merge_give_up(abort_flag);
+            break;
+          }
+          cur_tm = tm;
+          ++b_loads;
+        }
+        const int ab = it & 1;
+        if (!mbar_wait(&tail->acc_empty[ab], static_cast<uint32_t>(((it >> 1) & 1) ^ 1),
+                       timeout_ns, abort_flag)) {
+          merge_give_up(abort_flag);
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * kMergeN);
+        for (int k = 0; k < P.kb; ++k) {
+          if (!mbar_wait(&tail->full[stage], phase, timeout_ns, abort_flag)) {
+            merge_give_up(abort_flag);
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t a0 = smem_addr(s_b + k * kMergeOperandBytes);
+          const uint32_t b0 = smem_addr(s_at + stage * kMergeOperandBytes);
+#pragma unroll
+          for (int kk = 0; kk < kMergeK / 16; ++kk)
+            umma_bf16(d_tmem, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32),
+                      P.idesc, (k > 0 || kk > 0) ? 1u : 0u);
+          issued_any = true;
+          umma_commit(&tail->empty[stage]);
+          if (++stage == stages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tail->acc_full[ab]);
+      }
+      if (issued_any) {
+        umma_commit(&tail->drain);
+        mbar_wait(&tail->drain, 0, kDrainTimeoutNs, nullptr);
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue (warps 0-3)
+    // Thread = row of the tile = TMEM lane; per 32-column chunk it reads the
+    // accumulator, the row's W0 values from the 128-byte-swizzled staging
+    // buffer, and writes W' over them.
+    const int row = threadIdx.x;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    bool stored_any = false;
+    for (int t = t_begin, it = 0; t < t_end; ++t, ++it) {
+      const int tm = t / P.tiles_n, tn = t % P.tiles_n;
+      const int ab = it & 1;
+      const uint32_t par = static_cast<uint32_t>((it >> 1) & 1);
+      bool ok = mbar_wait(&tail->acc_full[ab], par, timeout_ns, abort_flag) &&
+                mbar_wait(&tail->w_full[ab], par, timeout_ns, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        merge_give_up(abort_flag);
+        break;
+      }
+      tc_fence_after_sync();
+      const int grow = tm * kMergeM + row;
+      float g = 0.f;
+      if (grow < P.d_out) g = __fdiv_rn(__ldg(P.m + grow), fmaxf(__ldg(P.n + grow), P.eps));
+      uint8_t* wtile = s_w + ab * kMergeTileBytes;
+#pragma unroll 1
+      for (int j = 0; j < kMergeN / 32; ++j) {
+        float acc[32];
+        __syncwarp();
+        tmem_load_32cols(tmem_base + lane_base + static_cast<uint32_t>(ab * kMergeN + j * 32), acc);
+        uint8_t* rowp = wtile + (j >> 1) * kMergeBoxBytes + row * 128;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int c = (j & 1) * 4 + q;  // 16-byte chunk of the 128-byte row
+          uint4* p = reinterpret_cast<uint4*>(rowp + ((c ^ (row & 7)) << 4));
+          const uint4 w = *p;
+          const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float lo = g * fmaf(P.s, acc[q * 8 + 2 * e], bf16lo_to_f32(wv[e]));
+            const float hi = g * fmaf(P.s, acc[q * 8 + 2 * e + 1], bf16hi_to_f32(wv[e]));
+            o[e] = pack_bf16x2_rn(lo, hi);
+          }
+          *p = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&tail->acc_empty[ab]);
+        mbar_arrive(&tail->epi_done[ab]);
+      }
+      if (threadIdx.x == 0) {
+        if (!mbar_wait(&tail->epi_done[ab], par, timeout_ns, abort_flag)) {
+          merge_give_up(abort_flag);
+        } else {
+          for (int h = 0; h < kMergeN / 64; ++h)
+            tma_store_2d(&P.tm_out, wtile + h * kMergeBoxBytes, tn * kMergeN + h * 64,
+                         tm * kMergeM);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+          stored_any = true;
+          mbar_arrive(&tail->w_empty[ab]);
+        }
+      }
+    }
+    if (threadIdx.x == 0 && stored_any) bulk_wait_group0();
+  }
+
+  __syncwarp();
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, 2 * kMergeN);
+  }
+}
+
+}  // namespace dora

@@ -249,6 +249,28 @@ dora_status_t dora_compose_bwd_grouped(const dora_compose_problem_t *problems, i
                                        dora_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Merged inference weight  ["LoRA & DoRA: The Math, Memory, and Trade-offs",
+ * section 6: magnitude and direction fold into one dense weight for
+ * inference; "Scaling DoRA ...", section 4 precision bullet for g]
+ *
+ *   W_out[i, j] = g_i (W0[i, j] + s sum_k B[i, k] A[k, j]),  g_i = m_i / max(n_i, eps)
+ * with the sum over k formed on the tensor cores in fp32 and the rest in fp32,
+ * rounded once to bf16.  n is the row norm of W0 + s B A (from
+ * dora_factored_norm); it is not recomputed.  W0, W_out: bf16 [d_out, d_in];
+ * A: bf16 [r, d_in]; B: bf16 [d_out, r]; m, n: fp32 [d_out].  W_out may
+ * equal W0 (in-place merge); no other overlap.  bf16 only; d_in and r
+ * multiples of 8, pointers 16-byte aligned, 1 <= r <= 512
+ * (DORA_ERR_UNSUPPORTED otherwise).  Workspace:
+ * dora_merge_weight_workspace_size() bytes, 256-byte aligned (holds A^T).
+ * Two launches (transpose of A, then the fused GEMM + epilogue).
+ * ---------------------------------------------------------------------- */
+size_t dora_merge_weight_workspace_size(int64_t d_out, int64_t d_in, int64_t r);
+dora_status_t dora_merge_weight(const void *W0, const void *A, const void *B, const float *m,
+                                const float *n, float s, float eps, int64_t d_out,
+                                int64_t d_in, int64_t r, void *W_out, void *ws,
+                                size_t ws_bytes, dora_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Compose backward without a workspace (no counterpart on the pages: it is
  * an interface convenience, not part of the method).
  *

@@ -121,6 +121,29 @@ def test_training_and_grouped_validation(built_library):
     assert dora.dora_launch_count() == before
 
 
+def test_merge_validation(built_library):
+    lib = dora.load_library(built_library)
+    before = dora.dora_launch_count()
+    vp = ctypes.c_void_p
+    W0, A, B, m, n, ws = (vp(0x100000), vp(0x200000), vp(0x300000), vp(0x400000),
+                          vp(0x500000), vp(0x600000))
+    out = vp(0x700000)
+    # r not a multiple of 8, d_in not a multiple of 8, rank above the limit
+    for d_in, r in ((64, 12), (60, 8), (64, 520)):
+        assert lib.dora_merge_weight(W0, A, B, m, n, 2.0, 0.0, 16, d_in, r, out, ws, 1 << 20,
+                                     None) == _abi.DORA_ERR_UNSUPPORTED
+    # W_out overlapping A; missing workspace; null m
+    assert lib.dora_merge_weight(W0, A, B, m, n, 2.0, 0.0, 16, 64, 8, vp(0x200010), ws, 1 << 20,
+                                 None) == _abi.DORA_ERR_INVALID_ARG
+    assert lib.dora_merge_weight(W0, A, B, m, n, 2.0, 0.0, 16, 64, 8, out, None, 0,
+                                 None) == _abi.DORA_ERR_WORKSPACE
+    assert lib.dora_merge_weight(W0, A, B, None, n, 2.0, 0.0, 16, 64, 8, out, ws, 1 << 20,
+                                 None) == _abi.DORA_ERR_INVALID_ARG
+    assert lib.dora_merge_weight_workspace_size(8192, 8192, 384) == 8192 * 384 * 2
+    assert lib.dora_merge_weight_workspace_size(8, 8, 600) == 0
+    assert dora.dora_launch_count() == before
+
+
 def test_grouped_workspace_sizes(built_library):
     lib = dora.load_library(built_library)
     arr = (_abi.ComposeProblem * 3)()
