@@ -149,15 +149,18 @@ def dist_setup(n_gpus: int):
 
 def barrier(pg, local):
     if pg is not None:
-        import torch
-        pg.barrier(device_ids=[local])
+        if pg.get_backend() == "nccl":
+            pg.barrier(device_ids=[local])
+        else:
+            pg.barrier()
 
 
 def max_over_ranks(pg, x: float) -> float:
     if pg is None:
         return x
     import torch
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if pg.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return float(t.item())
 

@@ -37,6 +37,7 @@ EXPORTED = (
     "dora_compose_fwd_train", "dora_compose_bwd_inner", "dora_compose_bwd_frozen",
     "dora_compose_fwd_grouped", "dora_compose_bwd_grouped_workspace_size",
     "dora_compose_bwd_grouped", "dora_merge_weight_workspace_size", "dora_merge_weight",
+    "dora_factored_norm_sq", "dora_norm_finalize",
 )
 
 
@@ -146,6 +147,11 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.dora_merge_weight.argtypes = [c_vp, c_vp, c_vp, c_vp, c_vp, c_f, c_f, c_i64, c_i64,
                                           c_i64, c_vp, c_vp, c_sz, c_vp]
         lib.dora_merge_weight.restype = c_i
+        lib.dora_factored_norm_sq.argtypes = [c_vp, c_vp, c_vp, c_i, c_i64, c_i64, c_i64, c_f,
+                                              c_vp, c_vp, c_sz, c_vp]
+        lib.dora_factored_norm_sq.restype = c_i
+        lib.dora_norm_finalize.argtypes = [c_vp, c_vp, c_f, c_i64, c_vp, c_vp, c_vp]
+        lib.dora_norm_finalize.restype = c_i
         _lib = lib
         return lib
 
@@ -506,3 +512,41 @@ def dora_merge_weight(W0: torch.Tensor, A: torch.Tensor, B: torch.Tensor, m: tor
         _dev(W_out, "W_out", torch.bfloat16, (d_out, d_in)), _dev(ws, "ws"),
         ws.numel() * ws.element_size(), _stream(stream)), "dora_merge_weight")
     return W_out
+
+
+def dora_factored_norm_sq(W0: torch.Tensor, A: torch.Tensor, B: torch.Tensor, s: float,
+                          sq_out: Optional[torch.Tensor] = None,
+                          ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Squared row-norm contribution of one column shard (W0[:, J], A[:, J],
+    whole B), fp32 [d_out], before any clamp or square root."""
+    lib = load_library()
+    dt = _dtype_code(W0)
+    d_out, d_in = W0.shape
+    r = A.shape[0]
+    dev = W0.device
+    sq_out = torch.empty(d_out, dtype=torch.float32, device=dev) if sq_out is None else sq_out
+    ws = _workspace(lib.dora_factored_norm_workspace_size(d_out, d_in, r, dt), dev, ws)
+    _check(lib.dora_factored_norm_sq(
+        _dev(W0, "W0", W0.dtype), _dev(A, "A", W0.dtype, (r, d_in)),
+        _dev(B, "B", W0.dtype, (d_out, r)), dt, d_out, d_in, r, float(s),
+        _dev(sq_out, "sq_out", torch.float32, (d_out,)), _dev(ws, "ws"),
+        ws.numel() * ws.element_size(), _stream(stream)), "dora_factored_norm_sq")
+    return sq_out
+
+
+def dora_norm_finalize(sq: torch.Tensor, m: Optional[torch.Tensor] = None, eps: float = 0.0,
+                       n_out: Optional[torch.Tensor] = None,
+                       g_out: Optional[torch.Tensor] = None, stream=None):
+    """n = sqrt(max(sq, 0)) and, with m, g = m / max(n, eps).  Returns (n, g or None)."""
+    lib = load_library()
+    d_out = sq.shape[0]
+    dev = sq.device
+    n_out = torch.empty(d_out, dtype=torch.float32, device=dev) if n_out is None else n_out
+    if m is not None and g_out is None:
+        g_out = torch.empty(d_out, dtype=torch.float32, device=dev)
+    _check(lib.dora_norm_finalize(
+        _dev(sq, "sq", torch.float32, (d_out,)), _dev(m, "m", torch.float32, (d_out,)),
+        float(eps), d_out, _dev(n_out, "n_out", torch.float32, (d_out,)),
+        _dev(g_out if m is not None else None, "g_out", torch.float32, (d_out,)),
+        _stream(stream)), "dora_norm_finalize")
+    return n_out, (g_out if m is not None else None)

@@ -86,7 +86,10 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Whether [a, a + na) and [b, b + nb) share a byte; an absent (NULL) buffer
+// overlaps nothing.
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  if (a == nullptr || b == nullptr) return false;
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
   return x < y + nb && y < x + na;
 }
@@ -431,7 +434,7 @@ dora_status_t check_problem(const dora_norm_problem_t& p) {
 }
 
 dora_status_t run_tc_group(const dora_norm_problem_t* probs, int count, bool grouped, float eps,
-                           void* ws, size_t ws_bytes, cudaStream_t st) {
+                           void* ws, size_t ws_bytes, cudaStream_t st, bool emit_sq = false) {
   const DeviceInfo* di = device_info();
   if (di == nullptr) return DORA_ERR_CUDA;
   if (!di->supported) return DORA_ERR_UNSUPPORTED;
@@ -455,6 +458,7 @@ dora_status_t run_tc_group(const dora_norm_problem_t* probs, int count, bool gro
   for (int i = 0; i < count; ++i) {
     if (!fill_descriptors(probs[i], L.plans[i], base, ub, jb, nds[i], gds[i]))
       return DORA_ERR_INVALID_ARG;
+    nds[i].emit_sq = emit_sq ? 1 : 0;
     ub += L.plans[i].units;
     jb += L.plans[i].pairs * L.plans[i].S;
   }
@@ -607,17 +611,23 @@ size_t dora_factored_norm_workspace_size(int64_t d_out, int64_t d_in, int64_t r,
   return std::max(L.total_bytes, simt_workspace(r));
 }
 
-dora_status_t dora_factored_norm(const void* W0, const void* A, const void* B, dora_dtype_t dt,
-                                 int64_t d_out, int64_t d_in, int64_t r, float s, const float* m,
-                                 float eps, float* n_out, float* g_out, void* ws, size_t ws_bytes,
-                                 dora_stream_t stream) {
+}  // extern "C"
+
+namespace {
+// The single-module norm; with emit_sq the squared-norm sums (before the
+// clamp and sqrt) go to n_out and g is not formed.
+dora_status_t norm_impl(const void* W0, const void* A, const void* B, dora_dtype_t dt,
+                        int64_t d_out, int64_t d_in, int64_t r, float s, const float* m, float eps,
+                        float* n_out, float* g_out, void* ws, size_t ws_bytes,
+                        dora_stream_t stream, bool emit_sq) {
   if (dt != DORA_F32 && dt != DORA_BF16) return DORA_ERR_INVALID_ARG;
   dora_norm_problem_t p{W0, A, B, m, n_out, g_out, d_out, d_in, r, s};
   dora_status_t st = check_problem(p);
   if (st != DORA_OK) return st;
   if (!(eps >= 0.f)) return DORA_ERR_INVALID_ARG;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  if (dt == DORA_BF16 && tc_eligible(p)) return run_tc_group(&p, 1, false, eps, ws, ws_bytes, cs);
+  if (dt == DORA_BF16 && tc_eligible(p))
+    return run_tc_group(&p, 1, false, eps, ws, ws_bytes, cs, emit_sq);
 
   const DeviceInfo* di = device_info();
   if (di == nullptr) return DORA_ERR_CUDA;
@@ -626,13 +636,15 @@ dora_status_t dora_factored_norm(const void* W0, const void* A, const void* B, d
   float* G = static_cast<float*>(ws);
   const long long warps = r * r;
   const unsigned gblocks = static_cast<unsigned>(ceil_div_ll(warps * 32, 256));
+  const int esq = emit_sq ? 1 : 0;
   if (dt == DORA_F32) {
     gram_simt_kernel<float><<<gblocks, 256, 0, cs>>>(static_cast<const float*>(A), (int)r,
                                                      (int)d_in, G);
     if ((st = launch_status()) != DORA_OK) return st;
     norm_simt_kernel<float><<<(unsigned)d_out, 256, 0, cs>>>(
         static_cast<const float*>(W0), static_cast<const float*>(A),
-        static_cast<const float*>(B), G, (int)d_out, (int)d_in, (int)r, s, m, eps, n_out, g_out);
+        static_cast<const float*>(B), G, (int)d_out, (int)d_in, (int)r, s, m, eps, n_out, g_out,
+        esq);
   } else {
     gram_simt_kernel<__nv_bfloat16><<<gblocks, 256, 0, cs>>>(
         static_cast<const __nv_bfloat16*>(A), (int)r, (int)d_in, G);
@@ -640,8 +652,45 @@ dora_status_t dora_factored_norm(const void* W0, const void* A, const void* B, d
     norm_simt_kernel<__nv_bfloat16><<<(unsigned)d_out, 256, 0, cs>>>(
         static_cast<const __nv_bfloat16*>(W0), static_cast<const __nv_bfloat16*>(A),
         static_cast<const __nv_bfloat16*>(B), G, (int)d_out, (int)d_in, (int)r, s, m, eps, n_out,
-        g_out);
+        g_out, esq);
   }
+  return launch_status();
+}
+}  // namespace
+
+extern "C" {
+
+dora_status_t dora_factored_norm(const void* W0, const void* A, const void* B, dora_dtype_t dt,
+                                 int64_t d_out, int64_t d_in, int64_t r, float s, const float* m,
+                                 float eps, float* n_out, float* g_out, void* ws, size_t ws_bytes,
+                                 dora_stream_t stream) {
+  return norm_impl(W0, A, B, dt, d_out, d_in, r, s, m, eps, n_out, g_out, ws, ws_bytes, stream,
+                   false);
+}
+
+dora_status_t dora_factored_norm_sq(const void* W0, const void* A, const void* B, dora_dtype_t dt,
+                                    int64_t d_out, int64_t d_in, int64_t r, float s,
+                                    float* sq_out, void* ws, size_t ws_bytes,
+                                    dora_stream_t stream) {
+  return norm_impl(W0, A, B, dt, d_out, d_in, r, s, nullptr, 0.f, sq_out, nullptr, ws, ws_bytes,
+                   stream, true);
+}
+
+dora_status_t dora_norm_finalize(const float* sq, const float* m, float eps, int64_t d_out,
+                                 float* n_out, float* g_out, dora_stream_t stream) {
+  if (sq == nullptr || n_out == nullptr || d_out < 1) return DORA_ERR_INVALID_ARG;
+  if ((m == nullptr) != (g_out == nullptr)) return DORA_ERR_INVALID_ARG;
+  if (!(eps >= 0.f)) return DORA_ERR_INVALID_ARG;
+  if (d_out > (1ll << 31) - 1) return DORA_ERR_UNSUPPORTED;
+  const size_t vb = static_cast<size_t>(d_out) * 4;
+  if ((n_out != sq && overlaps(n_out, vb, sq, vb)) || overlaps(g_out, vb, sq, vb) ||
+      overlaps(g_out, vb, n_out, vb) || overlaps(n_out, vb, m, vb) || overlaps(g_out, vb, m, vb))
+    return DORA_ERR_INVALID_ARG;
+  const DeviceInfo* di = device_info();
+  if (di == nullptr) return DORA_ERR_CUDA;
+  if (!di->supported) return DORA_ERR_UNSUPPORTED;
+  launch_pdl(norm_finalize_sq_kernel, dim3((unsigned)ceil_div_ll(d_out, 256)), dim3(256), 0,
+             reinterpret_cast<cudaStream_t>(stream), sq, (int)d_out, m, eps, n_out, g_out);
   return launch_status();
 }
 

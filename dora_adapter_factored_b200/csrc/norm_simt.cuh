@@ -7,6 +7,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace dora {
 
@@ -66,7 +67,7 @@ __global__ void __launch_bounds__(256)
     norm_simt_kernel(const T* __restrict__ W0, const T* __restrict__ A, const T* __restrict__ B,
                      const float* __restrict__ G, int d_out, int d_in, int r, float s,
                      const float* __restrict__ m, float eps, float* __restrict__ n_out,
-                     float* __restrict__ g_out) {
+                     float* __restrict__ g_out, int emit_sq) {
   __shared__ float U[DORA_MAX_RANK];
   __shared__ float Bi[DORA_MAX_RANK];
   __shared__ float red[8];
@@ -108,10 +109,28 @@ __global__ void __launch_bounds__(256)
 
   if (tid == 0) {
     const float sq = ss + 2.f * s * cross + s * s * gram;
+    if (emit_sq) {
+      n_out[i] = sq;
+      return;
+    }
     const float n = __fsqrt_rn(fmaxf(sq, 0.f));
     n_out[i] = n;
     if (m != nullptr && g_out != nullptr) g_out[i] = __fdiv_rn(m[i], fmaxf(n, eps));
   }
+}
+
+// n_i = sqrt(max(sq_i, 0)), g_i = m_i / max(n_i, eps): the finalize of a norm
+// whose squared sums were reduced across devices.
+__global__ void __launch_bounds__(256)
+    norm_finalize_sq_kernel(const float* __restrict__ sq, int d_out, const float* __restrict__ m,
+                            float eps, float* __restrict__ n_out, float* __restrict__ g_out) {
+  grid_dependency_wait();
+  grid_dependency_trigger();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= d_out) return;
+  const float n = __fsqrt_rn(fmaxf(sq[i], 0.f));
+  n_out[i] = n;
+  if (m != nullptr && g_out != nullptr) g_out[i] = __fdiv_rn(m[i], fmaxf(n, eps));
 }
 
 }  // namespace dora

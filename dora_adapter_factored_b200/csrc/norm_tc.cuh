@@ -72,6 +72,7 @@ struct alignas(64) NormProblemDev {
   int n0, n1;            // N of the two accumulator chunks (n1 = 0: single chunk)
   int box_rows, nbox;    // N-side operand: boxes per stage and rows per box
   int slab3d;            // tm_a / tm_g / tm_glo are 3-D {64, box_rows, nbox}: one box per slab
+  int emit_sq;           // write the squared-norm sum itself to n_out (no clamp, sqrt or g)
   int kb_w, kb_r, kb_tile, tiles, seg_slots;  // kb_tile = kb_w + 2 kb_r (hi, then lo)
   uint32_t stage_tx;     // bytes landing per stage
   uint32_t idesc0, idesc1;
@@ -508,10 +509,14 @@ __global__ void __maxnreg__(kNormMaxRegs)
             if (valid) {
               float sum = 0.f;
               for (int c = 0; c < nseg; ++c) sum += __ldcg(part_t + static_cast<size_t>(c) * kTileM);
-              const float n = __fsqrt_rn(fmaxf(sum, 0.f));
-              P->n_out[grow] = n;
-              if (P->m != nullptr && P->g_out != nullptr)
-                P->g_out[grow] = __fdiv_rn(__ldg(P->m + grow), fmaxf(n, eps));
+              if (P->emit_sq) {
+                P->n_out[grow] = sum;
+              } else {
+                const float n = __fsqrt_rn(fmaxf(sum, 0.f));
+                P->n_out[grow] = n;
+                if (P->m != nullptr && P->g_out != nullptr)
+                  P->g_out[grow] = __fdiv_rn(__ldg(P->m + grow), fmaxf(n, eps));
+              }
             }
           }
         }

@@ -122,6 +122,28 @@ dora_status_t dora_factored_norm_grouped(const dora_norm_problem_t *problems,
                                          dora_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * d_in-sharded norm  ["Scaling DoRA ...", section 6: sharded base weights need
+ * chunk-wise partial sums followed by an all-reduce; section 2: every term of
+ * the squared row norm is a sum over the columns of W0]
+ *
+ * With W0 and A split by columns into shards k (W0^(k) = W0[:, J_k],
+ * A^(k) = A[:, J_k], B whole), the squared row norm is the sum over shards of
+ *   sq_i^(k) = ||W0_i^(k)||^2 + 2 s B_i.(W0^(k) A^(k)T)_i + s^2 B_i A^(k) A^(k)T B_i^T.
+ * dora_factored_norm_sq computes sq^(k) for one shard (arguments as for
+ * dora_factored_norm, with d_in the shard's width; the same workspace size)
+ * and writes it to sq_out [d_out] fp32, before any clamp or square root.
+ * After the caller sums sq over the shards (one all-reduce of d_out floats),
+ * dora_norm_finalize writes n = sqrt(max(sq, 0)) and, when m and g_out are
+ * given, g = m / max(n, eps).  n_out may equal sq.
+ * ---------------------------------------------------------------------- */
+dora_status_t dora_factored_norm_sq(const void *W0, const void *A, const void *B,
+                                    dora_dtype_t dt, int64_t d_out, int64_t d_in, int64_t r,
+                                    float s, float *sq_out, void *ws, size_t ws_bytes,
+                                    dora_stream_t stream);
+dora_status_t dora_norm_finalize(const float *sq, const float *m, float eps, int64_t d_out,
+                                 float *n_out, float *g_out, dora_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Fused compose forward  ["Scaling DoRA ...", section 3 and Data Availability]
  *
  * With n_c = max(n, eps), g = m / n_c and (g - 1) = (m - n_c) / n_c in fp32:

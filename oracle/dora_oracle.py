@@ -53,6 +53,7 @@ __all__ = [
     "dora_param_count",
     "dense_row_norm",
     "factored_row_norm",
+    "factored_row_norm_sq",
     "factored_intermediate_elems",
     "magnitude_scale",
     "compose_fwd",
@@ -144,6 +145,20 @@ def factored_row_norm(W0, A, B, s: float) -> np.ndarray:
     gram = np.sum((B @ G) * B, axis=1)
     sq = base + 2.0 * s * cross + (s * s) * gram
     return np.sqrt(np.maximum(sq, 0.0))
+
+
+def factored_row_norm_sq(W0, A, B, s: float) -> np.ndarray:
+    """The squared row norm in factored form, before the clamp and the square
+    root: ||W0_i||^2 + 2 s B_i.(W0 A^T)_i + s^2 B_i (A A^T) B_i^T
+    [ScalingDoRA, section 2].  Every term is a sum over the columns of W0 (and
+    of A), so for a column split of W0 and A the values of the parts add up to
+    the whole: the per-shard partial of a d_in-sharded norm [ScalingDoRA,
+    section 6, chunk-wise partial sums followed by an all-reduce]."""
+    W0, A, B = _f64(W0), _f64(A), _f64(B)
+    base = np.sum(W0 * W0, axis=1)
+    cross = np.sum(B * (W0 @ A.T), axis=1)
+    gram = np.sum((B @ (A @ A.T)) * B, axis=1)
+    return base + 2.0 * s * cross + (s * s) * gram
 
 
 # --------------------------------------------------------------------------

@@ -144,6 +144,33 @@ def test_merge_validation(built_library):
     assert dora.dora_launch_count() == before
 
 
+def torch_cuda_available():
+    import torch
+    return torch.cuda.is_available()
+
+
+def test_sharded_norm_validation(built_library):
+    lib = dora.load_library(built_library)
+    before = dora.dora_launch_count()
+    vp = ctypes.c_void_p
+    p = vp(0x10000)
+    # squared partial: null output, rank above the limit
+    assert lib.dora_factored_norm_sq(p, p, p, _abi.DORA_BF16, 8, 8, 8, 2.0, None, p, 1 << 20,
+                                     None) == _abi.DORA_ERR_INVALID_ARG
+    assert lib.dora_factored_norm_sq(p, p, p, _abi.DORA_BF16, 8, 8, 513, 2.0, vp(0x20000), p,
+                                     1 << 20, None) == _abi.DORA_ERR_UNSUPPORTED
+    # finalize: m without g_out; g_out overlapping n_out
+    assert lib.dora_norm_finalize(p, vp(0x20000), 0.0, 8, vp(0x30000), None,
+                                  None) == _abi.DORA_ERR_INVALID_ARG
+    assert lib.dora_norm_finalize(p, vp(0x20000), 0.0, 8, vp(0x30000), vp(0x30010),
+                                  None) == _abi.DORA_ERR_INVALID_ARG
+    assert dora.dora_launch_count() == before
+    # neither m nor g_out: valid arguments (the call then needs a device)
+    if not torch_cuda_available():
+        assert lib.dora_norm_finalize(p, None, 0.0, 8, vp(0x30000), None,
+                                      None) == _abi.DORA_ERR_CUDA
+
+
 def test_grouped_workspace_sizes(built_library):
     lib = dora.load_library(built_library)
     arr = (_abi.ComposeProblem * 3)()

@@ -363,6 +363,25 @@ def test_merged_forward_equals_compose():
     np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
 
 
+# ---------------------------------------------------------------- d_in shards
+
+def test_shard_partials_add_up_to_the_dense_squared_norm():
+    # Any column split: the shards' squared partials sum to ||(W0 + sBA)_i||^2
+    # computed densely (brute force on the materialised V).
+    rng = np.random.default_rng(18)
+    W0, A, B = _rand_module(rng, 7, 13, 4)
+    s = 1.7
+    V = W0 + s * (B @ A)
+    dense_sq = np.sum(V * V, axis=1)
+    for cuts in ([0, 13], [0, 5, 13], [0, 1, 2, 9, 13], [0, 0, 13]):
+        total = sum(oracle.factored_row_norm_sq(W0[:, a:b], A[:, a:b], B, s)
+                    for a, b in zip(cuts[:-1], cuts[1:]))
+        np.testing.assert_allclose(total, dense_sq, rtol=1e-12)
+    # one shard's partial is not the whole (the split matters)
+    part = oracle.factored_row_norm_sq(W0[:, :5], A[:, :5], B, s)
+    assert not np.allclose(part, dense_sq, rtol=1e-3)
+
+
 # ---------------------------------------------------------------- planted mistakes
 
 def test_pins_catch_planted_mistakes():
