@@ -468,7 +468,7 @@ def run_gpu(args):
             "components": components,
             "clocks": clk,
             "gpu_launches": int(launches),
-            "launch": "CUDA graph replay of the step's API calls (7 kernels, programmatic "
+            "launch": "CUDA graph replay of the step's API calls (6 kernels, programmatic "
                       "dependent launches)",
             "eager_ms_per_step": eager_ms,
             "e2e": e2e,
@@ -573,12 +573,345 @@ def measure_cpu_baseline(t_roof):
                        f"({t:.2f} s per full step)")}
 
 
+# --------------------------------------------------------------------------- suite
+
+def _device_time(fn, iters, flush):
+    """Median device time (s) of fn(i), each call bracketed by CUDA events on
+    the current stream; a write of a buffer larger than L2 runs between calls
+    (outside the events), so every call starts with a cold L2."""
+    import torch
+    st = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(iters)]
+    for i in range(iters):
+        flush.zero_()
+        evs[i][0].record(st)
+        fn(i)
+        evs[i][1].record(st)
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in evs) * 1e-3
+
+
+def _oracle_seconds(fn, scale, budget_s=2.0):
+    """Mean wall time of the oracle sample fn(), times `scale` (the sample's
+    share of the full call), over about budget_s seconds."""
+    fn()
+    ts = []
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s and len(ts) < 50:
+        t1 = time.perf_counter()
+        fn()
+        ts.append(time.perf_counter() - t1)
+    return statistics.mean(ts) * scale, len(ts)
+
+
+def run_suite(args):
+    """One JSON line per workload beyond the headline step, each timed on the
+    device against the roofline of its algorithmic work (measured peaks), with
+    the oracle timed on a host sample beside it."""
+    import numpy as np
+    import torch
+    import oracle
+    import dora_adapter_factored_b200 as dora
+    from dora_adapter_factored_b200 import synth
+    if int(os.environ.get("WORLD_SIZE", "1")) != 1:
+        raise SystemExit("--suite runs on one GPU")
+    peaks = load_peaks()
+    HBM, TC = peaks["hbm_gbs"] * 1e9, peaks["bf16_tflops"] * 1e12
+    dev = torch.device("cuda")
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)  # 256 MB > L2
+    eps = synth.eps_for("bf16")
+    iters = max(5, min(args.steps, 30))
+    cores = blas_threads()
+
+    def emit(name, workload, t_gpu, flops, nbytes, oracle_s=None, sample=None, extra=None):
+        t_roof = max(flops / TC, nbytes / HBM)
+        bound = "tensor" if flops / TC >= nbytes / HBM else "hbm"
+        line = {"suite": name, "workload": workload, "us": t_gpu * 1e6,
+                "roofline_us": t_roof * 1e6, "frac_of_roofline": t_roof / t_gpu, "bound": bound,
+                "achieved": (flops / t_gpu / 1e12) if bound == "tensor" else (nbytes / t_gpu / 1e9),
+                "peak": peaks["bf16_tflops"] if bound == "tensor" else peaks["hbm_gbs"],
+                "unit": "TFLOP/s" if bound == "tensor" else "GB/s",
+                "algorithmic": {"flops": flops, "bytes": nbytes}, "l2": "flushed between calls",
+                "peak_source": peaks["source"]}
+        if oracle_s is not None:
+            line["cpu_baseline"] = {"kind": "oracle", "seconds_per_call": oracle_s,
+                                    "cores": cores, "sample": sample,
+                                    "gpu_speedup": oracle_s / t_gpu}
+        if extra:
+            line.update(extra)
+        print(json.dumps(line), flush=True)
+
+    def two_sets(w, index=0):
+        W0, A, B = synth.module_weights(w, index=index, device=dev)
+        return [(W0, A, B), (W0.flip(0).contiguous(), A, B.flip(0).contiguous())]
+
+    # ---- factored norm on each single-module configuration
+    for key in ("norm_4096_r64", "headline_8192_r384", "mlp_up_25600x5120_r384"):
+        w = synth.WORKLOADS[key]
+        ms = w.modules[0]
+        sets = two_sets(w)
+        n = torch.empty(ms.d_out, device=dev)
+        ws = torch.empty(dora.dora_factored_norm_workspace_size(ms.d_out, ms.d_in, ms.r,
+                                                               torch.bfloat16),
+                         dtype=torch.uint8, device=dev)
+        fn = lambda i: dora.dora_factored_norm(*sets[i % 2], ms.s, n_out=n, ws=ws)
+        for i in range(3):
+            fn(i)
+        t = _device_time(fn, iters, flush)
+        W0h, Ah, Bh = (x.float().cpu().numpy() for x in sets[0])
+        rows = 16
+        o_s, reps = _oracle_seconds(lambda: oracle.rows_dense_row_norm(
+            W0h[:rows].astype(np.float64), Ah.astype(np.float64), Bh[:rows].astype(np.float64),
+            ms.s), ms.d_out / rows)
+        emit("factored_norm", key, t, 2.0 * ms.d_out * ms.d_in * ms.r,
+             2.0 * (ms.d_out * ms.d_in + ms.r * ms.d_in + ms.d_out * ms.r), o_s,
+             f"fp64 dense norm of {rows} of {ms.d_out} rows ({reps} repeats), scaled")
+        del sets, ws
+
+    # ---- grouped norm over the 56-module layer stack
+    w = synth.WORKLOADS["layer_stack_56"]
+    mods = []
+    for i, ms in enumerate(w.modules):
+        W0, A, B = synth.module_weights(w, index=i, device=dev)
+        mods.append(dict(W0=W0, A=A, B=B, s=ms.s, n_out=torch.empty(ms.d_out, device=dev)))
+    ws = torch.empty(dora.dora_factored_norm_grouped_workspace_size(mods), dtype=torch.uint8,
+                     device=dev)
+    fn = lambda i: dora.dora_factored_norm_grouped(mods, ws=ws)
+    for i in range(3):
+        fn(i)
+    t = _device_time(fn, max(5, iters // 3), flush)
+    fl = sum(2.0 * m_.d_out * m_.d_in * m_.r for m_ in w.modules)
+    by = sum(2.0 * (m_.d_out * m_.d_in + m_.r * m_.d_in + m_.d_out * m_.r) for m_ in w.modules)
+    kinds = {}
+    for i, m_ in enumerate(w.modules[:7]):
+        kinds[i] = m_
+    def stack_sample():
+        for i, m_ in kinds.items():
+            p = mods[i]
+            oracle.rows_dense_row_norm(p["W0"][:4].float().cpu().numpy().astype(np.float64),
+                                       p["A"].float().cpu().numpy().astype(np.float64),
+                                       p["B"][:4].float().cpu().numpy().astype(np.float64), m_.s)
+    layer_rows = sum(m_.d_out for m_ in w.modules[:7])
+    o_s, reps = _oracle_seconds(stack_sample, (layer_rows / 28.0) * (len(w.modules) / 7), 3.0)
+    emit("grouped_norm", "layer_stack_56", t, fl, by, o_s,
+         f"fp64 dense norm of 4 rows of each of one layer's 7 modules ({reps} repeats), scaled "
+         "to all rows of the 56 modules", {"modules": len(w.modules)})
+    del mods, ws
+
+    # ---- compose forward / backward on the MLP up-projection activations
+    def acts(T, d_out, seed):
+        g = torch.Generator(device=dev).manual_seed(seed)
+        a = {k: torch.randn(T, d_out, device=dev, generator=g).bfloat16()
+             for k in ("base", "lora", "dy")}
+        a["n"] = torch.rand(d_out, device=dev, generator=g) + 1.0
+        a["m"] = a["n"] * (1.0 + 0.005 * torch.randn(d_out, device=dev, generator=g))
+        return a
+
+    def eager_fwd(a, s):
+        nc = a["n"].clamp_min(eps)
+        g = a["m"] / nc
+        gm1 = (a["m"] - nc) / nc
+        b, l = a["base"], a["lora"]
+        return b + (gm1.to(b.dtype) * b + (g * s).to(b.dtype) * l)  # 4 elementwise ops
+
+    def eager_bwd(a, s):
+        nc = a["n"].clamp_min(eps)
+        g = a["m"] / nc
+        d = a["dy"]
+        db = d * g.to(d.dtype)
+        dl = d * (g * s).to(d.dtype)
+        dm = (d.float() * (a["base"].float() + s * a["lora"].float())).sum(0) / nc
+        return db, dl, dm
+
+    def compose_pair(key, T, d_out, s, label):
+        sets = [acts(T, d_out, 11), acts(T, d_out, 12)]
+        ws = torch.empty(max(256, dora.dora_compose_bwd_workspace_size(T, d_out, torch.bfloat16)),
+                         dtype=torch.uint8, device=dev)
+        y = torch.empty(T, d_out, dtype=torch.bfloat16, device=dev)
+        db, dl = torch.empty_like(y), torch.empty_like(y)
+        dm = torch.empty(d_out, device=dev)
+        act = 2.0 * T * d_out
+        res = {}
+        for direction, fused, eager, passes in (
+                ("fwd", lambda i: dora.dora_compose_fwd(sets[i % 2]["base"], sets[i % 2]["lora"],
+                                                        sets[i % 2]["m"], sets[i % 2]["n"], s,
+                                                        eps, y=y),
+                 lambda i: eager_fwd(sets[i % 2], s), 3),
+                ("bwd", lambda i: dora.dora_compose_bwd(sets[i % 2]["dy"], sets[i % 2]["base"],
+                                                        sets[i % 2]["lora"], sets[i % 2]["m"],
+                                                        sets[i % 2]["n"], s, eps, d_base=db,
+                                                        d_lora=dl, dm=dm, ws=ws),
+                 lambda i: eager_bwd(sets[i % 2], s), 5)):
+            for i in range(3):
+                fused(i)
+                eager(i)
+            tf = _device_time(fused, iters, flush)
+            te = _device_time(eager, max(5, iters // 3), flush)
+            res[direction] = (tf, te, passes)
+        return res, act, sets
+
+    res, act, sets = compose_pair("mlp_up", 8192, 25600, 2.0, "C4")
+    h = {k: v[:64].float().cpu().numpy().astype(np.float64) for k, v in sets[0].items()
+         if k in ("base", "lora", "dy")}
+    mh, nh = sets[0]["m"].double().cpu().numpy(), sets[0]["n"].double().cpu().numpy()
+    for direction, (tf, te, passes) in res.items():
+        if direction == "fwd":
+            smp = lambda: oracle.compose_fwd(h["base"], h["lora"], mh, nh, 2.0, eps)
+        else:
+            smp = lambda: oracle.compose_bwd(h["dy"], h["base"], h["lora"], mh, nh, 2.0, eps)
+        o_s, reps = _oracle_seconds(smp, 8192 / 64)
+        emit(f"compose_{direction}", "mlp_up [8192, 25600] bf16", tf, 0.0, passes * act, o_s,
+             f"fp64 compose {direction} on 64 of 8192 tokens ({reps} repeats), scaled",
+             {"eager_torch_us": te * 1e6, "speedup_vs_eager": te / tf})
+    del sets
+
+    # ---- training-step variants at the headline activations
+    T, d_out, s = 4096, 8192, 2.0
+    sets = [acts(T, d_out, 21), acts(T, d_out, 22)]
+    for a in sets:
+        a["inner"] = torch.empty_like(a["base"])
+    y = torch.empty(T, d_out, dtype=torch.bfloat16, device=dev)
+    db, dl = torch.empty_like(y), torch.empty_like(y)
+    dm = torch.empty(d_out, device=dev)
+    ws = torch.empty(dora.dora_compose_bwd_workspace_size(T, d_out, torch.bfloat16),
+                     dtype=torch.uint8, device=dev)
+    act = 2.0 * T * d_out
+    variants = (
+        ("compose_fwd_train", 4, lambda i: dora.dora_compose_fwd_train(
+            sets[i % 2]["base"], sets[i % 2]["lora"], sets[i % 2]["m"], sets[i % 2]["n"], s, eps,
+            y=y, inner=sets[i % 2]["inner"])),
+        ("compose_bwd_inner", 4, lambda i: dora.dora_compose_bwd_inner(
+            sets[i % 2]["dy"], sets[i % 2]["inner"], sets[i % 2]["m"], sets[i % 2]["n"], s, eps,
+            d_base=db, d_lora=dl, dm=dm, ws=ws)),
+        ("compose_bwd_frozen", 3, lambda i: dora.dora_compose_bwd_frozen(
+            sets[i % 2]["dy"], sets[i % 2]["m"], sets[i % 2]["n"], s, eps, d_base=db, d_lora=dl)),
+    )
+    hb = {k: v[:64].float().cpu().numpy().astype(np.float64) for k, v in sets[0].items()
+          if k in ("base", "lora", "dy")}
+    mh, nh = sets[0]["m"].double().cpu().numpy(), sets[0]["n"].double().cpu().numpy()
+    samples = {
+        "compose_fwd_train": lambda: (oracle.compose_fwd(hb["base"], hb["lora"], mh, nh, s, eps),
+                                      oracle.compose_inner(hb["base"], hb["lora"], s)),
+        "compose_bwd_inner": lambda: oracle.compose_bwd_from_inner(
+            hb["dy"], hb["base"] + s * hb["lora"], mh, nh, s, eps),
+        "compose_bwd_frozen": lambda: oracle.compose_bwd_frozen(hb["dy"], mh, nh, s, eps),
+    }
+    for name, passes, fn in variants:
+        for i in range(3):
+            fn(i)
+        t = _device_time(fn, iters, flush)
+        o_s, reps = _oracle_seconds(samples[name], T / 64)
+        emit(name, "headline [4096, 8192] bf16", t, 0.0, passes * act, o_s,
+             f"fp64 on 64 of {T} tokens ({reps} repeats), scaled")
+    del sets
+
+    # ---- compose sweep: fused vs eager over the layer-stack shapes
+    for d in (1024, 4096, 14336):
+        for T in (512, 2048, 8192, 32768):
+            res, act, sets = compose_pair("sweep", T, d, 2.0, "C5")
+            for direction, (tf, te, passes) in res.items():
+                emit(f"compose_sweep_{direction}", f"[{T}, {d}] bf16", tf, 0.0, passes * act,
+                     extra={"eager_torch_us": te * 1e6, "speedup_vs_eager": te / tf})
+            del sets
+
+    # ---- grouped compose: one decoder layer's 7 modules
+    layer = (4096, 1024, 1024, 4096, 14336, 14336, 4096)
+    for T in (512, 2048, 8192):
+        mods = [acts(T, d, 31 + i) for i, d in enumerate(layer)]
+        for a in mods:
+            a["y"] = torch.empty_like(a["base"])
+            a["d_base"], a["d_lora"] = torch.empty_like(a["base"]), torch.empty_like(a["base"])
+            a["dm_out"] = torch.empty(a["base"].shape[1], device=dev)
+            a["ws"] = torch.empty(max(256, dora.dora_compose_bwd_workspace_size(
+                T, a["base"].shape[1], torch.bfloat16)), dtype=torch.uint8, device=dev)
+        fitems = [dict(base=a["base"], lora=a["lora"], m=a["m"], n=a["n"], s=2.0, y=a["y"])
+                  for a in mods]
+        bitems = [dict(dy=a["dy"], base=a["base"], lora=a["lora"], m=a["m"], n=a["n"], s=2.0,
+                       d_base=a["d_base"], d_lora=a["d_lora"], dm=a["dm_out"]) for a in mods]
+        gws = torch.empty(max(256, dora.dora_compose_bwd_grouped_workspace_size(bitems)),
+                          dtype=torch.uint8, device=dev)
+        act = sum(2.0 * T * d for d in layer)
+        cases = (
+            ("fwd", 3, lambda i: dora.dora_compose_fwd_grouped(fitems, eps),
+             lambda i: [dora.dora_compose_fwd(a["base"], a["lora"], a["m"], a["n"], 2.0, eps,
+                                              y=a["y"]) for a in mods]),
+            ("bwd", 5, lambda i: dora.dora_compose_bwd_grouped(bitems, eps, ws=gws),
+             lambda i: [dora.dora_compose_bwd(a["dy"], a["base"], a["lora"], a["m"], a["n"], 2.0,
+                                              eps, d_base=a["d_base"], d_lora=a["d_lora"],
+                                              dm=a["dm_out"], ws=a["ws"]) for a in mods]),
+        )
+        for direction, passes, grouped, single in cases:
+            for i in range(3):
+                grouped(i)
+                single(i)
+            tg = _device_time(grouped, iters, flush)
+            ts_ = _device_time(single, iters, flush)
+            emit(f"compose_grouped_{direction}", f"one layer (7 modules) at T={T} bf16", tg, 0.0,
+                 passes * act, extra={"seven_calls_us": ts_ * 1e6, "speedup_vs_calls": ts_ / tg})
+        del mods
+
+    # ---- merged inference weight
+    for key in ("headline_8192_r384", "mlp_up_25600x5120_r384"):
+        w = synth.WORKLOADS[key]
+        ms = w.modules[0]
+        sets = two_sets(w)
+        ns = []
+        for W0, A, B in sets:
+            n_, _ = dora.dora_factored_norm(W0, A, B, ms.s)
+            ns.append((n_, n_ * 1.001))
+        out = torch.empty_like(sets[0][0])
+        ws = torch.empty(dora.dora_merge_weight_workspace_size(ms.d_out, ms.d_in, ms.r),
+                         dtype=torch.uint8, device=dev)
+        fn = lambda i: dora.dora_merge_weight(*sets[i % 2], ns[i % 2][1], ns[i % 2][0], ms.s, eps,
+                                              W_out=out, ws=ws)
+        for i in range(3):
+            fn(i)
+        t = _device_time(fn, iters, flush)
+        W0h, Ah, Bh = (x.float().cpu().numpy().astype(np.float64) for x in sets[0])
+        mh, nh = ns[0][1].double().cpu().numpy(), ns[0][0].double().cpu().numpy()
+        rows = 16
+        o_s, reps = _oracle_seconds(lambda: oracle.merge_weight_given_norm(
+            W0h[:rows], Ah, Bh[:rows], mh[:rows], nh[:rows], ms.s, eps), ms.d_out / rows)
+        emit("merge_weight", key, t, 2.0 * ms.d_out * ms.d_in * ms.r,
+             2.0 * (2 * ms.d_out * ms.d_in + ms.r * ms.d_in + ms.d_out * ms.r), o_s,
+             f"fp64 merge of {rows} of {ms.d_out} rows ({reps} repeats), scaled")
+        del sets, ws, out
+
+    # ---- one column shard of the headline module (d_in-sharded norm, 2 ranks)
+    w = synth.WORKLOADS["headline_8192_r384"]
+    ms = w.modules[0]
+    W0, A, B = synth.module_weights(w, device=dev)
+    a0, b0 = dora.column_shard(ms.d_in, 0, 2)
+    shards = [(W0[:, a0:b0].contiguous(), A[:, a0:b0].contiguous(), B),
+              (W0.flip(0)[:, a0:b0].contiguous(), A[:, a0:b0].contiguous(), B.flip(0).contiguous())]
+    del W0
+    sq = torch.empty(ms.d_out, device=dev)
+    ws = torch.empty(dora.dora_factored_norm_workspace_size(ms.d_out, b0 - a0, ms.r,
+                                                           torch.bfloat16),
+                     dtype=torch.uint8, device=dev)
+    fn = lambda i: dora.dora_factored_norm_sq(*shards[i % 2], ms.s, sq_out=sq, ws=ws)
+    for i in range(3):
+        fn(i)
+    t = _device_time(fn, iters, flush)
+    wd = b0 - a0
+    emit("factored_norm_sq_shard", f"headline module, columns [{a0}, {b0}) of 2 shards", t,
+         2.0 * ms.d_out * wd * ms.r, 2.0 * (ms.d_out * wd + ms.r * wd + ms.d_out * ms.r))
+    if dora.dora_get_device_status() != 0:
+        raise RuntimeError("a kernel reported an error during the suite")
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--suite", action="store_true",
+                    help="instead of the headline line: one JSON line per further workload "
+                         "(the other configurations and the training / grouped / merge / "
+                         "sharded calls), each against its roofline with the oracle beside it")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
@@ -588,6 +921,8 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     with torch.cuda.stream(torch.cuda.Stream()):  # a non-default stream for the whole run
+        if args.suite:
+            return run_suite(args)
         return run_gpu(args)
 
 

@@ -96,8 +96,12 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 
 // Launch with programmatic stream serialization: the kernel may start while
 // its predecessor drains; every kernel of the library executes
-// griddepcontrol.wait before it reads anything a predecessor writes, and
-// before it lets its own dependents launch.
+// griddepcontrol.wait before it reads or writes anything a predecessor
+// touches.  Most let their dependents launch only after that wait, so that a
+// kernel's launch implies its predecessor's predecessor has completed; the
+// Gram reduce lets the norm GEMM launch at once, which is safe because the
+// GEMM waits for the reduce (hence for the Gram) before it touches their
+// outputs.
 // If the runtime rejects the programmatic attribute for this stream, the
 // kernel is launched again without it (plain stream order).
 thread_local char t_last_error[512] = "";
@@ -942,7 +946,7 @@ dora_status_t dora_compose_bwd_frozen(const void* dy, const float* m, const floa
 namespace dora {
 namespace {
 struct MergeLayout {
-  int kb, stages, tiles_m, tiles_n, r8;
+  int kb, stages, wbufs, tiles_m, tiles_n, r8;
   size_t smem_bytes, ws_bytes;
 };
 
@@ -952,8 +956,11 @@ bool merge_layout(int64_t d_out, int64_t d_in, int64_t r, MergeLayout& L) {
   L.r8 = round_up_int(static_cast<int>(r), 8);
   L.tiles_m = static_cast<int>(ceil_div_ll(d_out, kMergeM));
   L.tiles_n = static_cast<int>(ceil_div_ll(d_in, kMergeN));
+  // Shared memory: W0 / W' staging buffers (the HBM stream: several tiles in
+  // flight) and k-block stages (the L2 stream of A^T), 4 + 6 at the limit.
   const size_t tail = align_up(sizeof(MergeSmemTail), 128);
-  const size_t fixed = 1024 + 2 * kMergeTileBytes + static_cast<size_t>(L.kb) * kMergeOperandBytes + tail;
+  L.wbufs = kMergeMaxWBufs;
+  const size_t fixed = 1024 + static_cast<size_t>(L.wbufs) * kMergeTileBytes + tail;
   if (fixed + 2 * kMergeOperandBytes > static_cast<size_t>(kMaxDynSmem)) return false;
   L.stages = static_cast<int>(std::min<size_t>(kMergeMaxStages,
                                                (kMaxDynSmem - fixed) / kMergeOperandBytes));
@@ -1004,7 +1011,7 @@ dora_status_t dora_merge_weight(const void* W0, const void* A, const void* B, co
   uint16_t* At = static_cast<uint16_t*>(ws);
   bool ok = true;
   ok &= make_tmap_bf16(&P.tm_w0, W0, d_out, d_in, d_in, 64, kMergeM);
-  ok &= make_tmap_bf16(&P.tm_out, W_out, d_out, d_in, d_in, 64, kMergeM);
+  ok &= make_tmap_bf16(&P.tm_out, W_out, d_out, d_in, d_in, 64, 32);
   ok &= make_tmap_bf16(&P.tm_b, B, d_out, r, r, kMergeK, kMergeM);
   ok &= make_tmap_bf16(&P.tm_at, At, d_in, r, L.r8, kMergeK, kMergeN);
   if (!ok) return DORA_ERR_INVALID_ARG;
@@ -1028,7 +1035,7 @@ dora_status_t dora_merge_weight(const void* W0, const void* A, const void* B, co
   const int ctas = std::min(di->sms, P.tiles);
   TimedLaunch tl(cs);
   launch_pdl(merge_kernel, dim3(ctas), dim3(kMergeThreads), L.smem_bytes, cs, P, L.stages,
-             g_timeout_ns.load());
+             L.wbufs, g_timeout_ns.load());
   return launch_status();
 }
 

@@ -10,14 +10,18 @@
 //   merge_kernel           persistent, one CTA per SM over 128 x 128 tiles of
 //                          W' in row-major order.  Per tile the tensor cores
 //                          form acc = B_tile A^T_tile over K = r into one of two
-//                          TMEM accumulators (128 columns each); four epilogue
+//                          TMEM accumulators (128 columns each); eight epilogue
 //                          warps then read the W0 tile (staged by TMA into one
-//                          of two shared buffers), write g_i (W0_ij + s acc_ij)
+//                          of up to four shared buffers, so that several tiles
+//                          of W0 are in flight), write g_i (W0_ij + s acc_ij)
 //                          rounded once to bf16 over it in place, and one thread
-//                          stores the tile with TMA.  The CTA keeps its row
-//                          block's B tile (128 x r) resident in shared memory
-//                          while it walks that block's column tiles, so only
-//                          A^T streams through the k-block stages.
+//                          stores the tile with TMA, handing the buffer back
+//                          when its next tile begins.  The CTA keeps its row
+//                          block's B tile (128 x r) resident in TMEM -- copied
+//                          there once per row block (tcgen05.cp) and used as
+//                          the MMAs' A operand -- while it walks that block's
+//                          column tiles, so only A^T streams through the
+//                          shared-memory k-block stages, as many as fit.
 // HBM-bound: W0 is read once and W' written once (2 x 2 bytes per element);
 // the 2 d_out d_in r MMA FLOPs overlap with that traffic.
 #pragma once
@@ -30,15 +34,19 @@ namespace dora {
 constexpr int kMergeM = 128;        // rows of W' per tile (TMEM lanes)
 constexpr int kMergeN = 128;        // columns of W' per tile (accumulator columns)
 constexpr int kMergeK = 64;         // r per k-block: one 128-byte swizzle row
-constexpr int kMergeThreads = 192;  // warps 0-3 epilogue, 4 TMA producer, 5 MMA issuer
-constexpr int kMergeMaxStages = 4;
+constexpr int kMergeEpiWarps = 8;   // two per TMEM lane quadrant, each half of the columns
+constexpr int kMergeThreads = (kMergeEpiWarps + 2) * 32;  // + warp 8 TMA, warp 9 MMA
+constexpr int kMergeMaxStages = 10;
+constexpr int kMergeMaxWBufs = 4;
+constexpr uint32_t kMergeTmemCols = 512;  // 2 x 128 accumulator columns + B (r / 2 columns)
+constexpr uint32_t kMergeTmemB = 2 * kMergeN;  // first TMEM column of the resident B tile
 constexpr uint32_t kMergeOperandBytes = kMergeM * kMergeK * 2;  // 16 KiB: B or A^T k-block
 constexpr uint32_t kMergeTileBytes = kMergeM * kMergeN * 2;     // 32 KiB: W0 in, W' out
 constexpr uint32_t kMergeBoxBytes = kMergeM * 64 * 2;           // 16 KiB: one 64-column box
 
 struct alignas(64) MergeDev {
   CUtensorMap tm_w0;   // W0 [d_out, d_in], box 64 x 128 (load)
-  CUtensorMap tm_out;  // W' [d_out, d_in], box 64 x 128 (store)
+  CUtensorMap tm_out;  // W' [d_out, d_in], box 64 x 32 (store: one epilogue warp's rows)
   CUtensorMap tm_b;    // B  [d_out, r],    box 64 x 128
   CUtensorMap tm_at;   // A^T [d_in, r],    box 64 x 128
   const float* m;
@@ -51,12 +59,11 @@ struct alignas(64) MergeDev {
 };
 
 struct MergeSmemTail {
-  uint64_t full[kMergeMaxStages];   // A^T k-block landed
-  uint64_t empty[kMergeMaxStages];  // MMAs done with the k-block
-  uint64_t b_full, b_empty;         // resident B tile landed / no longer read
-  uint64_t w_full[2], w_empty[2];   // W0 tile landed / W' tile stored out of the buffer
+  uint64_t full[kMergeMaxStages];   // k-block landed (B when a row block starts, else A^T)
+  uint64_t empty[kMergeMaxStages];  // copy or MMAs done with the k-block
+  uint64_t b_swap;                  // every MMA reading the resident B tile has completed
+  uint64_t w_full[kMergeMaxWBufs], w_empty[kMergeMaxWBufs];  // W0 landed / W' stored out
   uint64_t acc_full[2], acc_empty[2];
-  uint64_t epi_done[2];             // the four epilogue warps wrote the buffer
   uint64_t drain;
   uint32_t tmem_slot;
   int abort_flag;
@@ -82,6 +89,7 @@ __device__ __forceinline__ void bulk_commit_group() {
 __device__ __forceinline__ void bulk_wait_group_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
+
 __device__ __forceinline__ void bulk_wait_group0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
@@ -113,13 +121,13 @@ __global__ void __launch_bounds__(256)
 }
 
 __global__ void __launch_bounds__(kMergeThreads, 1)
-    merge_kernel(const __grid_constant__ MergeDev P, int stages, unsigned long long timeout_ns) {
+    merge_kernel(const __grid_constant__ MergeDev P, int stages, int wbufs,
+                 unsigned long long timeout_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* s_w = smem;                                        // 2 x 32 KiB W0 / W' tiles
-  uint8_t* s_b = s_w + 2 * kMergeTileBytes;                   // kb x 16 KiB resident B
-  uint8_t* s_at = s_b + P.kb * kMergeOperandBytes;            // stages x 16 KiB A^T
+  uint8_t* s_w = smem;                                        // wbufs x 32 KiB W0 / W' tiles
+  uint8_t* s_at = s_w + wbufs * kMergeTileBytes;              // stages x 16 KiB B / A^T
   MergeSmemTail* tail =
       reinterpret_cast<MergeSmemTail*>(s_at + stages * kMergeOperandBytes);
   volatile int* abort_flag = &tail->abort_flag;
@@ -135,24 +143,24 @@ __global__ void __launch_bounds__(kMergeThreads, 1)
       mbar_init(&tail->full[s], 1);
       mbar_init(&tail->empty[s], 1);
     }
-    mbar_init(&tail->b_full, 1);
-    mbar_init(&tail->b_empty, 1);
-    for (int b = 0; b < 2; ++b) {
+    mbar_init(&tail->b_swap, 1);
+    for (int b = 0; b < wbufs; ++b) {
       mbar_init(&tail->w_full[b], 1);
-      mbar_init(&tail->w_empty[b], 1);
+      mbar_init(&tail->w_empty[b], kMergeEpiWarps);  // each warp's store has read its rows
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&tail->acc_full[b], 1);
-      mbar_init(&tail->acc_empty[b], 4);
-      mbar_init(&tail->epi_done[b], 4);
+      mbar_init(&tail->acc_empty[b], kMergeEpiWarps);
     }
     mbar_init(&tail->drain, 1);
     tail->abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(&tail->tmem_slot, 2 * kMergeN);
+    tmem_alloc(&tail->tmem_slot, kMergeTmemCols);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kMergeEpiWarps && lane == 0) {
     prefetch_tmap(&P.tm_w0);
     prefetch_tmap(&P.tm_out);
     prefetch_tmap(&P.tm_b);
@@ -166,34 +174,40 @@ __global__ void __launch_bounds__(kMergeThreads, 1)
   grid_dependency_wait();
   grid_dependency_trigger();
 
-  if (warp == 4) {
+  if (warp == kMergeEpiWarps) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && t_begin < t_end) {
       const uint64_t pol_stream = policy_evict_first();
       const uint64_t pol_keep = policy_evict_last();
-      int stage = 0, cur_tm = -1, b_loads = 0;
+      int stage = 0, cur_tm = -1;
       uint32_t phase = 0;
       long long issued = 0;
       bool ok = true;
+      // One k-block into the next stage of the ring.
+      auto load_kblock = [&](const CUtensorMap* map, int kx, int row, uint64_t pol) -> bool {
+        if (!mbar_wait(&tail->empty[stage], phase ^ 1u, timeout_ns, abort_flag)) {
+          merge_give_up(abort_flag);
+          return false;
+        }
+        mbar_arrive_expect_tx(&tail->full[stage], kMergeOperandBytes);
+        tma_load_2d(s_at + stage * kMergeOperandBytes, map, &tail->full[stage], kx, row, pol);
+        ++issued;
+        if (++stage == stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        return true;
+      };
       for (int t = t_begin, it = 0; ok && t < t_end; ++t, ++it) {
         const int tm = t / P.tiles_n, tn = t % P.tiles_n;
-        if (tm != cur_tm) {
-          if (b_loads > 0 &&
-              !mbar_wait(&tail->b_empty, static_cast<uint32_t>((b_loads - 1) & 1), timeout_ns,
-                         abort_flag)) {
-            merge_give_up(abort_flag);
-            break;
-          }
-          mbar_arrive_expect_tx(&tail->b_full, P.kb * kMergeOperandBytes);
-          for (int k = 0; k < P.kb; ++k)
-            tma_load_2d(s_b + k * kMergeOperandBytes, &P.tm_b, &tail->b_full, k * kMergeK,
-                        tm * kMergeM, pol_keep);
+        if (tm != cur_tm) {  // the row block's B tile, to be copied into TMEM
+          for (int k = 0; ok && k < P.kb; ++k)
+            ok = load_kblock(&P.tm_b, k * kMergeK, tm * kMergeM, pol_keep);
           cur_tm = tm;
-          ++b_loads;
         }
-        const int wb = it & 1;
-        if (!mbar_wait(&tail->w_empty[wb], static_cast<uint32_t>(((it >> 1) & 1) ^ 1), timeout_ns,
-                       abort_flag)) {
+        const int wb = it % wbufs;
+        if (!ok || !mbar_wait(&tail->w_empty[wb], static_cast<uint32_t>(((it / wbufs) & 1) ^ 1),
+                              timeout_ns, abort_flag)) {
           merge_give_up(abort_flag);
           break;
         }
@@ -201,21 +215,8 @@ __global__ void __launch_bounds__(kMergeThreads, 1)
         for (int h = 0; h < kMergeN / 64; ++h)
           tma_load_2d(s_w + wb * kMergeTileBytes + h * kMergeBoxBytes, &P.tm_w0, &tail->w_full[wb],
                       tn * kMergeN + h * 64, tm * kMergeM, pol_stream);
-        for (int k = 0; k < P.kb; ++k) {
-          if (!mbar_wait(&tail->empty[stage], phase ^ 1u, timeout_ns, abort_flag)) {
-            merge_give_up(abort_flag);
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&tail->full[stage], kMergeOperandBytes);
-          tma_load_2d(s_at + stage * kMergeOperandBytes, &P.tm_at, &tail->full[stage],
-                      k * kMergeK, tn * kMergeN, pol_keep);
-          ++issued;
-          if (++stage == stages) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
+        for (int k = 0; ok && k < P.kb; ++k)
+          ok = load_kblock(&P.tm_at, k * kMergeK, tn * kMergeN, pol_keep);
       }
       // Let every operand copy already issued land before the block can exit.
       const long long first = issued > stages ? issued - stages : 0;
@@ -223,23 +224,47 @@ __global__ void __launch_bounds__(kMergeThreads, 1)
         mbar_wait(&tail->full[j % stages], static_cast<uint32_t>((j / stages) & 1),
                   kDrainTimeoutNs, nullptr);
     }
-  } else if (warp == 5) {
+  } else if (warp == kMergeEpiWarps + 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && t_begin < t_end) {
-      int stage = 0, cur_tm = -1, b_loads = 0;
+      int stage = 0, cur_tm = -1, swaps = 0;
       uint32_t phase = 0;
       bool issued_any = false, ok = true;
+      const uint32_t b_tmem = tmem_base + kMergeTmemB;
       for (int t = t_begin, it = 0; ok && t < t_end; ++t, ++it) {
         const int tm = t / P.tiles_n;
         if (tm != cur_tm) {
-          if (b_loads > 0) umma_commit(&tail->b_empty);  // previous row block's MMAs
-          if (!mbar_wait(&tail->b_full, static_cast<uint32_t>(b_loads & 1), timeout_ns,
-                         abort_flag)) {
-            merge_give_up(abort_flag);
-            break;
+          // Overwrite the resident B tile only once every MMA reading it is done.
+          if (issued_any) {
+            umma_commit(&tail->b_swap);
+            if (!mbar_wait(&tail->b_swap, static_cast<uint32_t>(swaps & 1), timeout_ns,
+                           abort_flag)) {
+              merge_give_up(abort_flag);
+              break;
+            }
+            ++swaps;
+            tc_fence_after_sync();
           }
+          for (int k = 0; k < P.kb; ++k) {
+            if (!mbar_wait(&tail->full[stage], phase, timeout_ns, abort_flag)) {
+              merge_give_up(abort_flag);
+              ok = false;
+              break;
+            }
+            tc_fence_after_sync();
+            const uint32_t b0 = smem_addr(s_at + stage * kMergeOperandBytes);
+#pragma unroll
+            for (int kk = 0; kk < kMergeK / 16; ++kk)
+              tmem_copy_128x32B(b_tmem + static_cast<uint32_t>(k * 32 + kk * 8),
+                                sw128_kmajor_desc(b0 + kk * 32));
+            umma_commit(&tail->empty[stage]);
+            if (++stage == stages) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          if (!ok) break;
           cur_tm = tm;
-          ++b_loads;
         }
         const int ab = it & 1;
         if (!mbar_wait(&tail->acc_empty[ab], static_cast<uint32_t>(((it >> 1) & 1) ^ 1),
@@ -256,12 +281,11 @@ __global__ void __launch_bounds__(kMergeThreads, 1)
             break;
           }
           tc_fence_after_sync();
-          const uint32_t a0 = smem_addr(s_b + k * kMergeOperandBytes);
           const uint32_t b0 = smem_addr(s_at + stage * kMergeOperandBytes);
 #pragma unroll
           for (int kk = 0; kk < kMergeK / 16; ++kk)
-            umma_bf16(d_tmem, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32),
-                      P.idesc, (k > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16_tmem_a(d_tmem, b_tmem + static_cast<uint32_t>(k * 32 + kk * 8),
+                             sw128_kmajor_desc(b0 + kk * 32), P.idesc, (k > 0 || kk > 0) ? 1u : 0u);
           issued_any = true;
           umma_commit(&tail->empty[stage]);
           if (++stage == stages) {
@@ -278,19 +302,31 @@ __global__ void __launch_bounds__(kMergeThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------ epilogue (warps 0-3)
-    // Thread = row of the tile = TMEM lane; per 32-column chunk it reads the
-    // accumulator, the row's W0 values from the 128-byte-swizzled staging
-    // buffer, and writes W' over them.
-    const int row = threadIdx.x;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    bool stored_any = false;
+    // ------------------------------------------------ epilogue (warps 0-7)
+    // Warp w: TMEM lanes 32 (w % 4) .. + 31 (its rows) and the 64 columns of
+    // box w / 4 (two 32-column chunks).  Per chunk it reads the accumulator,
+    // the rows' W0 values from the 128-byte-swizzled staging buffer, and
+    // writes W' over them; then it stores its 32 x 64 sub-box with TMA itself
+    // and hands the staging buffer back (one arrival per warp) once that store
+    // has read it, at the start of its next tile.
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const int half = warp >> 2;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    int prev_wb = -1;
     for (int t = t_begin, it = 0; t < t_end; ++t, ++it) {
       const int tm = t / P.tiles_n, tn = t % P.tiles_n;
-      const int ab = it & 1;
+      const int ab = it & 1;  // accumulator
       const uint32_t par = static_cast<uint32_t>((it >> 1) & 1);
+      const int wb = it % wbufs;  // W0 / W' staging buffer
+      const uint32_t wpar = static_cast<uint32_t>((it / wbufs) & 1);
+      if (lane == 0 && prev_wb >= 0) {
+        bulk_wait_group_read0();
+        mbar_arrive(&tail->w_empty[prev_wb]);
+        prev_wb = -1;
+      }
       bool ok = mbar_wait(&tail->acc_full[ab], par, timeout_ns, abort_flag) &&
-                mbar_wait(&tail->w_full[ab], par, timeout_ns, abort_flag);
+                mbar_wait(&tail->w_full[wb], wpar, timeout_ns, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
         merge_give_up(abort_flag);
         break;
@@ -299,16 +335,17 @@ __global__ void __launch_bounds__(kMergeThreads, 1)
       const int grow = tm * kMergeM + row;
       float g = 0.f;
       if (grow < P.d_out) g = __fdiv_rn(__ldg(P.m + grow), fmaxf(__ldg(P.n + grow), P.eps));
-      uint8_t* wtile = s_w + ab * kMergeTileBytes;
+      uint8_t* box = s_w + wb * kMergeTileBytes + half * kMergeBoxBytes;
+      uint8_t* rowp = box + row * 128;
 #pragma unroll 1
-      for (int j = 0; j < kMergeN / 32; ++j) {
+      for (int jj = 0; jj < 2; ++jj) {
+        const int j = half * 2 + jj;  // 32-column chunk of the tile
         float acc[32];
         __syncwarp();
         tmem_load_32cols(tmem_base + lane_base + static_cast<uint32_t>(ab * kMergeN + j * 32), acc);
-        uint8_t* rowp = wtile + (j >> 1) * kMergeBoxBytes + row * 128;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int c = (j & 1) * 4 + q;  // 16-byte chunk of the 128-byte row
+          const int c = jj * 4 + q;  // 16-byte chunk of the 128-byte row
           uint4* p = reinterpret_cast<uint4*>(rowp + ((c ^ (row & 7)) << 4));
           const uint4 w = *p;
           const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
@@ -327,23 +364,15 @@ __global__ void __launch_bounds__(kMergeThreads, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&tail->acc_empty[ab]);
-        mbar_arrive(&tail->epi_done[ab]);
-      }
-      if (threadIdx.x == 0) {
-        if (!mbar_wait(&tail->epi_done[ab], par, timeout_ns, abort_flag)) {
-          merge_give_up(abort_flag);
-        } else {
-          for (int h = 0; h < kMergeN / 64; ++h)
-            tma_store_2d(&P.tm_out, wtile + h * kMergeBoxBytes, tn * kMergeN + h * 64,
-                         tm * kMergeM);
-          bulk_commit_group();
-          bulk_wait_group_read0();
-          stored_any = true;
-          mbar_arrive(&tail->w_empty[ab]);
-        }
+        // rows 32 quad .. + 31 of the box: 4 KiB, 1024-byte aligned, so the
+        // 128-byte swizzle pattern is the box's own
+        tma_store_2d(&P.tm_out, box + quad * 32 * 128, tn * kMergeN + half * 64,
+                     tm * kMergeM + quad * 32);
+        bulk_commit_group();
+        prev_wb = wb;
       }
     }
-    if (threadIdx.x == 0 && stored_any) bulk_wait_group0();
+    if (lane == 0) bulk_wait_group0();
   }
 
   __syncwarp();
@@ -351,7 +380,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1)
   __syncthreads();
   if (warp == 0) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, 2 * kMergeN);
+    tmem_dealloc(tmem_base, kMergeTmemCols);
   }
 }
 

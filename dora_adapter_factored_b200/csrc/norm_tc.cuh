@@ -704,8 +704,10 @@ template <bool kGrouped>
 __global__ void __launch_bounds__(256)
     gram_reduce_kernel(const __grid_constant__ GramProblemDev single,
                        const GramProblemDev* __restrict__ table) {
-  grid_dependency_wait();
+  // Let the norm GEMM launch now: its W0 k-blocks need nothing from the Gram,
+  // and it waits for this grid before it reads G' or the arrival counters.
   grid_dependency_trigger();
+  grid_dependency_wait();
   const GramProblemDev* P = kGrouped ? &table[blockIdx.z] : &single;
   if (blockIdx.x == 0 && blockIdx.y == 0)
     for (int k = threadIdx.x; k < P->cnt_len; k += blockDim.x) P->tile_cnt[k] = 0;
