@@ -258,20 +258,54 @@ void plan_module(int64_t d_out, int64_t d_in, int64_t r, ModulePlan& p) {
   p.S = std::max(1, std::min(by_k, by_sm));
 }
 
-// Largest number of stream-K segments on any tile of any module.
-int max_seg_slots(const std::vector<ModulePlan>& plans, long long total_units, int C) {
+// Re-read operands (A and G') of one stream-K wave of the grouped norm: well
+// inside the 126 MB L2, which also carries the W0 stream.
+constexpr size_t kWaveBudgetBytes = size_t(40) << 20;
+
+// Largest number of stream-K segments on any tile of any module; module i
+// lies in the wave starting at unit wave_of[i] with wave_units[i] units.
+int max_seg_slots(const std::vector<ModulePlan>& plans, const std::vector<long long>& wave_of,
+                  const std::vector<long long>& wave_units, int C) {
   int best = 1;
   long long begin = 0;
-  for (const auto& p : plans) {
+  for (size_t i = 0; i < plans.size(); ++i) {
+    const auto& p = plans[i];
     for (int t = 0; t < p.tiles; ++t) {
-      const long long x0 = begin + static_cast<long long>(t) * p.kb_tile;
-      const int c0 = first_cta_of_unit(x0, total_units, C);
-      const int c1 = first_cta_of_unit(x0 + p.kb_tile - 1, total_units, C);
+      const long long x0 = begin - wave_of[i] + static_cast<long long>(t) * p.kb_tile;
+      const int c0 = first_cta_of_unit(x0, wave_units[i], C);
+      const int c1 = first_cta_of_unit(x0 + p.kb_tile - 1, wave_units[i], C);
       best = std::max(best, c1 - c0 + 1);
     }
     begin += p.units;
   }
   return best;
+}
+
+// Splits the modules, in order, into stream-K waves: a wave closes before a
+// module that would take its re-read operands (A, G'_hi, G'_lo) past
+// `budget` bytes, provided it already holds at least `ctas` units; a last
+// wave smaller than that joins the one before.  Returns the waves' first
+// units (and the total at the end).
+std::vector<long long> plan_waves(const std::vector<ModulePlan>& plans, const int64_t* d_in,
+                                  const int64_t* r, long long total, int ctas, size_t budget) {
+  std::vector<long long> begin{0};
+  long long units = 0, at = 0;
+  size_t bytes = 0;
+  for (size_t i = 0; i < plans.size(); ++i) {
+    const size_t mb = static_cast<size_t>(r[i]) * d_in[i] * 2 +
+                      2 * static_cast<size_t>(r[i]) * plans[i].r8 * 2;
+    if (units > 0 && bytes + mb > budget && units >= ctas) {
+      begin.push_back(at);
+      units = 0;
+      bytes = 0;
+    }
+    units += plans[i].units;
+    at += plans[i].units;
+    bytes += mb;
+  }
+  if (begin.size() > 1 && total - begin.back() < ctas) begin.pop_back();
+  begin.push_back(total);
+  return begin;
 }
 
 struct GroupLayout {
@@ -281,6 +315,8 @@ struct GroupLayout {
   int seg_slots = 1;
   uint32_t b_region = 0;
   int tmem_cols = 32;
+  std::vector<long long> waves;                 // first unit of each wave, then the total
+  std::vector<long long> wave_of, wave_units;   // per module: its wave's first unit, units
   int stages = 0;
   size_t smem_bytes = 0;
   int gram_jobs = 0;
@@ -293,8 +329,20 @@ bool layout_group(const int64_t* d_out, const int64_t* d_in, const int64_t* r, i
                   bool grouped, int sms, GroupLayout& L) {
   L.plans.resize(count);
   L.total_units = 0;
+  for (int i = 0; i < count; ++i) plan_module(d_out[i], d_in[i], r[i], L.plans[i]);
+  if (grouped && count > 1) {
+    // K splits of the Gram for a group: the modules themselves give
+    // parallelism, so aim at about two waves of jobs of equal length over the
+    // whole group instead of filling the GPU with each module's splits.
+    long long work = 0;  // k-blocks over all (pair, k-block) of the group
+    for (const auto& p : L.plans) work += static_cast<long long>(p.pairs) * p.kb_gram;
+    const long long per_job = std::max(1ll, ceil_div_ll(work, 2ll * sms));
+    for (auto& p : L.plans) {
+      const long long by_len = std::max(1ll, (p.kb_gram + per_job / 2) / per_job);
+      p.S = static_cast<int>(std::min<long long>(by_len, std::max(1, p.kb_gram / 8)));
+    }
+  }
   for (int i = 0; i < count; ++i) {
-    plan_module(d_out[i], d_in[i], r[i], L.plans[i]);
     L.total_units += L.plans[i].units;
     L.b_region = std::max(L.b_region, L.plans[i].b_region);
     L.tmem_cols = std::max(L.tmem_cols, L.plans[i].tmem_cols);
@@ -303,7 +351,25 @@ bool layout_group(const int64_t* d_out, const int64_t* d_in, const int64_t* r, i
   }
   L.ctas = static_cast<int>(std::min<long long>(sms, L.total_units));
   if (L.ctas < 1) return false;
-  L.seg_slots = max_seg_slots(L.plans, L.total_units, L.ctas);
+  {
+    size_t budget = grouped ? kWaveBudgetBytes : SIZE_MAX;
+    L.waves = plan_waves(L.plans, d_in, r, L.total_units, L.ctas, budget);
+    while (static_cast<int>(L.waves.size()) - 1 > kMaxWaves) {
+      budget *= 2;
+      L.waves = plan_waves(L.plans, d_in, r, L.total_units, L.ctas, budget);
+    }
+    L.wave_of.resize(count);
+    L.wave_units.resize(count);
+    long long at = 0;
+    size_t w = 0;
+    for (int i = 0; i < count; ++i) {
+      while (at >= L.waves[w + 1]) ++w;
+      L.wave_of[i] = L.waves[w];
+      L.wave_units[i] = L.waves[w + 1] - L.waves[w];
+      at += L.plans[i].units;
+    }
+  }
+  L.seg_slots = max_seg_slots(L.plans, L.wave_of, L.wave_units, L.ctas);
   const uint32_t stage_bytes = kTileABytes + L.b_region;
   const int tail_bytes = static_cast<int>(align_up(sizeof(NormSmemTail), 128));
   L.stages = std::min<int>(kMaxStages, (kMaxDynSmem - 1024 - tail_bytes) / stage_bytes);
@@ -463,11 +529,16 @@ dora_status_t run_tc_group(const dora_norm_problem_t* probs, int count, bool gro
     if (!fill_descriptors(probs[i], L.plans[i], base, ub, jb, nds[i], gds[i]))
       return DORA_ERR_INVALID_ARG;
     nds[i].emit_sq = emit_sq ? 1 : 0;
+    nds[i].wave_begin = L.wave_of[i];
+    nds[i].wave_units = L.wave_units[i];
     ub += L.plans[i].units;
     jb += L.plans[i].pairs * L.plans[i].S;
   }
   const unsigned long long tmo = g_timeout_ns.load();
   const int gram_smem = 1024 + kGramStages * kGramStageBytes + 256;
+  static thread_local WaveList wl;
+  wl.n = static_cast<int>(L.waves.size()) - 1;
+  for (int w = 0; w <= wl.n; ++w) wl.begin[w] = L.waves[w];
   dora_status_t s;
   const dim3 red_grid(kTileM * kTileM / 256, L.max_pairs, grouped ? count : 1);
   if (!grouped) {
@@ -481,7 +552,7 @@ dora_status_t run_tc_group(const dora_norm_problem_t* probs, int count, bool gro
       TimedLaunch tl(st);
       launch_pdl(norm_main_kernel<false>, dim3(L.ctas), dim3(kNormThreads), L.smem_bytes, st,
                  nds[0], static_cast<const NormProblemDev*>(nullptr), 1, L.total_units, L.stages,
-                 L.b_region, static_cast<uint32_t>(L.tmem_cols), eps, tmo, g_trace);
+                 L.b_region, static_cast<uint32_t>(L.tmem_cols), eps, wl, tmo, g_trace);
       return launch_status();
     }
   }
@@ -503,7 +574,7 @@ dora_status_t run_tc_group(const dora_norm_problem_t* probs, int count, bool gro
     TimedLaunch tl(st);
     launch_pdl(norm_main_kernel<true>, dim3(L.ctas), dim3(kNormThreads), L.smem_bytes, st, nds[0],
                static_cast<const NormProblemDev*>(ntab), count, L.total_units, L.stages,
-               L.b_region, static_cast<uint32_t>(L.tmem_cols), eps, tmo, g_trace);
+               L.b_region, static_cast<uint32_t>(L.tmem_cols), eps, wl, tmo, g_trace);
     return launch_status();
   }
 }

@@ -68,6 +68,7 @@ struct alignas(64) NormProblemDev {
   float* n_out;          // [d_out]
   float* g_out;          // [d_out] or null
   long long unit_begin;  // first global stream-K unit of this problem
+  long long wave_begin, wave_units;  // the stream-K wave holding this problem
   int d_out, r;
   int n0, n1;            // N of the two accumulator chunks (n1 = 0: single chunk)
   int box_rows, nbox;    // N-side operand: boxes per stage and rows per box
@@ -90,8 +91,20 @@ struct alignas(64) GramProblemDev {
   float half_s;
 };
 
+// Waves: the grouped call splits its modules (in order) into waves whose
+// operands that every tile re-reads (A and G') fit in L2 together, and runs
+// stream-K over one wave at a time across all CTAs.  begin[w] .. begin[w+1]
+// are wave w's global units; one module alone is one wave.  Every wave has at
+// least as many units as there are CTAs, so no CTA's share of a wave is empty.
+constexpr int kMaxWaves = 64;
+struct WaveList {
+  int n;
+  long long begin[kMaxWaves + 1];
+};
+
 // ---------------------------------------------------------------------------
-// Stream-K bookkeeping.  CTA c of C owns global units [c U / C, (c+1) U / C).
+// Stream-K bookkeeping (per wave, U = the wave's units, X relative to the
+// wave's first unit).  CTA c of C owns units [c U / C, (c+1) U / C).
 // The CTAs that touch the tile starting at unit X are first_cta(X) ..
 // first_cta(X + kb_tile - 1); the segment of CTA c on that tile goes to slot
 // c - first_cta(X).
@@ -190,7 +203,8 @@ __global__ void __maxnreg__(kNormMaxRegs)
     norm_main_kernel(const __grid_constant__ NormProblemDev single,
                      const NormProblemDev* __restrict__ table, int nprob, long long total_units,
                      int stages, uint32_t b_region, uint32_t tmem_cols, float eps,
-                     unsigned long long timeout_ns, unsigned long long* __restrict__ trace) {
+                     const __grid_constant__ WaveList waves, unsigned long long timeout_ns,
+                     unsigned long long* __restrict__ trace) {
   // trace (optional, diagnostics): per CTA 8 words -- entry and exit global
   // time, MMA-issuer cycles waiting for data / for the accumulator, issued
   // k-blocks, segments, SM id.
@@ -207,8 +221,13 @@ __global__ void __maxnreg__(kNormMaxRegs)
   const int lane = threadIdx.x & 31;
   const int C = gridDim.x;
   const int cta = blockIdx.x;
-  const long long u_begin = static_cast<long long>(cta) * total_units / C;
-  const long long u_end = static_cast<long long>(cta + 1) * total_units / C;
+  (void)total_units;
+  // This CTA's units of wave w.
+  auto wave_range = [&](int w, long long& ub, long long& ue) {
+    const long long b = waves.begin[w], U = waves.begin[w + 1] - b;
+    ub = b + static_cast<long long>(cta) * U / C;
+    ue = b + static_cast<long long>(cta + 1) * U / C;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
@@ -252,6 +271,10 @@ __global__ void __maxnreg__(kNormMaxRegs)
       uint32_t phase = 0;
       long long issued = 0;
       bool waited = false;  // G' (written by the preceding kernel) is visible
+      bool ok = true;
+      for (int wv = 0; ok && wv < waves.n; ++wv) {
+      long long u_begin, u_end;
+      wave_range(wv, u_begin, u_end);
       if (u_begin < u_end) cur.start(u_begin);
       for (long long u = u_begin; u < u_end; ++u, ++cur.local) {
         cur.settle(u);
@@ -260,6 +283,7 @@ __global__ void __maxnreg__(kNormMaxRegs)
         const int kb = cur.kblock();
         if (!mbar_wait(&empty[stage], phase ^ 1u, timeout_ns, abort_flag)) {
           give_up(abort_flag);
+          ok = false;
           break;
         }
         uint8_t* sa = smem + stage * stage_bytes;
@@ -298,6 +322,7 @@ __global__ void __maxnreg__(kNormMaxRegs)
           phase ^= 1u;
         }
       }
+      }
       if (!waited) {
         grid_dependency_wait();
         grid_dependency_trigger();
@@ -310,14 +335,18 @@ __global__ void __maxnreg__(kNormMaxRegs)
     }
   } else if (warp == kEpiWarps + 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && u_begin < u_end) {
+    if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool issued_any = false;
       long long wait_data = 0, wait_acc = 0, nseg = 0, nkb = 0;
+      bool ok = true;
+      for (int wv = 0; ok && wv < waves.n; ++wv) {
+      long long u_begin, u_end;
+      wave_range(wv, u_begin, u_end);
+      if (u_begin >= u_end) continue;
       cur.start(u_begin);
       long long u = u_begin;
-      bool ok = true;
       while (ok && u < u_end) {
         cur.settle(u);
         const NormProblemDev* P = cur.P;
@@ -326,6 +355,7 @@ __global__ void __maxnreg__(kNormMaxRegs)
         const long long c0 = clock64();
         if (!mbar_wait(&tail->acc_empty, acc_phase ^ 1u, timeout_ns, abort_flag)) {
           give_up(abort_flag);
+          ok = false;
           break;
         }
         wait_acc += clock64() - c0;
@@ -367,6 +397,7 @@ __global__ void __maxnreg__(kNormMaxRegs)
         umma_commit(&tail->acc_full);
         acc_phase ^= 1u;
       }
+      }
       if (issued_any) {
         umma_commit(&tail->drain);
         mbar_wait(&tail->drain, 0, kDrainTimeoutNs, nullptr);
@@ -389,10 +420,13 @@ __global__ void __maxnreg__(kNormMaxRegs)
     int stage = 0;
     uint32_t phase = 0, acc_phase = 0, seg_count = 0;
     bool dep_waited = false;
-    if (u_begin < u_end) {
+    bool ok = true;
+    for (int wv = 0; ok && wv < waves.n; ++wv) {
+      long long u_begin, u_end;
+      wave_range(wv, u_begin, u_end);
+      if (u_begin >= u_end) continue;
       cur.start(u_begin);
       long long u = u_begin;
-      bool ok = true;
       while (ok && u < u_end) {
         cur.settle(u);
         const NormProblemDev* P = cur.P;
@@ -446,6 +480,7 @@ __global__ void __maxnreg__(kNormMaxRegs)
         if (!ok) break;
         if (!mbar_wait(&tail->acc_full, acc_phase, timeout_ns, abort_flag)) {
           give_up(abort_flag);
+          ok = false;
           break;
         }
         tc_fence_after_sync();
@@ -486,11 +521,12 @@ __global__ void __maxnreg__(kNormMaxRegs)
           mbar_arrive(&tail->acc_empty);
           if (!__all_sync(0xffffffffu, got_one)) {
             give_up(abort_flag);
+            ok = false;
             break;
           }
-          const long long x0 = P->unit_begin + static_cast<long long>(t) * P->kb_tile;
-          const int c0 = first_cta_of_unit(x0, total_units, C);
-          const int nseg = first_cta_of_unit(x0 + P->kb_tile - 1, total_units, C) - c0 + 1;
+          const long long x0 = P->unit_begin - P->wave_begin + static_cast<long long>(t) * P->kb_tile;
+          const int c0 = first_cta_of_unit(x0, P->wave_units, C);
+          const int nseg = first_cta_of_unit(x0 + P->kb_tile - 1, P->wave_units, C) - c0 + 1;
           float* part_t = P->partial + static_cast<size_t>(t) * P->seg_slots * kTileM + row;
           if (valid) part_t[static_cast<size_t>(cta - c0) * kTileM] = part + other;
           // The last of the tile's segments to post its partials (per warp:
