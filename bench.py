@@ -902,12 +902,130 @@ def run_suite(args):
     return 0
 
 
+# --------------------------------------------------------------------------- single cases
+
+CASES = ("merge", "fwd_train", "bwd_inner", "bwd_frozen", "fwd_grouped", "bwd_grouped",
+         "norm_grouped", "norm_sq_shard")
+
+
+def run_case(args):
+    """One API call, repeated on two rotating input sets (each larger than L2
+    except where noted): the headline module / activations for the merge, the
+    training and frozen compose variants and the d_in shard; one decoder
+    layer (7 modules, [2048, d_out] activations) for the grouped compose;
+    one layer's 7 modules for the grouped norm."""
+    import torch
+    import dora_adapter_factored_b200 as dora
+    from dora_adapter_factored_b200 import synth
+    dev = torch.device("cuda")
+    eps = synth.eps_for("bf16")
+    w = synth.WORKLOADS[WORKLOAD]
+    ms = w.modules[0]
+    name = args.case
+    if name in ("merge", "norm_sq_shard"):
+        W0, A, B = synth.module_weights(w, device=dev)
+        sets = [(W0, A, B), (W0.flip(0).contiguous(), A, B.flip(0).contiguous())]
+        if name == "merge":
+            ns = [dora.dora_factored_norm(*x, ms.s)[0] for x in sets]
+            out = torch.empty_like(W0)
+            ws = torch.empty(dora.dora_merge_weight_workspace_size(ms.d_out, ms.d_in, ms.r),
+                             dtype=torch.uint8, device=dev)
+            fn = lambda i: dora.dora_merge_weight(*sets[i % 2], ns[i % 2] * 1.001, ns[i % 2], ms.s,
+                                                  eps, W_out=out, ws=ws)
+        else:
+            a, b = dora.column_shard(ms.d_in, 0, 2)
+            sh = [(x[0][:, a:b].contiguous(), x[1][:, a:b].contiguous(), x[2]) for x in sets]
+            sq = torch.empty(ms.d_out, device=dev)
+            ws = torch.empty(dora.dora_factored_norm_workspace_size(ms.d_out, b - a, ms.r,
+                                                                   torch.bfloat16),
+                             dtype=torch.uint8, device=dev)
+            fn = lambda i: dora.dora_factored_norm_sq(*sh[i % 2], ms.s, sq_out=sq, ws=ws)
+    elif name in ("fwd_train", "bwd_inner", "bwd_frozen"):
+        T, d = w.tokens, ms.d_out
+        sets = []
+        for k in range(2):
+            base, lora, dy = synth.activations(w, T, d, device=dev, index=k)
+            n = torch.full((d,), 1.3, device=dev)
+            sets.append(dict(base=base, lora=lora, dy=dy, inner=torch.empty_like(base), n=n,
+                             m=n * 1.001))
+        y, db, dl = (torch.empty(T, d, dtype=torch.bfloat16, device=dev) for _ in range(3))
+        dm = torch.empty(d, device=dev)
+        ws = torch.empty(dora.dora_compose_bwd_workspace_size(T, d, torch.bfloat16),
+                         dtype=torch.uint8, device=dev)
+        if name == "fwd_train":
+            fn = lambda i: dora.dora_compose_fwd_train(
+                sets[i % 2]["base"], sets[i % 2]["lora"], sets[i % 2]["m"], sets[i % 2]["n"], ms.s,
+                eps, y=y, inner=sets[i % 2]["inner"])
+        elif name == "bwd_inner":
+            fn = lambda i: dora.dora_compose_bwd_inner(
+                sets[i % 2]["dy"], sets[i % 2]["base"], sets[i % 2]["m"], sets[i % 2]["n"], ms.s,
+                eps, d_base=db, d_lora=dl, dm=dm, ws=ws)
+        else:
+            fn = lambda i: dora.dora_compose_bwd_frozen(
+                sets[i % 2]["dy"], sets[i % 2]["m"], sets[i % 2]["n"], ms.s, eps, d_base=db,
+                d_lora=dl)
+    elif name in ("fwd_grouped", "bwd_grouped"):
+        T = 2048
+        groups = []
+        for k in range(2):
+            items = []
+            for i, d in enumerate((4096, 1024, 1024, 4096, 14336, 14336, 4096)):
+                g = torch.Generator(device=dev).manual_seed(100 * k + i)
+                t = {x: torch.randn(T, d, device=dev, generator=g).bfloat16()
+                     for x in ("base", "lora", "dy")}
+                n = torch.full((d,), 1.3, device=dev)
+                if name == "fwd_grouped":
+                    items.append(dict(base=t["base"], lora=t["lora"], m=n * 1.001, n=n, s=2.0,
+                                      y=torch.empty_like(t["base"])))
+                else:
+                    items.append(dict(dy=t["dy"], base=t["base"], lora=t["lora"], m=n * 1.001,
+                                      n=n, s=2.0, d_base=torch.empty_like(t["base"]),
+                                      d_lora=torch.empty_like(t["base"]),
+                                      dm=torch.empty(d, device=dev)))
+            groups.append(items)
+        if name == "fwd_grouped":
+            fn = lambda i: dora.dora_compose_fwd_grouped(groups[i % 2], eps)
+        else:
+            gws = torch.empty(max(256, dora.dora_compose_bwd_grouped_workspace_size(groups[0])),
+                              dtype=torch.uint8, device=dev)
+            fn = lambda i: dora.dora_compose_bwd_grouped(groups[i % 2], eps, ws=gws)
+    else:  # norm_grouped: one layer (7 modules) of the layer stack
+        ws_ = synth.WORKLOADS["layer_stack_56"]
+        mods = []
+        for i, m_ in enumerate(ws_.modules[:7]):
+            W0, A, B = synth.module_weights(ws_, index=i, device=dev)
+            mods.append(dict(W0=W0, A=A, B=B, s=m_.s, n_out=torch.empty(m_.d_out, device=dev)))
+        ws = torch.empty(dora.dora_factored_norm_grouped_workspace_size(mods), dtype=torch.uint8,
+                         device=dev)
+        fn = lambda i: dora.dora_factored_norm_grouped(mods, ws=ws)
+    for i in range(args.warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for i in range(args.steps):
+        evs[i][0].record(st)
+        fn(i)
+        evs[i][1].record(st)
+    torch.cuda.synchronize()
+    if dora.dora_get_device_status() != 0:
+        raise RuntimeError("a kernel reported an error")
+    us = statistics.median(a.elapsed_time(b) for a, b in evs) * 1e3
+    print(json.dumps({"case": name, "us": us, "steps": args.steps, "warmup": args.warmup}),
+          flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--case", default=None, choices=sorted(CASES),
+                    help="run one API call on its workload (steps + warmup times) and print "
+                         "its median device time: a small, fixed command for kernel profiles")
     ap.add_argument("--suite", action="store_true",
                     help="instead of the headline line: one JSON line per further workload "
                          "(the other configurations and the training / grouped / merge / "
@@ -921,6 +1039,8 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     with torch.cuda.stream(torch.cuda.Stream()):  # a non-default stream for the whole run
+        if args.case:
+            return run_case(args)
         if args.suite:
             return run_suite(args)
         return run_gpu(args)
