@@ -85,11 +85,11 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
-// Waits until the bulk stores committed so far have finished reading shared memory.
-__device__ __forceinline__ void bulk_wait_group_read0() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+// Waits until every bulk store group committed so far but the most recent one
+// has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_group_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
-
 __device__ __forceinline__ void bulk_wait_group0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
@@ -306,24 +306,30 @@ __global__ void __launch_bounds__(kMergeThreads, 1)
     // Warp w: TMEM lanes 32 (w % 4) .. + 31 (its rows) and the 64 columns of
     // box w / 4 (two 32-column chunks).  Per chunk it reads the accumulator,
     // the rows' W0 values from the 128-byte-swizzled staging buffer, and
-    // writes W' over them; then it stores its 32 x 64 sub-box with TMA itself
-    // and hands the staging buffer back (one arrival per warp) once that store
-    // has read it, at the start of its next tile.
+    // writes W' over them; then it stores its 32 x 64 sub-box with TMA itself.
+    // A staging buffer goes back to the producer (one arrival per warp) two
+    // tiles later, once that store has read it -- by then it has, so the
+    // storing lane does not hold its warp.  g depends on the row block only.
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const int half = warp >> 2;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    int prev_wb = -1;
+    int g_tm = -1;
+    float g = 0.f;
     for (int t = t_begin, it = 0; t < t_end; ++t, ++it) {
       const int tm = t / P.tiles_n, tn = t % P.tiles_n;
       const int ab = it & 1;  // accumulator
       const uint32_t par = static_cast<uint32_t>((it >> 1) & 1);
       const int wb = it % wbufs;  // W0 / W' staging buffer
       const uint32_t wpar = static_cast<uint32_t>((it / wbufs) & 1);
-      if (lane == 0 && prev_wb >= 0) {
-        bulk_wait_group_read0();
-        mbar_arrive(&tail->w_empty[prev_wb]);
-        prev_wb = -1;
+      if (lane == 0 && it >= 2) {
+        bulk_wait_group_read1();  // tile it-2's store has read its buffer
+        mbar_arrive(&tail->w_empty[(it - 2) % wbufs]);
+      }
+      if (tm != g_tm) {
+        const int grow = tm * kMergeM + row;
+        g = grow < P.d_out ? __fdiv_rn(__ldg(P.m + grow), fmaxf(__ldg(P.n + grow), P.eps)) : 0.f;
+        g_tm = tm;
       }
       bool ok = mbar_wait(&tail->acc_full[ab], par, timeout_ns, abort_flag) &&
                 mbar_wait(&tail->w_full[wb], wpar, timeout_ns, abort_flag);
@@ -332,9 +338,6 @@ __global__ void __launch_bounds__(kMergeThreads, 1)
         break;
       }
       tc_fence_after_sync();
-      const int grow = tm * kMergeM + row;
-      float g = 0.f;
-      if (grow < P.d_out) g = __fdiv_rn(__ldg(P.m + grow), fmaxf(__ldg(P.n + grow), P.eps));
       uint8_t* box = s_w + wb * kMergeTileBytes + half * kMergeBoxBytes;
       uint8_t* rowp = box + row * 128;
 #pragma unroll 1
@@ -369,7 +372,6 @@ __global__ void __launch_bounds__(kMergeThreads, 1)
         tma_store_2d(&P.tm_out, box + quad * 32 * 128, tn * kMergeN + half * 64,
                      tm * kMergeM + quad * 32);
         bulk_commit_group();
-        prev_wb = wb;
       }
     }
     if (lane == 0) bulk_wait_group0();
