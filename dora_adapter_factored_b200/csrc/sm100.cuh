@@ -67,41 +67,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
-// ---------------------------------------------------------------- clusters
-
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-// Every thread of every CTA of the cluster (a hardware barrier: the kernels
-// that use it reach it on every path, the same number of times).
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
-}
-
-// Address of the same shared-memory object in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t map_shared_rank(const void* p, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
-  return r;
-}
-
-// Loads from another CTA's shared memory.  No memory clobber, so that several
-// can be in flight; callers order them against writes with cluster barriers.
-__device__ __forceinline__ float4 ld_shared_cluster_f4(uint32_t cluster_addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(cluster_addr));
-  return v;
-}
-
 // ---------------------------------------------------------------- PDL
-// Programmatic dependent launch: wait for the preceding grid (and, through
-// its own wait, everything before it) to complete and be visible; allow the
-// next grid to launch.  Every kernel of the library waits before it triggers.
+// Programmatic dependent launch: wait for the preceding grid to complete and
+// its writes to be visible; allow the next grid to launch.
 __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
