@@ -1017,7 +1017,7 @@ dora_status_t dora_compose_bwd_frozen(const void* dy, const float* m, const floa
 namespace dora {
 namespace {
 struct MergeLayout {
-  int kb, stages, wbufs, tiles_m, tiles_n, r8;
+  int kb, stages, tiles_m, tiles_n, r8;
   size_t smem_bytes, ws_bytes;
 };
 
@@ -1027,15 +1027,14 @@ bool merge_layout(int64_t d_out, int64_t d_in, int64_t r, MergeLayout& L) {
   L.r8 = round_up_int(static_cast<int>(r), 8);
   L.tiles_m = static_cast<int>(ceil_div_ll(d_out, kMergeM));
   L.tiles_n = static_cast<int>(ceil_div_ll(d_in, kMergeN));
-  // Shared memory: W0 / W' staging buffers (the HBM stream: several tiles in
-  // flight) and k-block stages (the L2 stream of A^T), 4 + 6 at the limit.
+  // Shared memory: two W0 / W' staging tiles and as many 32 KiB k-block
+  // stages (A^T, or B while a row block starts) as fit: three.
   const size_t tail = align_up(sizeof(MergeSmemTail), 128);
-  L.wbufs = kMergeMaxWBufs;
-  const size_t fixed = 1024 + static_cast<size_t>(L.wbufs) * kMergeTileBytes + tail;
-  if (fixed + 2 * kMergeOperandBytes > static_cast<size_t>(kMaxDynSmem)) return false;
+  const size_t fixed = 1024 + static_cast<size_t>(kMergeWBufs) * kMergeTileBytes + tail;
+  if (fixed + 2 * kMergeStageBytes > static_cast<size_t>(kMaxDynSmem)) return false;
   L.stages = static_cast<int>(std::min<size_t>(kMergeMaxStages,
-                                               (kMaxDynSmem - fixed) / kMergeOperandBytes));
-  L.smem_bytes = fixed + static_cast<size_t>(L.stages) * kMergeOperandBytes;
+                                               (kMaxDynSmem - fixed) / kMergeStageBytes));
+  L.smem_bytes = fixed + static_cast<size_t>(L.stages) * kMergeStageBytes;
   L.ws_bytes = align_up(static_cast<size_t>(d_in) * L.r8 * 2, 256);
   return true;
 }
@@ -1084,7 +1083,7 @@ dora_status_t dora_merge_weight(const void* W0, const void* A, const void* B, co
   ok &= make_tmap_bf16(&P.tm_w0, W0, d_out, d_in, d_in, 64, kMergeM);
   ok &= make_tmap_bf16(&P.tm_out, W_out, d_out, d_in, d_in, 64, 32);
   ok &= make_tmap_bf16(&P.tm_b, B, d_out, r, r, kMergeK, kMergeM);
-  ok &= make_tmap_bf16(&P.tm_at, At, d_in, r, L.r8, kMergeK, kMergeN);
+  ok &= make_tmap_bf16(&P.tm_at, At, d_in, r, L.r8, kMergeK, kMergeN);  // 256-row boxes
   if (!ok) return DORA_ERR_INVALID_ARG;
   P.m = m;
   P.n = n;
@@ -1106,7 +1105,7 @@ dora_status_t dora_merge_weight(const void* W0, const void* A, const void* B, co
   const int ctas = std::min(di->sms, P.tiles);
   TimedLaunch tl(cs);
   launch_pdl(merge_kernel, dim3(ctas), dim3(kMergeThreads), L.smem_bytes, cs, P, L.stages,
-             L.wbufs, g_timeout_ns.load());
+             g_timeout_ns.load());
   return launch_status();
 }
 
