@@ -18,6 +18,8 @@ from ._abi import (  # noqa: F401
     load_library, status_string,
 )
 
-from .sharded import column_shard, sharded_factored_norm  # noqa: F401,E402
+from .sharded import (  # noqa: F401,E402
+    all_gather_rows, column_shard, module_shard, row_shard, sharded_factored_norm,
+)
 
 __version__ = "0.1.0"

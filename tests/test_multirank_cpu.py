@@ -1,7 +1,9 @@
 """Multi-process host logic on CPU (gloo, world size 2): the d_in-sharded norm's
-column split and its all-reduce of squared partials, and the bench's
-cross-rank timing helpers (barrier, max over ranks).  Each rank is a spawned
-process; the oracle stands in for the GPU partial (there is no GPU here)."""
+column split and its all-reduce of squared partials, the row-sharded norm's
+all-gather, the module split of a grouped call, the bench's cross-rank timing
+helpers (barrier, max over ranks), and a rank that fails before a collective.
+Each rank is a spawned process; the oracle stands in for the GPU calls (there
+is no GPU here)."""
 import datetime
 import os
 import socket
@@ -39,6 +41,15 @@ def _sharded_norm(rank, world):
     return np.sqrt(np.maximum(sq.numpy(), 0.0))
 
 
+def _row_sharded_norm(rank, world):
+    import oracle
+    from dora_adapter_factored_b200.sharded import all_gather_rows, row_shard
+    W0, A, B = _module(d_out=37)
+    a, b = row_shard(37, rank, world, align=8)
+    n_local = torch.from_numpy(oracle.dense_row_norm(W0[a:b], A, B[a:b], 1.5))
+    return all_gather_rows(n_local, 37, align=8).numpy()
+
+
 def _bench_helpers(rank, world):
     import bench
     bench.barrier(dist, 0)
@@ -60,8 +71,8 @@ def _failing_rank(rank, world):
     return "completed"
 
 
-FNS = {"sharded_norm": _sharded_norm, "bench_helpers": _bench_helpers,
-       "failing_rank": _failing_rank}
+FNS = {"sharded_norm": _sharded_norm, "row_sharded_norm": _row_sharded_norm,
+       "bench_helpers": _bench_helpers, "failing_rank": _failing_rank}
 
 
 def _worker(rank, world, port, name, timeout_s, q):
@@ -126,6 +137,34 @@ def test_sharded_norm_all_reduce_two_ranks():
         status, n = out[rank]
         assert status == "ok", n
         np.testing.assert_allclose(n, dense, rtol=1e-12)
+
+
+def test_row_sharded_norm_all_gather_two_ranks():
+    import oracle
+    out = _run("row_sharded_norm")
+    W0, A, B = _module(d_out=37)
+    dense = oracle.dense_row_norm(W0, A, B, 1.5)
+    for rank in range(WORLD):
+        status, n = out[rank]
+        assert status == "ok", n
+        np.testing.assert_array_equal(n, dense)
+
+
+def test_module_shard_balances_and_covers():
+    from dora_adapter_factored_b200.sharded import module_shard
+    rng = np.random.default_rng(5)
+    for world in (1, 2, 3, 8):
+        flops = list(rng.uniform(1, 10, 56))
+        parts = module_shard(flops, world)
+        assert sorted(i for p in parts for i in p) == list(range(56))
+        assert all(p == sorted(p) for p in parts)
+        loads = [sum(flops[i] for i in p) for p in parts]
+        assert max(loads) <= sum(flops) / world + max(flops) + 1e-9
+        assert module_shard(flops, world) == parts  # deterministic
+    # a decoder layer's seven modules on three ranks: each gets a share
+    layer = [2 * 4096 * 4096, 2 * 1024 * 4096, 2 * 1024 * 4096, 2 * 4096 * 4096,
+             2 * 14336 * 4096, 2 * 14336 * 4096, 2 * 4096 * 14336]
+    assert all(module_shard(layer, 3))
 
 
 def test_bench_rank_helpers_two_ranks():

@@ -116,3 +116,18 @@ def test_sharded_norm_through_a_one_rank_nccl_group():
                        text=True, timeout=240, env=env)
     assert r.returncode == 0, r.stderr[-2000:]
     assert "SAME" in r.stdout, r.stdout
+
+
+def test_row_shards_on_one_gpu():
+    """Row sharding: each rank's block of rows is an independent norm call;
+    the blocks put together equal the oracle's norm of the whole module."""
+    W0, A, B = _module(1000, 512, 64, torch.bfloat16, 41)
+    s, parts = 2.0, []
+    for rank in range(3):
+        a, b = dora.row_shard(1000, rank, 3)
+        n, _ = dora.dora_factored_norm(W0[a:b].contiguous().cuda(), A.cuda(),
+                                       B[a:b].contiguous().cuda(), s)
+        parts.append(n)
+    torch.cuda.synchronize()
+    ref = oracle.dense_row_norm(_np(W0), _np(A), _np(B), s)
+    check_rel(_np(torch.cat(parts)), ref, 1e-3, "n from row shards")
