@@ -49,8 +49,10 @@ struct StreamGrid {
 };
 
 // `slots`: blocks the grid aims at (a module of a grouped launch gets its
-// share of the launch's slots).
-inline StreamGrid stream_grid(long long T, int ncv, int unroll, long long slots = kStreamSlots) {
+// share of the launch's slots).  `bx_fixed` > 0 sets the block's width in
+// column vectors; otherwise the widest with the fewest idle columns.
+inline StreamGrid stream_grid(long long T, int ncv, int unroll, long long slots = kStreamSlots,
+                              int bx_fixed = 0) {
   StreamGrid g;
   int best = 256;
   long long best_waste = -1;
@@ -61,8 +63,8 @@ inline StreamGrid stream_grid(long long T, int ncv, int unroll, long long slots 
       best_waste = waste;
     }
   }
-  g.bx = best;
-  g.by = kStreamThreads / best;
+  g.bx = bx_fixed > 0 ? bx_fixed : best;
+  g.by = kStreamThreads / g.bx;
   g.gx = static_cast<int>(ceil_div_ll(ncv, g.bx));
   long long want_y = slots / g.gx;
   if (want_y < 1) want_y = 1;

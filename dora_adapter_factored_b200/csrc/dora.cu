@@ -862,7 +862,12 @@ BwdShape bwd_shape(int64_t T, int64_t d_out, dora_dtype_t dt, bool aligned, int 
   BwdShape b;
   const int v = dt == DORA_BF16 ? 8 : 4;
   b.vec = (aligned && d_out % v == 0) ? v : 1;
-  b.g = stream_grid(T, static_cast<int>(d_out / b.vec), unroll);
+  // Blocks 32 vectors wide when the columns divide evenly: the backward then
+  // has few row chunks (9 at d_out = 8192 rather than 74), so the dm
+  // finalize sums few partials per column; measured 0.3-7 % faster per call
+  // than the widest blocks, most on [8192, 25600] and [2048, 4096].
+  const int ncv = static_cast<int>(d_out / b.vec);
+  b.g = stream_grid(T, ncv, unroll, kStreamSlots, ncv % 32 == 0 ? 32 : 0);
   return b;
 }
 
