@@ -197,6 +197,10 @@ def test_workspace_sizes_are_host_computable(built_library):
     wb = lib.dora_compose_bwd_workspace_size(8192, 25600, _abi.DORA_BF16)
     assert 25600 * 4 <= wb < 64 << 20
     assert lib.dora_compose_bwd_workspace_size(0, 16, _abi.DORA_BF16) >= 0
+    # the backward's blocks are 32 vectors (256 bf16 columns) wide: at the
+    # headline shape 32 column blocks x 9 row chunks fill the 296 block slots,
+    # so the workspace holds 9 rows of d_out fp32 partials
+    assert lib.dora_compose_bwd_workspace_size(4096, 8192, _abi.DORA_BF16) == 9 * 8192 * 4
 
 
 def test_binding_rejects_cpu_tensors(built_library):
