@@ -1033,6 +1033,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
+    if args.steps < 1:
+        raise SystemExit("--steps must be at least 1")
     if args.impl == "reference":
         return run_reference(args)
     import torch
