@@ -167,28 +167,25 @@ def max_over_ranks(pg, x: float) -> float:
 
 # --------------------------------------------------------------------------- oracle arm
 
-def oracle_step_seconds(W0, A, B, m, base, lora, dy, s, eps, rows, tokens, T_full=4096):
-    """Times the fp64 oracle on a sample (`rows` rows of the norm, `tokens` rows
-    of the compose) and scales it to the full step."""
-    import numpy as np
+def oracle_step_seconds(H, frac=1.0):
+    """Times one step of the fp64 oracle on the host: the dense norm of W0 + sBA
+    (with g = m / max(n, eps)), then the compose forward and backward, over
+    the leading `frac` of the rows and of the tokens (the whole step when
+    frac = 1).  Returns the seconds taken."""
     import oracle
-    d_out = W0.shape[0]
-    T = T_full
-    Wr = W0[:rows].astype(np.float64)
-    Br = B[:rows].astype(np.float64)
-    Af = A.astype(np.float64)
+    d_out, T = H["W0"].shape[0], H["base"].shape[0]
+    rows = max(1, int(round(frac * d_out)))
+    toks = max(1, int(round(frac * T)))
     t0 = time.perf_counter()
-    n_rows = oracle.rows_dense_row_norm(Wr, Af, Br, s)
-    oracle.magnitude_scale(m[:rows], n_rows, eps)
-    t1 = time.perf_counter()
-    n_full = np.full(d_out, float(np.mean(n_rows)))
-    b = base[:tokens].astype(np.float64)
-    l = lora[:tokens].astype(np.float64)
-    d = dy[:tokens].astype(np.float64)
-    oracle.compose_fwd(b, l, m, n_full, s, eps)
-    oracle.compose_bwd(d, b, l, m, n_full, s, eps)
-    t2 = time.perf_counter()
-    return (t1 - t0) * d_out / rows + (t2 - t1) * T / tokens
+    n = oracle.rows_dense_row_norm(H["W0"][:rows], H["A"], H["B"][:rows], H["s"])
+    oracle.magnitude_scale(H["m"][:rows], n, H["eps"])
+    if rows < d_out:  # the compose reads a norm for every column
+        import numpy as np
+        n = np.concatenate([n, np.full(d_out - rows, float(np.mean(n)))])
+    oracle.compose_fwd(H["base"][:toks], H["lora"][:toks], H["m"], n, H["s"], H["eps"])
+    oracle.compose_bwd(H["dy"][:toks], H["base"][:toks], H["lora"][:toks], H["m"], n, H["s"],
+                       H["eps"])
+    return time.perf_counter() - t0
 
 
 def blas_threads() -> int:
@@ -199,41 +196,52 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-def host_sample_inputs(seed=7):
-    """The headline workload's inputs on the host, drawn with the same recipe
-    (bf16-rounded values) as the GPU run."""
+def host_step_inputs():
+    """The headline workload's full inputs on the host in fp64 (bf16-rounded
+    values, drawn with the same recipe as the GPU run)."""
     import numpy as np
-    import torch
     from dora_adapter_factored_b200 import synth
     w = synth.WORKLOADS[WORKLOAD]
     W0, A, B = synth.module_weights(w)
     m = synth.magnitude_from_base_rows(w, W0).double().numpy()
-    base, lora, dy = synth.activations(w, 256, W0.shape[0])
-    f = lambda t: t.float().numpy()
-    return f(W0), f(A), f(B), m, f(base), f(lora), f(dy), w.modules[0].s, synth.eps_for("bf16")
+    base, lora, dy = synth.activations(w, w.tokens, W0.shape[0])
+    f = lambda t: t.double().numpy()
+    return {"W0": f(W0), "A": f(A), "B": f(B), "m": m, "base": f(base), "lora": f(lora),
+            "dy": f(dy), "s": w.modules[0].s, "eps": synth.eps_for("bf16")}
+
+
+# Host seconds the oracle arm may spend on its timed and warm-up steps.
+ORACLE_BUDGET_S = 150.0
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    import numpy as np
     from dora_adapter_factored_b200 import synth
     w = synth.WORKLOADS[WORKLOAD]
     ms = w.modules[0]
     peaks = load_peaks()
     wm = work_model(ms.d_out, ms.d_in, ms.r, w.tokens)
     t_roof = sum(roofline_times(wm, peaks))
-    W0, A, B, m, base, lora, dy, s, eps = host_sample_inputs()
-    rows, tokens = 16, 8
-    for _ in range(args.warmup):
-        oracle_step_seconds(W0, A, B, m, base, lora, dy, s, eps, rows, tokens)
-    ts = [oracle_step_seconds(W0, A, B, m, base, lora, dy, s, eps, rows, tokens)
-          for _ in range(args.steps)]
+    H = host_step_inputs()
+    # Whole steps when the run fits the budget; otherwise every step is the
+    # same leading fraction of the rows and tokens (the value then compares
+    # that fraction of the roofline work with the time measured for it).
+    t_first = oracle_step_seconds(H)
+    frac = min(1.0, ORACLE_BUDGET_S / max(1e-9, (args.steps + args.warmup) * t_first))
+    for _ in range(max(0, args.warmup - 1)):
+        oracle_step_seconds(H, frac)
+    ts = [oracle_step_seconds(H, frac) for _ in range(args.steps)]
     t = statistics.mean(ts)
-    value = 100.0 * t_roof / t
-    sample = (f"per step: fp64 dense norm of {rows} of {ms.d_out} rows and compose fwd+bwd on "
-              f"{tokens} of {w.tokens} tokens, scaled to the full step")
+    value = 100.0 * frac * t_roof / t
+    if frac >= 1.0:
+        sample = (f"whole steps: fp64 dense norm of all {ms.d_out} rows, compose fwd+bwd on all "
+                  f"{w.tokens} tokens")
+    else:
+        sample = (f"each step the leading {frac:.4f} of the {ms.d_out} norm rows and "
+                  f"{w.tokens} tokens (a whole step takes {t_first:.2f} s); value against that "
+                  "fraction of the roofline work")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
@@ -355,10 +363,13 @@ def run_gpu(args):
     # calls (programmatic launches keep their overlap inside the graph).
     graphs = []
     cap = torch.cuda.Stream()
+    kernels_per_step = 0
     for k in range(2):
         g = torch.cuda.CUDAGraph()
+        c0 = dora.dora_launch_count()
         with torch.cuda.graph(g, stream=cap):
             step(k)
+        kernels_per_step = dora.dora_launch_count() - c0  # our kernels in one step's graph
         graphs.append(g)
     for i in range(args.warmup):
         graphs[i % 2].replay()
@@ -367,63 +378,97 @@ def run_gpu(args):
 
     clocks = ClockSampler(local)
     clocks.start()
-    launches0 = dora.dora_launch_count()
-    kernels_per_step = 6  # Gram, Gram reduce, norm GEMM (with finalize), compose fwd, compose bwd, dm finalize
     ms_step = timed(lambda i: graphs[i % 2].replay(), args.steps)
     launches = args.steps * kernels_per_step
     clk = clocks.stop()
     if dora.dora_get_device_status() != 0:
         raise RuntimeError("a kernel reported an error in the timed region")
 
-    # Per-kernel durations: CUDA events around each API call and around each
-    # call's principal kernel, captured into one graph per input set (the
-    # library records its hook events as graph nodes), so that the events see
-    # the kernels as they run inside a replayed step.  Kept out of the step
-    # time above, since event nodes between kernels stop them overlapping.
-    names = ("s0", "s1", "s2", "s3", "nk0", "nk1", "fk0", "fk1", "bk0", "bk1")
-    ev_sets = [{k: torch.cuda.Event(enable_timing=True) for k in names} for _ in range(2)]
-    for e in ev_sets:
-        for x in e.values():  # create the underlying CUDA events
-            x.record(stream)
-    torch.cuda.synchronize()
+    # Per-call durations: each API call captured K times back to back into a
+    # graph (input sets alternating, as in the step), the graph replayed R
+    # times between a pair of CUDA events on this stream: the call's time as
+    # it runs in a stream of such calls, with the same launch overlap as in
+    # the step (so the three add up to about the step time).
+    def amortized_s(call, K=10, R=None):
+        R = R if R is not None else max(3, min(args.steps, 20))
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            for i in range(K):
+                call(i)
+        for _ in range(2):
+            g.replay()
+        torch.cuda.synchronize()
+        a_ = torch.cuda.Event(enable_timing=True)
+        b_ = torch.cuda.Event(enable_timing=True)
+        st_ = torch.cuda.current_stream()
+        a_.record(st_)
+        for _ in range(R):
+            g.replay()
+        b_.record(st_)
+        torch.cuda.synchronize()
+        del g
+        return a_.elapsed_time(b_) * 1e-3 / (R * K)
+
+    def norm_call(i):
+        S_ = sets[i % 2]
+        dora.dora_factored_norm(S_["W0"], S_["A"], S_["B"], s, S_["m"], eps, n_out=outs["n"],
+                                g_out=outs["g"], ws=ws_norm)
+
+    def fwd_call(i):
+        S_ = sets[i % 2]
+        dora.dora_compose_fwd(S_["base"], S_["lora"], S_["m"], outs["n"], s, eps, y=outs["y"])
+
+    def bwd_call(i):
+        S_ = sets[i % 2]
+        dora.dora_compose_bwd(S_["dy"], S_["base"], S_["lora"], S_["m"], outs["n"], s, eps,
+                              d_base=outs["d_base"], d_lora=outs["d_lora"], dm=outs["dm"],
+                              ws=ws_bwd)
+
+    t_norm_call = amortized_s(norm_call)
+    t_fwd_call = amortized_s(fwd_call)
+    t_bwd_call = amortized_s(bwd_call)
+
+    # The fused norm GEMM alone: its CTAs stamp %globaltimer at entry and
+    # exit (the library's trace hook); the kernel's span is the last exit
+    # less the first entry, from one-call graphs replayed one at a time.
+    trace = torch.zeros(16 * 2 * 148, dtype=torch.int64, device=dev)
+    dora.dora_set_trace_buffer(trace)
     tgraphs = []
     for k in range(2):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=cap):
-            step(k, ev_sets[k], graph_events=True)
+            norm_call(k)
         tgraphs.append(g)
-    k_steps = min(args.steps, 200)
-    evs = []
-    for i in range(k_steps + 2):
+    dora.dora_set_trace_buffer(None)
+    spans = []
+    for i in range(max(6, min(args.steps, 40)) + 2):
+        trace.zero_()
         tgraphs[i % 2].replay()
         torch.cuda.synchronize()
-        if i >= 2:
-            e = ev_sets[i % 2]
-            evs.append({(a, b): e[a].elapsed_time(e[b]) for a, b in
-                        (("s0", "s1"), ("s1", "s2"), ("s2", "s3"), ("nk0", "nk1"),
-                         ("fk0", "fk1"), ("bk0", "bk1"))})
-    stream = torch.cuda.current_stream()
-
-    avg = lambda a, b: statistics.mean(e[(a, b)] for e in evs)
-    t_norm_call = avg("s0", "s1") * 1e-3
-    t_norm_k = avg("nk0", "nk1") * 1e-3
-    t_fwd_k = avg("fk0", "fk1") * 1e-3
-    t_bwd_call = avg("s2", "s3") * 1e-3
-    t_bwd_k = avg("bk0", "bk1") * 1e-3
-    t_fwd_call = avg("s1", "s2") * 1e-3
+        if i < 2:
+            continue
+        tr = trace.view(-1, 16).cpu()
+        ran = tr[:, 1] > 0
+        spans.append(float((tr[ran, 1].max() - tr[ran, 0].min()).item()) * 1e-9)
+    del tgraphs
+    t_norm_k = statistics.median(spans)
     value = world * 100.0 * t_roof / (ms_step * 1e-3)
 
     tc_peak, hbm_peak = peaks["bf16_tflops"], peaks["hbm_gbs"]
     kernels = {
         "norm_main_kernel": {"us": t_norm_k * 1e6, "bound": "tensor",
                              "achieved": wm["norm_flops"] / t_norm_k / 1e12, "peak": tc_peak,
-                             "unit": "TFLOP/s"},
-        "compose_fwd_kernel": {"us": t_fwd_k * 1e6, "bound": "hbm",
-                               "achieved": wm["fwd_bytes"] / t_fwd_k / 1e9, "peak": hbm_peak,
-                               "unit": "GB/s"},
-        "compose_bwd_kernel": {"us": t_bwd_k * 1e6, "bound": "hbm",
-                               "achieved": wm["bwd_bytes"] / t_bwd_k / 1e9, "peak": hbm_peak,
-                               "unit": "GB/s"},
+                             "unit": "TFLOP/s",
+                             "timing": "in-kernel %globaltimer span (first CTA entry to last "
+                                       "exit), median of one-call graph replays"},
+        "compose_fwd_kernel": {"us": t_fwd_call * 1e6, "bound": "hbm",
+                               "achieved": wm["fwd_bytes"] / t_fwd_call / 1e9, "peak": hbm_peak,
+                               "unit": "GB/s",
+                               "timing": "the call (this one kernel), graph of 10 calls"},
+        "compose_bwd_kernel": {"us": t_bwd_call * 1e6, "bound": "hbm",
+                               "achieved": wm["bwd_bytes"] / t_bwd_call / 1e9, "peak": hbm_peak,
+                               "unit": "GB/s",
+                               "timing": "the call (all its kernels), graph of 10 calls"},
     }
     for k in kernels.values():
         k["frac"] = k["achieved"] / k["peak"]
@@ -443,8 +488,11 @@ def run_gpu(args):
         "compose_bwd_gbs": wm["bwd_bytes"] / t_bwd_call / 1e9,
         "compose_bwd_frac_of_hbm": wm["bwd_bytes"] / t_bwd_call / 1e9 / hbm_peak,
         "compose_bwd_us": t_bwd_call * 1e6,
+        "calls_sum_us": (t_norm_call + t_fwd_call + t_bwd_call) * 1e6,
         "roofline_us": {"norm": t_roof_norm * 1e6, "compose_fwd": t_roof_fwd * 1e6,
                         "compose_bwd": t_roof_bwd * 1e6},
+        "timing": "each call captured 10 times back to back into a graph (input sets "
+                  "alternating), replayed; time per call",
         "peaks": f"{peaks['source']}: HBM {hbm_peak} GB/s, bf16 {tc_peak} TFLOP/s (burst)",
     }
 
@@ -468,8 +516,8 @@ def run_gpu(args):
             "components": components,
             "clocks": clk,
             "gpu_launches": int(launches),
-            "launch": "CUDA graph replay of the step's API calls (6 kernels, programmatic "
-                      "dependent launches)",
+            "launch": f"CUDA graph replay of the step's API calls ({kernels_per_step} kernels, "
+                      "programmatic dependent launches)",
             "eager_ms_per_step": eager_ms,
             "e2e": e2e,
             "cpu_baseline": cpu,
@@ -510,67 +558,111 @@ def load_traffic(kernel: str):
 
 def measure_e2e(args, dora, w, S_, s, eps, t_roof, dev, stream, pg, local, world):
     """The same step through the public API with host (pinned) buffers: every
-    step copies its inputs host->device and reads its results back."""
+    step copies its inputs host->device and reads its results back.  Copies
+    and kernels are pipelined on three streams (PCIe is full duplex): the
+    norm starts once W0, A and B have landed while the activations are still
+    crossing, y goes back while the backward runs, and the next step's inputs
+    cross while this step computes and returns (device buffers alternate
+    between two sets)."""
     import torch
-    host = {k: S_[k].cpu().pin_memory() for k in ("W0", "A", "B", "m", "base", "lora", "dy")}
-    dev_in = {k: torch.empty_like(S_[k]) for k in host}
+    keys_w = ("W0", "A", "B", "m")
+    keys_a = ("base", "lora", "dy")
+    host = {k: S_[k].cpu().pin_memory() for k in keys_w + keys_a}
     T, d_out = S_["base"].shape
-    outs_dev = dict(n=torch.empty(d_out, device=dev), g=torch.empty(d_out, device=dev),
+    dev_in = [{k: torch.empty_like(S_[k]) for k in host} for _ in range(2)]
+
+    def outs():
+        return dict(n=torch.empty(d_out, device=dev), g=torch.empty(d_out, device=dev),
                     y=torch.empty(T, d_out, dtype=torch.bfloat16, device=dev),
                     d_base=torch.empty(T, d_out, dtype=torch.bfloat16, device=dev),
                     d_lora=torch.empty(T, d_out, dtype=torch.bfloat16, device=dev),
                     dm=torch.empty(d_out, device=dev))
-    outs_host = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in outs_dev.items()}
+    dev_out = [outs() for _ in range(2)]
+    host_out = [{k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in o.items()}
+                for o in dev_out]
+    ws_norm = [torch.empty(dora.dora_factored_norm_workspace_size(
+        S_["W0"].shape[0], S_["W0"].shape[1], S_["A"].shape[0], torch.bfloat16),
+        dtype=torch.uint8, device=dev) for _ in range(2)]
+    ws_bwd = [torch.empty(max(256, dora.dora_compose_bwd_workspace_size(T, d_out, torch.bfloat16)),
+                          dtype=torch.uint8, device=dev) for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = sum(t.numel() * t.element_size() for t in outs_host.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out[0].values())
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    done_cmp = [ev(), ev()]   # set k's inputs are free again
+    done_out = [ev(), ev()]   # set k's outputs have been read back
+    for k in range(2):
+        done_cmp[k].record(s_cmp)
+        done_out[k].record(s_out)
 
-    def e2e_step():
-        for k in host:
-            dev_in[k].copy_(host[k], non_blocking=True)
-        dora.dora_factored_norm(dev_in["W0"], dev_in["A"], dev_in["B"], s, dev_in["m"], eps,
-                                n_out=outs_dev["n"], g_out=outs_dev["g"])
-        dora.dora_compose_fwd(dev_in["base"], dev_in["lora"], dev_in["m"], outs_dev["n"], s, eps,
-                              y=outs_dev["y"])
-        dora.dora_compose_bwd(dev_in["dy"], dev_in["base"], dev_in["lora"], dev_in["m"],
-                              outs_dev["n"], s, eps, d_base=outs_dev["d_base"],
-                              d_lora=outs_dev["d_lora"], dm=outs_dev["dm"])
-        for k in outs_dev:
-            outs_host[k].copy_(outs_dev[k], non_blocking=True)
+    def e2e_step(i):
+        k = i % 2
+        D, O, HO = dev_in[k], dev_out[k], host_out[k]
+        ev_w, ev_a, ev_y, ev_b = ev(), ev(), ev(), ev()
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(done_cmp[k])
+            for x in keys_w:
+                D[x].copy_(host[x], non_blocking=True)
+            ev_w.record(s_in)
+            for x in keys_a:
+                D[x].copy_(host[x], non_blocking=True)
+            ev_a.record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(done_out[k])
+            s_cmp.wait_event(ev_w)
+            dora.dora_factored_norm(D["W0"], D["A"], D["B"], s, D["m"], eps, n_out=O["n"],
+                                    g_out=O["g"], ws=ws_norm[k])
+            s_cmp.wait_event(ev_a)
+            dora.dora_compose_fwd(D["base"], D["lora"], D["m"], O["n"], s, eps, y=O["y"])
+            ev_y.record(s_cmp)
+            dora.dora_compose_bwd(D["dy"], D["base"], D["lora"], D["m"], O["n"], s, eps,
+                                  d_base=O["d_base"], d_lora=O["d_lora"], dm=O["dm"],
+                                  ws=ws_bwd[k])
+            ev_b.record(s_cmp)
+            done_cmp[k].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_y)
+            for x in ("n", "g", "y"):
+                HO[x].copy_(O[x], non_blocking=True)
+            s_out.wait_event(ev_b)
+            for x in ("d_base", "d_lora", "dm"):
+                HO[x].copy_(O[x], non_blocking=True)
+            done_out[k].record(s_out)
 
     steps = max(3, min(20, args.steps))
-    for _ in range(3):
-        e2e_step()
+    for i in range(3):
+        e2e_step(i)
     torch.cuda.synchronize()
     barrier(pg, local)
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        e2e_step()
-    b.record(stream)
+    a.record(s_in)
+    for i in range(steps):
+        e2e_step(i)
+    s_in.wait_stream(s_out)
+    b.record(s_in)
     torch.cuda.synchronize()
     barrier(pg, local)
     ms = max_over_ranks(pg, a.elapsed_time(b)) / steps
     return {"value": world * 100.0 * t_roof / (ms * 1e-3), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "ms_per_step": ms, "steps": steps}
+            "ms_per_step": ms, "steps": steps,
+            "pipeline": "H2D / kernels / D2H on three streams, two device buffer sets"}
 
 
 def measure_cpu_baseline(t_roof):
-    """The oracle as it stands on the host cores, on a bounded sample of the
-    same workload (about 10 s of CPU work), scaled to one full step."""
-    W0, A, B, m, base, lora, dy, s, eps = host_sample_inputs()
-    rows, tokens = 512, 64
-    oracle_step_seconds(W0, A, B, m, base, lora, dy, s, eps, 16, 4)  # warm
-    ts = []
+    """The oracle as it stands on the host cores: whole steps of the same
+    workload (the function the reference arm times), about 10-20 s of them."""
+    H = host_step_inputs()
+    ts = [oracle_step_seconds(H)]
     t0 = time.perf_counter()
-    while time.perf_counter() - t0 < 10.0 and len(ts) < 200:
-        ts.append(oracle_step_seconds(W0, A, B, m, base, lora, dy, s, eps, rows, tokens))
+    while time.perf_counter() - t0 < 10.0 and len(ts) < 50:
+        ts.append(oracle_step_seconds(H))
+    ts = ts[1:] if len(ts) > 1 else ts
     t = statistics.mean(ts)
     return {"value": 100.0 * t_roof / t, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": (f"{len(ts)} repeats of: fp64 dense norm of {rows} of 8192 rows and "
-                       f"compose fwd+bwd on {tokens} of 4096 tokens, scaled to one full step "
-                       f"({t:.2f} s per full step)")}
+            "sample": (f"{len(ts)} whole steps (fp64 dense norm of all 8192 rows, compose "
+                       f"fwd+bwd on all 4096 tokens), {t:.2f} s per step")}
 
 
 # --------------------------------------------------------------------------- suite
@@ -897,6 +989,30 @@ def run_suite(args):
     wd = b0 - a0
     emit("factored_norm_sq_shard", f"headline module, columns [{a0}, {b0}) of 2 shards", t,
          2.0 * ms.d_out * wd * ms.r, 2.0 * (ms.d_out * wd + ms.r * wd + ms.d_out * ms.r))
+    # ---- stable compose against a naive bf16 evaluation near g = 1 ("Scaling
+    # DoRA", section 3: about 3.0x lower peak error at d_out = 8192, d_in =
+    # 2048, against fp64); read as [2048, 8192] activations, g = 1 + N(0, 0.0015)
+    T, d_out, s = 2048, 8192, 2.0
+    g_ = torch.Generator().manual_seed(2048)
+    base = torch.randn(T, d_out, generator=g_).bfloat16()
+    lora = torch.randn(T, d_out, generator=g_).bfloat16()
+    n = torch.empty(d_out).uniform_(0.5, 2.0, generator=g_)
+    m = (n.double() * (1.0 + 0.0015 * torch.randn(d_out, generator=g_).double())).float()
+    y = dora.dora_compose_fwd(base.to(dev), lora.to(dev), m.to(dev), n.to(dev), s, eps)
+    gb = (m.to(dev) / n.to(dev).clamp_min(eps)).bfloat16()
+    bd, ld = base.to(dev), lora.to(dev)
+    y_naive = bd + ((gb - 1) * bd + (gb * s) * ld)
+    torch.cuda.synchronize()
+    ref = oracle.compose_fwd(base.double().numpy(), lora.double().numpy(), m.double().numpy(),
+                             n.double().numpy(), s, eps)
+    e_st = float(np.max(np.abs(y.double().cpu().numpy() - ref)))
+    e_nv = float(np.max(np.abs(y_naive.double().cpu().numpy() - ref)))
+    print(json.dumps({"suite": "compose_stability", "workload": "[2048, 8192] bf16, g = 1 + N(0, 0.0015)",
+                      "peak_abs_err_stable": e_st, "peak_abs_err_naive_bf16": e_nv,
+                      "ratio": e_nv / e_st, "pages_ratio": 3.0,
+                      "naive": "g rounded to bf16, base + ((g - 1) base + g s lora) in bf16 ops"}),
+          flush=True)
+
     if dora.dora_get_device_status() != 0:
         raise RuntimeError("a kernel reported an error during the suite")
     return 0

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <cstdio>
 #include <cstring>
@@ -60,6 +61,7 @@ struct DeviceInfo {
   bool supported = false;
   int sms = 0;
   bool attrs_set = false;
+  int norm_pairs = 0;  // CTA pairs of the norm GEMM resident at once
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -176,18 +178,19 @@ PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
   return fn;
 }
 
-// Row-major bf16 matrix [nblk * blk_rows, cols] viewed as 3-D {cols, blk_rows,
-// nblk}, loaded as one box {box_cols, blk_rows, nblk} (128-byte swizzle).  The
-// caller guarantees nblk * blk_rows equals the matrix's row count.
-bool make_tmap_bf16_3d(CUtensorMap* map, const void* ptr, uint64_t blk_rows, uint64_t nblk,
-                       uint64_t cols, uint64_t ld, uint32_t box_cols) {
+// The N-side slab of a CTA pair: a row-major bf16 matrix of exactly 4 h rows
+// (two accumulator chunks of 2 h rows, each split between the two CTAs)
+// viewed as 4-D {cols, h, rank, chunk}; one box {box_cols, h, 1, 2} at
+// (x, 0, rank, 0) brings a CTA its h rows of both chunks (128-byte swizzle).
+bool make_tmap_bf16_pairslab(CUtensorMap* map, const void* ptr, uint64_t h, uint64_t cols,
+                             uint64_t ld, uint32_t box_cols) {
   auto enc = tmap_encoder();
   if (enc == nullptr) return false;
-  cuuint64_t dims[3] = {cols, blk_rows, nblk};
-  cuuint64_t strides[2] = {ld * 2, blk_rows * ld * 2};
-  cuuint32_t box[3] = {box_cols, static_cast<cuuint32_t>(blk_rows), static_cast<cuuint32_t>(nblk)};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+  cuuint64_t dims[4] = {cols, h, 2, 2};
+  cuuint64_t strides[3] = {ld * 2, h * ld * 2, 2 * h * ld * 2};
+  cuuint32_t box[4] = {box_cols, static_cast<cuuint32_t>(h), 1, 2};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -211,32 +214,30 @@ bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t c
 // ------------------------------------------------------------ norm planning
 
 struct ModulePlan {
-  // N side
-  int n_pad, n0, n1, box_rows, nbox, tmem_cols;
+  // N side (pair MMA chunks; each CTA stages h0 rows of each)
+  int n_pad, n0, n1, h0, tmem_cols;
   uint32_t b_region;
-  // K / tiles
-  int kb_w, kb_r, kb_tile, tiles;
-  long long units;
-  // Gram
-  int r8, tiles_r, pairs, kb_gram, S;
-  // workspace (relative offsets inside the module's region)
-  size_t off_g, off_gp, off_np, off_cnt, bytes;
-  int seg_slots;
+  // K and tiles (tiles of 256 rows; Gram pseudo-tiles of 256 rows of A)
+  int kb_w, kb_r, tiles, pg_tiles, r8;
+  long long units[3];  // Gram, W0 and G units
+  // workspace (byte offsets from the workspace base) and counters (ints
+  // from the start of the counter block)
+  size_t off_g, off_gp, off_np, off_tw, cnt_off;
 };
 
+// One accumulator chunk up to N = 256, else two equal chunks; each chunk's
+// slab rows are split evenly between the two CTAs in 8-row swizzle groups.
 void plan_n_side(int r, ModulePlan& p) {
-  p.n_pad = round_up_int(r, 16);
-  if (p.n_pad <= 256) {
+  if (r <= 256) {
+    p.n_pad = round_up_int(r, 16);
     p.n0 = p.n_pad;
     p.n1 = 0;
-    p.nbox = 1;
   } else {
-    p.n0 = round_up_int((p.n_pad + 1) / 2, 16);
-    p.n1 = p.n_pad - p.n0;
-    p.nbox = 2;
+    p.n_pad = round_up_int(r, 32);
+    p.n0 = p.n1 = p.n_pad / 2;
   }
-  p.box_rows = p.n0;
-  p.b_region = static_cast<uint32_t>(p.nbox * p.box_rows * 128);
+  p.h0 = p.n0 / 2;
+  p.b_region = static_cast<uint32_t>(p.n_pad / 2 * 128);
   int tc = 32;
   while (tc < p.n_pad) tc <<= 1;
   p.tmem_cols = tc;
@@ -246,163 +247,199 @@ void plan_module(int64_t d_out, int64_t d_in, int64_t r, ModulePlan& p) {
   plan_n_side(static_cast<int>(r), p);
   p.kb_w = static_cast<int>(ceil_div_ll(d_in, kBlockK));
   p.kb_r = static_cast<int>(ceil_div_ll(r, kBlockK));
-  p.kb_tile = p.kb_w + 2 * p.kb_r;  // W0 blocks, then B.G'_hi, then B.G'_lo
-  p.tiles = static_cast<int>(ceil_div_ll(d_out, kTileM));
-  p.units = static_cast<long long>(p.tiles) * p.kb_tile;
+  p.tiles = static_cast<int>(ceil_div_ll(d_out, kPairM));
+  p.pg_tiles = static_cast<int>(ceil_div_ll(r, kPairM));
   p.r8 = round_up_int(static_cast<int>(r), 8);
-  p.tiles_r = static_cast<int>(ceil_div_ll(r, kTileM));
-  p.pairs = p.tiles_r * (p.tiles_r + 1) / 2;
-  p.kb_gram = p.kb_w;
-  const int by_k = std::max(1, p.kb_gram / 8);
-  const int by_sm = std::max(1, 148 / p.pairs);
-  p.S = std::max(1, std::min(by_k, by_sm));
+  p.units[kPhaseGram] = static_cast<long long>(p.pg_tiles) * p.kb_w;
+  p.units[kPhaseW0] = static_cast<long long>(p.tiles) * p.kb_w;
+  p.units[kPhaseG] = static_cast<long long>(p.tiles) * 2 * p.kb_r;
 }
 
-// Re-read operands (A and G') of one stream-K wave of the grouped norm: well
-// inside the 126 MB L2, which also carries the W0 stream.
+int module_counters(const ModulePlan& p) { return p.tiles * 8 + p.pg_tiles * 2 + 1; }
+
+// Re-read operands (A and G') of one wave of the grouped norm: well inside
+// the 126 MB L2, which also carries the W0 stream.
 constexpr size_t kWaveBudgetBytes = size_t(40) << 20;
 
-// Largest number of stream-K segments on any tile of any module; module i
-// lies in the wave starting at unit wave_of[i] with wave_units[i] units.
-int max_seg_slots(const std::vector<ModulePlan>& plans, const std::vector<long long>& wave_of,
-                  const std::vector<long long>& wave_units, int C) {
-  int best = 1;
-  long long begin = 0;
-  for (size_t i = 0; i < plans.size(); ++i) {
-    const auto& p = plans[i];
-    for (int t = 0; t < p.tiles; ++t) {
-      const long long x0 = begin - wave_of[i] + static_cast<long long>(t) * p.kb_tile;
-      const int c0 = first_cta_of_unit(x0, wave_units[i], C);
-      const int c1 = first_cta_of_unit(x0 + p.kb_tile - 1, wave_units[i], C);
-      best = std::max(best, c1 - c0 + 1);
-    }
-    begin += p.units;
-  }
-  return best;
-}
-
-// Splits the modules, in order, into stream-K waves: a wave closes before a
-// module that would take its re-read operands (A, G'_hi, G'_lo) past
-// `budget` bytes, provided it already holds at least `ctas` units; a last
-// wave smaller than that joins the one before.  Returns the waves' first
-// units (and the total at the end).
-std::vector<long long> plan_waves(const std::vector<ModulePlan>& plans, const int64_t* d_in,
-                                  const int64_t* r, long long total, int ctas, size_t budget) {
-  std::vector<long long> begin{0};
-  long long units = 0, at = 0;
+// Splits the modules, in order, into waves: a wave closes before a module
+// that would take its re-read operands (A, G'_hi, G'_lo) past `budget`
+// bytes, provided it already holds at least `min_w` W0 units; a last wave
+// with fewer joins the one before.  Returns the waves' first modules (and
+// the module count at the end).
+std::vector<int> plan_waves(const std::vector<ModulePlan>& plans, const int64_t* d_in,
+                            const int64_t* r, long long min_w, size_t budget) {
+  std::vector<int> begin{0};
+  long long wunits = 0;
   size_t bytes = 0;
-  for (size_t i = 0; i < plans.size(); ++i) {
+  const int count = static_cast<int>(plans.size());
+  for (int i = 0; i < count; ++i) {
     const size_t mb = static_cast<size_t>(r[i]) * d_in[i] * 2 +
                       2 * static_cast<size_t>(r[i]) * plans[i].r8 * 2;
-    if (units > 0 && bytes + mb > budget && units >= ctas) {
-      begin.push_back(at);
-      units = 0;
+    if (wunits > 0 && bytes + mb > budget && wunits >= min_w) {
+      begin.push_back(i);
+      wunits = 0;
       bytes = 0;
     }
-    units += plans[i].units;
-    at += plans[i].units;
+    wunits += plans[i].units[kPhaseW0];
     bytes += mb;
   }
-  if (begin.size() > 1 && total - begin.back() < ctas) begin.pop_back();
-  begin.push_back(total);
+  if (begin.size() > 1 && wunits < min_w) begin.pop_back();
+  begin.push_back(count);
   return begin;
+}
+
+// Every pair's W0 range non-empty and every phase's ranges in order.
+bool sched_valid(const WaveInfo& w, int pairs) {
+  for (int j = 0; j < pairs; ++j)
+    for (int ph = kPhaseGram; ph <= kPhaseG; ++ph) {
+      const long long a = sched_begin(w, pairs, ph, j), b = sched_begin(w, pairs, ph, j + 1);
+      if (b < a || (ph == kPhaseW0 && b == a)) return false;
+    }
+  return true;
+}
+
+// Units a Gram pair's W0 share is cut by for each Gram segment it ends
+// (posting the partial and reducing its rows of G' take about that long).
+constexpr int kGramEpilogueUnits = 10;
+
+// The Gram pairs of a wave: about half a pair's share of work each (so the
+// Gram is done early), more when the schedule needs them.
+bool choose_gram_pairs(WaveInfo& w, int pairs) {
+  const double share = static_cast<double>(w.n[0] + w.n[1] + w.n[2]) / pairs;
+  int J = static_cast<int>(std::ceil(2.0 * w.n[0] / std::max(1.0, share)));
+  J = std::min(std::max(J, 1), pairs);
+  for (; J <= pairs; ++J) {
+    w.J = J;
+    w.gw = w.n[0] + static_cast<long long>(J) * kGramEpilogueUnits;
+    if (sched_valid(w, pairs)) return true;
+    w.gw = w.n[0];
+    if (sched_valid(w, pairs)) return true;
+  }
+  return false;
 }
 
 struct GroupLayout {
   std::vector<ModulePlan> plans;
-  long long total_units = 0;
-  int ctas = 0;
-  int seg_slots = 1;
+  NormSched sched;
+  int seg_slots = 1, gram_slots = 1;
   uint32_t b_region = 0;
   int tmem_cols = 32;
-  std::vector<long long> waves;                 // first unit of each wave, then the total
-  std::vector<long long> wave_of, wave_units;   // per module: its wave's first unit, units
   int stages = 0;
   size_t smem_bytes = 0;
-  int gram_jobs = 0;
-  int max_pairs = 0;
-  size_t table_bytes = 0;  // descriptor tables at the start of the workspace (grouped)
+  size_t table_bytes = 0;  // descriptor table at the start of the workspace (grouped)
+  size_t cnt_bytes = 0;    // the counter block, right after it
+  int cnt_ints = 0;
   size_t total_bytes = 0;
 };
 
+// `workers`: the CTA pairs the norm kernel may run (one per two SMs that
+// can hold a cluster).
 bool layout_group(const int64_t* d_out, const int64_t* d_in, const int64_t* r, int count,
-                  bool grouped, int sms, GroupLayout& L) {
+                  bool grouped, int workers, GroupLayout& L) {
   L.plans.resize(count);
-  L.total_units = 0;
   for (int i = 0; i < count; ++i) plan_module(d_out[i], d_in[i], r[i], L.plans[i]);
-  if (grouped && count > 1) {
-    // K splits of the Gram for a group: the modules themselves give
-    // parallelism, so aim at about two waves of jobs of equal length over the
-    // whole group instead of filling the GPU with each module's splits.
-    long long work = 0;  // k-blocks over all (pair, k-block) of the group
-    for (const auto& p : L.plans) work += static_cast<long long>(p.pairs) * p.kb_gram;
-    const long long per_job = std::max(1ll, ceil_div_ll(work, 2ll * sms));
-    for (auto& p : L.plans) {
-      const long long by_len = std::max(1ll, (p.kb_gram + per_job / 2) / per_job);
-      p.S = static_cast<int>(std::min<long long>(by_len, std::max(1, p.kb_gram / 8)));
-    }
+  long long total_w = 0;
+  for (const auto& p : L.plans) {
+    L.b_region = std::max(L.b_region, p.b_region);
+    L.tmem_cols = std::max(L.tmem_cols, p.tmem_cols);
+    total_w += p.units[kPhaseW0];
   }
-  for (int i = 0; i < count; ++i) {
-    L.total_units += L.plans[i].units;
-    L.b_region = std::max(L.b_region, L.plans[i].b_region);
-    L.tmem_cols = std::max(L.tmem_cols, L.plans[i].tmem_cols);
-    L.gram_jobs += L.plans[i].pairs * L.plans[i].S;
-    L.max_pairs = std::max(L.max_pairs, L.plans[i].pairs);
-  }
-  L.ctas = static_cast<int>(std::min<long long>(sms, L.total_units));
-  if (L.ctas < 1) return false;
-  {
+  // Pairs: about a dozen units each at least (every segment ends in an
+  // epilogue), at most one per W0 unit; fewer if some wave cannot give every
+  // pair a W0 range.
+  long long total = 0;
+  for (const auto& p : L.plans) total += p.units[0] + p.units[1] + p.units[2];
+  int pairs = static_cast<int>(std::min<long long>(
+      std::max(1, workers), std::min<long long>(total_w, std::max(1ll, total / 12))));
+  std::vector<int> wb;
+  while (true) {
     size_t budget = grouped ? kWaveBudgetBytes : SIZE_MAX;
-    L.waves = plan_waves(L.plans, d_in, r, L.total_units, L.ctas, budget);
-    while (static_cast<int>(L.waves.size()) - 1 > kMaxWaves) {
+    const long long min_w = 3ll * pairs;
+    wb = plan_waves(L.plans, d_in, r, min_w, budget);
+    while (static_cast<int>(wb.size()) - 1 > kMaxWaves) {
       budget *= 2;
-      L.waves = plan_waves(L.plans, d_in, r, L.total_units, L.ctas, budget);
+      wb = plan_waves(L.plans, d_in, r, min_w, budget);
     }
-    L.wave_of.resize(count);
-    L.wave_units.resize(count);
-    long long at = 0;
-    size_t w = 0;
-    for (int i = 0; i < count; ++i) {
-      while (at >= L.waves[w + 1]) ++w;
-      L.wave_of[i] = L.waves[w];
-      L.wave_units[i] = L.waves[w + 1] - L.waves[w];
-      at += L.plans[i].units;
+    bool ok = true;
+    NormSched& S = L.sched;
+    S.waves = static_cast<int>(wb.size()) - 1;
+    S.pairs = pairs;
+    for (int w = 0; w < S.waves && ok; ++w) {
+      WaveInfo& wi = S.w[w];
+      wi.m0 = wb[w];
+      wi.m1 = wb[w + 1];
+      wi.n[0] = wi.n[1] = wi.n[2] = 0;
+      for (int i = wi.m0; i < wi.m1; ++i)
+        for (int ph = 0; ph < 3; ++ph) wi.n[ph] += L.plans[i].units[ph];
+      if (wi.n[kPhaseW0] < pairs || !choose_gram_pairs(wi, pairs)) ok = false;
+    }
+    if (ok) break;
+    if (pairs == 1) return false;
+    pairs = std::max(1, pairs * 3 / 4);
+  }
+  // Segment slots: the most segments any tile (W0 + G) or pseudo-tile has.
+  const NormSched& S = L.sched;
+  L.seg_slots = 1;
+  L.gram_slots = 1;
+  std::vector<long long> mb(3 * count);
+  for (int w = 0; w < S.waves; ++w) {
+    long long at[3] = {0, 0, 0};
+    for (int i = S.w[w].m0; i < S.w[w].m1; ++i) {
+      const ModulePlan& p = L.plans[i];
+      for (int ph = 0; ph < 3; ++ph) {
+        mb[3 * i + ph] = at[ph];
+        at[ph] += p.units[ph];
+      }
+      for (int t = 0; t < p.pg_tiles; ++t) {
+        const long long x0 = mb[3 * i] + static_cast<long long>(t) * p.kb_w;
+        L.gram_slots = std::max(L.gram_slots, sched_segments(S.w[w], S.pairs, kPhaseGram, x0,
+                                                             x0 + p.kb_w, -1, nullptr));
+      }
+      for (int t = 0; t < p.tiles; ++t) {
+        const long long xw = mb[3 * i + 1] + static_cast<long long>(t) * p.kb_w;
+        const long long xg = mb[3 * i + 2] + static_cast<long long>(t) * 2 * p.kb_r;
+        L.seg_slots = std::max(
+            L.seg_slots,
+            sched_segments(S.w[w], S.pairs, kPhaseW0, xw, xw + p.kb_w, -1, nullptr) +
+                sched_segments(S.w[w], S.pairs, kPhaseG, xg, xg + 2 * p.kb_r, -1, nullptr));
+      }
     }
   }
-  L.seg_slots = max_seg_slots(L.plans, L.wave_of, L.wave_units, L.ctas);
   const uint32_t stage_bytes = kTileABytes + L.b_region;
   const int tail_bytes = static_cast<int>(align_up(sizeof(NormSmemTail), 128));
   L.stages = std::min<int>(kMaxStages, (kMaxDynSmem - 1024 - tail_bytes) / stage_bytes);
   if (L.stages < 2) return false;
   L.smem_bytes = 1024 + static_cast<size_t>(L.stages) * stage_bytes + tail_bytes;
-  size_t off = 0;
-  if (grouped) {
-    off = align_up(sizeof(NormProblemDev) * count, 256) + align_up(sizeof(GramProblemDev) * count, 256);
-  }
+  size_t off = grouped ? align_up(sizeof(NormProblemDev) * count, 256) : 0;
   L.table_bytes = off;
+  int cnt = 0;
   for (auto& p : L.plans) {
-    p.seg_slots = L.seg_slots;
+    p.cnt_off = static_cast<size_t>(cnt);
+    cnt += module_counters(p);
+  }
+  L.cnt_ints = cnt;
+  L.cnt_bytes = align_up(static_cast<size_t>(cnt) * sizeof(int), 256);
+  off += L.cnt_bytes;
+  for (auto& p : L.plans) {
     p.off_g = off;
-    off += align_up(static_cast<size_t>(2) * p.n_pad * p.r8 * 2, 256);  // G'_hi, G'_lo
+    off += align_up(static_cast<size_t>(2) * p.n_pad * p.r8 * 2, 256);  // G'_hi^T, G'_lo^T
     p.off_gp = off;
-    off += align_up(static_cast<size_t>(p.pairs) * p.S * kTileM * kTileM * 4, 256);
+    off += align_up(static_cast<size_t>(p.pg_tiles) * L.gram_slots * p.n_pad * kPairM * 4, 256);
     p.off_np = off;
-    off += align_up(static_cast<size_t>(p.tiles) * L.seg_slots * kTileM * 4, 256);
-    p.off_cnt = off;
-    off += align_up(static_cast<size_t>(p.tiles) * 4 * sizeof(int), 256);
+    off += align_up(static_cast<size_t>(p.tiles) * L.seg_slots * kPairM * 4, 256);
+    p.off_tw = off;
+    off += align_up(static_cast<size_t>(p.tiles) * sizeof(int), 256);
   }
   L.total_bytes = off;
   return true;
 }
 
-bool ensure_tc_attrs(int smem_norm) {
+bool ensure_tc_attrs() {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   std::lock_guard<std::mutex> lk(g_dev_mu);
   DeviceInfo& d = g_dev[dev];
   if (d.attrs_set) return true;
-  (void)smem_norm;
-  const int gram_smem = 1024 + kGramStages * kGramStageBytes + 256;
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(norm_main_kernel<false>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem)) !=
@@ -410,80 +447,99 @@ bool ensure_tc_attrs(int smem_norm) {
       (e = cudaFuncSetAttribute(norm_main_kernel<true>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem)) !=
           cudaSuccess ||
-      (e = cudaFuncSetAttribute(gram_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                gram_smem)) != cudaSuccess ||
-      (e = cudaFuncSetAttribute(gram_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                gram_smem)) != cudaSuccess ||
       (e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 kMaxDynSmem)) != cudaSuccess) {
     note_error("cudaFuncSetAttribute", e);
     return false;
   }
+  // How many CTA pairs of the norm kernel (one CTA per SM) can be resident at
+  // once: all of them must be, since the pairs that take the G units wait for
+  // the pairs that reduce the Gram.
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * std::max(1, sms / 2));
+  cfg.blockDim = dim3(kNormThreads);
+  cfg.dynamicSmemBytes = kMaxDynSmem;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, norm_main_kernel<false>, &cfg) != cudaSuccess ||
+      clusters < 1) {
+    (void)cudaGetLastError();
+    clusters = std::max(1, sms / 2);
+  }
+  d.norm_pairs = std::min(clusters, std::max(1, sms / 2));
   d.attrs_set = true;
   return true;
 }
 
-// Fills the device descriptors of one module.
-bool fill_descriptors(const dora_norm_problem_t& pr, const ModulePlan& p, uint8_t* ws_base,
-                      long long unit_begin, int gram_job_begin, NormProblemDev& nd,
-                      GramProblemDev& gd) {
+// Stream-K workers (CTA pairs) of the norm kernel on the current device; half
+// the SMs of a B200 when the device cannot be asked (workspace sizing on a
+// host without one).
+int norm_workers() {
+  int dev = 0;
+  if (ensure_tc_attrs() && cudaGetDevice(&dev) == cudaSuccess) return g_dev[dev].norm_pairs;
+  (void)cudaGetLastError();
+  return 74;
+}
+
+// Fills the device descriptor of module `i`; `phase_begin` are its first
+// units in its wave's Gram, W0 and G sequences.
+bool fill_descriptor(const dora_norm_problem_t& pr, const GroupLayout& L, int i,
+                     const long long* phase_begin, uint8_t* ws_base, NormProblemDev& nd) {
+  const ModulePlan& p = L.plans[i];
   std::memset(&nd, 0, sizeof(nd));
-  std::memset(&gd, 0, sizeof(gd));
-  uint16_t* gprime = reinterpret_cast<uint16_t*>(ws_base + p.off_g);
-  uint16_t* gprime_lo = gprime + static_cast<size_t>(p.n_pad) * p.r8;
+  uint16_t* g_hi = reinterpret_cast<uint16_t*>(ws_base + p.off_g);
+  uint16_t* g_lo = g_hi + static_cast<size_t>(p.n_pad) * p.r8;
   bool ok = true;
   ok &= make_tmap_bf16(&nd.tm_w0, pr.W0, pr.d_out, pr.d_in, pr.d_in, kBlockK, kTileM);
-  // The N-side slab in one 3-D box when its chunks are equal and cover r
-  // exactly (no dimension of the view can then reach past the matrix).
-  const bool slab3d = p.nbox == 2 && p.n0 == p.n1 && 2 * p.n0 == pr.r;
-  nd.slab3d = slab3d ? 1 : 0;
-  if (slab3d) {
-    ok &= make_tmap_bf16_3d(&nd.tm_a, pr.A, p.n0, 2, pr.d_in, pr.d_in, kBlockK);
-    ok &= make_tmap_bf16_3d(&nd.tm_g, gprime, p.n0, 2, pr.r, p.r8, kBlockK);
-    ok &= make_tmap_bf16_3d(&nd.tm_glo, gprime_lo, p.n0, 2, pr.r, p.r8, kBlockK);
+  ok &= make_tmap_bf16(&nd.tm_arow, pr.A, pr.r, pr.d_in, pr.d_in, kBlockK, kTileM);
+  // The N-side slab half of a CTA in one 4-D box when the two chunks are
+  // equal and cover r exactly (no dimension of the view then reaches past the
+  // matrix); otherwise one 2-D box of h0 rows per chunk (rows past r read 0).
+  const bool slab4d = p.n1 > 0 && 2 * p.n0 == pr.r;
+  nd.slab4d = slab4d ? 1 : 0;
+  if (slab4d) {
+    ok &= make_tmap_bf16_pairslab(&nd.tm_a, pr.A, p.h0, pr.d_in, pr.d_in, kBlockK);
+    ok &= make_tmap_bf16_pairslab(&nd.tm_g, g_hi, p.h0, pr.r, p.r8, kBlockK);
+    ok &= make_tmap_bf16_pairslab(&nd.tm_glo, g_lo, p.h0, pr.r, p.r8, kBlockK);
   } else {
-    ok &= make_tmap_bf16(&nd.tm_a, pr.A, pr.r, pr.d_in, pr.d_in, kBlockK, p.box_rows);
-    ok &= make_tmap_bf16(&nd.tm_g, gprime, pr.r, pr.r, p.r8, kBlockK, p.box_rows);
-    ok &= make_tmap_bf16(&nd.tm_glo, gprime_lo, pr.r, pr.r, p.r8, kBlockK, p.box_rows);
+    ok &= make_tmap_bf16(&nd.tm_a, pr.A, pr.r, pr.d_in, pr.d_in, kBlockK, p.h0);
+    ok &= make_tmap_bf16(&nd.tm_g, g_hi, pr.r, pr.r, p.r8, kBlockK, p.h0);
+    ok &= make_tmap_bf16(&nd.tm_glo, g_lo, pr.r, pr.r, p.r8, kBlockK, p.h0);
   }
   ok &= make_tmap_bf16(&nd.tm_b, pr.B, pr.d_out, pr.r, pr.r, kBlockK, kTileM);
-  ok &= make_tmap_bf16(&gd.tm_a, pr.A, pr.r, pr.d_in, pr.d_in, kBlockK, kTileM);
+  int* cnt = reinterpret_cast<int*>(ws_base + L.table_bytes) + p.cnt_off;
   nd.B = static_cast<const uint16_t*>(pr.B);
+  nd.g_hi = g_hi;
+  nd.g_lo = g_lo;
   nd.partial = reinterpret_cast<float*>(ws_base + p.off_np);
-  nd.tile_cnt = reinterpret_cast<int*>(ws_base + p.off_cnt);
+  nd.gram_part = reinterpret_cast<float*>(ws_base + p.off_gp);
+  nd.tile_cnt = cnt;
+  nd.gram_cnt = cnt + p.tiles * 8;
+  nd.g_ready = cnt + p.tiles * 8 + p.pg_tiles * 2;
+  nd.tile_w = reinterpret_cast<int*>(ws_base + p.off_tw);
   nd.m = pr.m;
   nd.n_out = pr.n_out;
   nd.g_out = pr.g_out;
-  nd.unit_begin = unit_begin;
+  for (int ph = 0; ph < 3; ++ph) nd.begin[ph] = phase_begin[ph];
   nd.d_out = static_cast<int>(pr.d_out);
   nd.r = static_cast<int>(pr.r);
+  nd.r8 = p.r8;
+  nd.n_pad = p.n_pad;
   nd.n0 = p.n0;
   nd.n1 = p.n1;
-  nd.box_rows = p.box_rows;
-  nd.nbox = p.nbox;
+  nd.h0 = p.h0;
   nd.kb_w = p.kb_w;
   nd.kb_r = p.kb_r;
-  nd.kb_tile = p.kb_tile;
   nd.tiles = p.tiles;
-  nd.seg_slots = p.seg_slots;
-  nd.stage_tx = kTileABytes + p.b_region;
-  nd.idesc0 = idesc_bf16_f32(kTileM, p.n0);
-  nd.idesc1 = p.n1 > 0 ? idesc_bf16_f32(kTileM, p.n1) : 0u;
+  nd.pg_tiles = p.pg_tiles;
+  nd.seg_slots = L.seg_slots;
+  nd.gram_slots = L.gram_slots;
+  nd.pair_tx = 2 * (kTileABytes + p.b_region);
+  nd.idesc0 = idesc_bf16_f32(kPairM, p.n0);
+  nd.idesc1 = p.n1 > 0 ? idesc_bf16_f32(kPairM, p.n1) : 0u;
   nd.two_s = 2.0f * pr.s;
-
-  gd.partial = reinterpret_cast<float*>(ws_base + p.off_gp);
-  gd.g_out = gprime;
-  gd.g_lo = gprime_lo;
-  gd.tile_cnt = nd.tile_cnt;
-  gd.cnt_len = p.tiles * 4;
-  gd.r = static_cast<int>(pr.r);
-  gd.r8 = p.r8;
-  gd.kb = p.kb_gram;
-  gd.tiles_r = p.tiles_r;
-  gd.pairs = p.pairs;
-  gd.S = p.S;
-  gd.job_begin = gram_job_begin;
-  gd.half_s = 0.5f * pr.s;
+  nd.half_s = 0.5f * pr.s;
   return ok;
 }
 
@@ -514,69 +570,55 @@ dora_status_t run_tc_group(const dora_norm_problem_t* probs, int count, bool gro
     d_in[i] = probs[i].d_in;
     r[i] = probs[i].r;
   }
-  GroupLayout L;
-  if (!layout_group(d_out.data(), d_in.data(), r.data(), count, grouped, di->sms, L))
+  if (!ensure_tc_attrs()) return DORA_ERR_CUDA;
+  static thread_local GroupLayout L;
+  if (!layout_group(d_out.data(), d_in.data(), r.data(), count, grouped, norm_workers(), L))
     return DORA_ERR_UNSUPPORTED;
   if (ws == nullptr || ws_bytes < L.total_bytes || !aligned256(ws)) return DORA_ERR_WORKSPACE;
-  if (!ensure_tc_attrs(static_cast<int>(L.smem_bytes))) return DORA_ERR_CUDA;
 
   uint8_t* base = static_cast<uint8_t*>(ws);
   std::vector<NormProblemDev> nds(count);
-  std::vector<GramProblemDev> gds(count);
-  long long ub = 0;
-  int jb = 0;
-  for (int i = 0; i < count; ++i) {
-    if (!fill_descriptors(probs[i], L.plans[i], base, ub, jb, nds[i], gds[i]))
-      return DORA_ERR_INVALID_ARG;
-    nds[i].emit_sq = emit_sq ? 1 : 0;
-    nds[i].wave_begin = L.wave_of[i];
-    nds[i].wave_units = L.wave_units[i];
-    ub += L.plans[i].units;
-    jb += L.plans[i].pairs * L.plans[i].S;
-  }
-  const unsigned long long tmo = g_timeout_ns.load();
-  const int gram_smem = 1024 + kGramStages * kGramStageBytes + 256;
-  static thread_local WaveList wl;
-  wl.n = static_cast<int>(L.waves.size()) - 1;
-  for (int w = 0; w <= wl.n; ++w) wl.begin[w] = L.waves[w];
-  dora_status_t s;
-  const dim3 red_grid(kTileM * kTileM / 256, L.max_pairs, grouped ? count : 1);
-  if (!grouped) {
-    launch_pdl(gram_kernel<false>, dim3(L.gram_jobs), dim3(kTcThreads), gram_smem, st, gds[0],
-               static_cast<const GramProblemDev*>(nullptr), 1, tmo);
-    if ((s = launch_status()) != DORA_OK) return s;
-    launch_pdl(gram_reduce_kernel<false>, red_grid, dim3(256), 0, st, gds[0],
-               static_cast<const GramProblemDev*>(nullptr));
-    if ((s = launch_status()) != DORA_OK) return s;
-    {
-      TimedLaunch tl(st);
-      launch_pdl(norm_main_kernel<false>, dim3(L.ctas), dim3(kNormThreads), L.smem_bytes, st,
-                 nds[0], static_cast<const NormProblemDev*>(nullptr), 1, L.total_units, L.stages,
-                 L.b_region, static_cast<uint32_t>(L.tmem_cols), eps, wl, tmo, g_trace);
-      return launch_status();
+  for (int w = 0; w < L.sched.waves; ++w) {
+    const WaveInfo& W = L.sched.w[w];
+    long long at[3] = {0, 0, 0};
+    for (int i = W.m0; i < W.m1; ++i) {
+      if (!fill_descriptor(probs[i], L, i, at, base, nds[i])) return DORA_ERR_INVALID_ARG;
+      nds[i].emit_sq = emit_sq ? 1 : 0;
+      for (int ph = 0; ph < 3; ++ph) at[ph] += L.plans[i].units[ph];
     }
   }
-  NormProblemDev* ntab = reinterpret_cast<NormProblemDev*>(base);
-  GramProblemDev* gtab =
-      reinterpret_cast<GramProblemDev*>(base + align_up(sizeof(NormProblemDev) * count, 256));
-  if (cudaMemcpyAsync(ntab, nds.data(), sizeof(NormProblemDev) * count, cudaMemcpyHostToDevice,
-                      st) != cudaSuccess ||
-      cudaMemcpyAsync(gtab, gds.data(), sizeof(GramProblemDev) * count, cudaMemcpyHostToDevice,
-                      st) != cudaSuccess)
-    return DORA_ERR_CUDA;
-  launch_pdl(gram_kernel<true>, dim3(L.gram_jobs), dim3(kTcThreads), gram_smem, st, gds[0],
-             static_cast<const GramProblemDev*>(gtab), count, tmo);
-  if ((s = launch_status()) != DORA_OK) return s;
-  launch_pdl(gram_reduce_kernel<true>, red_grid, dim3(256), 0, st, gds[0],
-             static_cast<const GramProblemDev*>(gtab));
-  if ((s = launch_status()) != DORA_OK) return s;
-  {
-    TimedLaunch tl(st);
-    launch_pdl(norm_main_kernel<true>, dim3(L.ctas), dim3(kNormThreads), L.smem_bytes, st, nds[0],
-               static_cast<const NormProblemDev*>(ntab), count, L.total_units, L.stages,
-               L.b_region, static_cast<uint32_t>(L.tmem_cols), eps, wl, tmo, g_trace);
-    return launch_status();
+  const unsigned long long tmo = g_timeout_ns.load();
+  int* cnt = reinterpret_cast<int*>(base + L.table_bytes);
+  const NormProblemDev* table = nullptr;
+  if (grouped) {
+    NormProblemDev* ntab = reinterpret_cast<NormProblemDev*>(base);
+    if (cudaMemcpyAsync(ntab, nds.data(), sizeof(NormProblemDev) * count,
+                        cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return DORA_ERR_CUDA;
+    table = ntab;
   }
+  int max_tiles = 1;
+  for (const auto& p : L.plans) max_tiles = std::max(max_tiles, p.tiles);
+  const unsigned prep_blocks = static_cast<unsigned>(
+      std::min<long long>(64, ceil_div_ll(std::max(L.cnt_ints, max_tiles), 256)));
+  if (grouped)
+    launch_pdl(norm_prep_kernel<true>, dim3(prep_blocks), dim3(256), 0, st, cnt, L.cnt_ints,
+               nds[0], table, count, L.sched);
+  else
+    launch_pdl(norm_prep_kernel<false>, dim3(prep_blocks), dim3(256), 0, st, cnt, L.cnt_ints,
+               nds[0], table, count, L.sched);
+  dora_status_t s;
+  if ((s = launch_status()) != DORA_OK) return s;
+  TimedLaunch tl(st);
+  if (grouped)
+    launch_pdl(norm_main_kernel<true>, dim3(2 * L.sched.pairs), dim3(kNormThreads),
+               L.smem_bytes, st, nds[0], table, L.sched, L.stages, L.b_region,
+               static_cast<uint32_t>(L.tmem_cols), eps, tmo, g_trace);
+  else
+    launch_pdl(norm_main_kernel<false>, dim3(2 * L.sched.pairs), dim3(kNormThreads),
+               L.smem_bytes, st, nds[0], table, L.sched, L.stages, L.b_region,
+               static_cast<uint32_t>(L.tmem_cols), eps, tmo, g_trace);
+  return launch_status();
 }
 
 
@@ -679,10 +721,8 @@ size_t dora_factored_norm_workspace_size(int64_t d_out, int64_t d_in, int64_t r,
                                          dora_dtype_t dt) {
   if (d_out < 1 || d_in < 1 || r < 1 || r > DORA_MAX_RANK) return 0;
   if (dt == DORA_F32 || d_in % 8 != 0 || r % 8 != 0) return simt_workspace(r);
-  const DeviceInfo* di = device_info();
-  const int sms = (di != nullptr && di->sms > 0) ? di->sms : 148;
-  GroupLayout L;
-  if (!layout_group(&d_out, &d_in, &r, 1, false, sms, L)) return 0;
+  static thread_local GroupLayout L;
+  if (!layout_group(&d_out, &d_in, &r, 1, false, norm_workers(), L)) return 0;
   return std::max(L.total_bytes, simt_workspace(r));
 }
 
@@ -781,10 +821,9 @@ size_t dora_factored_norm_grouped_workspace_size(const dora_norm_problem_t* prob
     d_in[i] = problems[i].d_in;
     r[i] = problems[i].r;
   }
-  const DeviceInfo* di = device_info();
-  const int sms = (di != nullptr && di->sms > 0) ? di->sms : 148;
-  GroupLayout L;
-  if (!layout_group(d_out.data(), d_in.data(), r.data(), count, true, sms, L)) return 0;
+  static thread_local GroupLayout L;
+  if (!layout_group(d_out.data(), d_in.data(), r.data(), count, true, norm_workers(), L))
+    return 0;
   return L.total_bytes;
 }
 
@@ -1080,7 +1119,7 @@ dora_status_t dora_merge_weight(const void* W0, const void* A, const void* B, co
   const DeviceInfo* di = device_info();
   if (di == nullptr) return DORA_ERR_CUDA;
   if (!di->supported) return DORA_ERR_UNSUPPORTED;
-  if (!ensure_tc_attrs(0)) return DORA_ERR_CUDA;
+  if (!ensure_tc_attrs()) return DORA_ERR_CUDA;
   static thread_local MergeDev P;
   std::memset(&P, 0, sizeof(P));
   uint16_t* At = static_cast<uint16_t*>(ws);
@@ -1413,24 +1452,35 @@ namespace {
 constexpr size_t kStaticScratchBytes = size_t(4) << 20;
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-// Device address of g_static_scratch on the current device, looked up once
-// per device (the name is only a host-side stand-in in host code).
-void* static_scratch_address() {
-  static void* addr[kMaxDevices] = {};
+// Device address of g_static_scratch on the current device (the name is only
+// a host-side stand-in in host code).  Looked up on every call, so that the
+// address stays right after a device reset; the first lookup on a device can
+// load the module, which must not happen inside a stream capture, so that
+// first call is refused while `st` is capturing.
+void* static_scratch_address(cudaStream_t st) {
+  static bool seen[kMaxDevices] = {};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lk(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
-    if (e != cudaSuccess) {
-      note_error("cudaGetSymbolAddress(static scratch)", e);
+  if (!seen[dev]) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs != cudaStreamCaptureStatusNone) {
+      snprintf(t_last_error, sizeof(t_last_error),
+               "dora_compose_bwd_static: the first call on device %d looks up the scratch "
+               "array and must not be made during stream capture",
+               dev);
       return nullptr;
     }
-    addr[dev] = p;
   }
-  return addr[dev];
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+  if (e != cudaSuccess) {
+    note_error("cudaGetSymbolAddress(static scratch)", e);
+    return nullptr;
+  }
+  seen[dev] = true;
+  return p;
 }
 }  // namespace
 }  // namespace dora
@@ -1453,8 +1503,14 @@ extern "C" dora_status_t dora_compose_bwd_static(const void* dy, const void* bas
   const DeviceInfo* di = device_info();
   if (di == nullptr) return DORA_ERR_CUDA;
   if (!di->supported) return DORA_ERR_UNSUPPORTED;
-  void* scratch = static_scratch_address();
-  if (scratch == nullptr) return DORA_ERR_CUDA;
+  void* scratch = static_scratch_address(reinterpret_cast<cudaStream_t>(stream));
+  if (scratch == nullptr) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    return (cudaStreamIsCapturing(reinterpret_cast<cudaStream_t>(stream), &cs) == cudaSuccess &&
+            cs != cudaStreamCaptureStatusNone)
+               ? DORA_ERR_UNSUPPORTED
+               : DORA_ERR_CUDA;
+  }
   // Every slot of the partial table the kernels read is written by the same
   // call first, so nothing has to be cleared between calls.
   return dora_compose_bwd(dy, base, lora, m, n, s, eps, dt, T, d_out, d_base, d_lora, dm,

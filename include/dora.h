@@ -308,9 +308,13 @@ dora_status_t dora_merge_weight(const void *W0, const void *A, const void *B, co
  *     see dora_compose_bwd_workspace_size) are rejected with
  *     DORA_ERR_UNSUPPORTED before anything is launched; dora_last_error()
  *     then says how much scratch the shape needs.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream
- *     capture.
+ *   - Every call looks up the array's device address (cudaGetSymbolAddress),
+ *     so the call stays valid after a device reset.  The first lookup on a
+ *     device can load the library's device code, which a stream capture does
+ *     not allow: a first call made on a capturing stream returns
+ *     DORA_ERR_UNSUPPORTED (dora_last_error() says why) and launches
+ *     nothing; make the first call on each device, and the first after a
+ *     device reset, outside any capture.
  *   - All calls share the one array: calls that overlap on the GPU (other
  *     streams, other host threads) race and give wrong results.  Nothing in
  *     the array needs to start at zero: each call writes every slot it
@@ -353,11 +357,18 @@ void dora_set_wait_timeout_ns(uint64_t ns);
  * graph, the events are recorded as event-record nodes of the graph, so each
  * replay re-records them around the kernel. */
 void dora_set_timing_events(void *before, void *after);
-/* Diagnostics: when `buf` is non-NULL, later norm calls record 8 uint64 words
- * per CTA of the fused norm GEMM into it (device memory, 8 * 148 words for
- * one B200): entry and exit %globaltimer, cycles the MMA issuer waited for
- * operands and for the accumulator, k-blocks issued, segments, SM id.  NULL
- * turns it off.  The buffer must outlive every call made while it is set. */
+/* Diagnostics: when `buf` is non-NULL, later norm calls record 16 uint64
+ * words per CTA of the fused norm kernel into it (device memory, 16 * 148
+ * words for one B200; a word the kernel does not set keeps its value):
+ * [0] entry and [1] exit %globaltimer, cycles the MMA issuer waited [2] for
+ * operands and [3] for the accumulator, [4] k-blocks issued, [5] segments,
+ * [6] SM id, [7] cycles waited for operands over the first four k-blocks,
+ * then %globaltimer when [8] the MMA issuer starts its W0 units and [9] its
+ * G units, and, for the first Gram segment of the CTA, when its epilogue
+ * [10] holds the accumulator, [11] has posted its partial, [12] sees every
+ * partial of the pseudo-tile posted and [13] has written its rows of G'.
+ * NULL turns it off.  The buffer must outlive every call made while it is
+ * set. */
 void dora_set_trace_buffer(void *buf);
 /* Launches one thread that waits, with the same bounded wait the
  * tensor-core pipelines use, on a barrier that nothing ever signals, giving

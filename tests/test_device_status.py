@@ -57,4 +57,4 @@ def test_launch_counter_counts_kernels():
     before = dora.dora_launch_count()
     dora.dora_factored_norm(W0.cuda(), A.cuda(), B.cuda(), 2.0)
     torch.cuda.synchronize()
-    assert dora.dora_launch_count() - before == 3  # gram, gram reduce, norm GEMM (+ finalize)
+    assert dora.dora_launch_count() - before == 2  # counter reset, fused norm kernel (Gram, GEMM, finalize)

@@ -127,25 +127,24 @@ def test_norm_4096_r64_all_rows():
     _check(W0, A, B, m, s, eps, n, g, 1e-3, "norm_4096_r64")
 
 
-@pytest.mark.parametrize("key", ["headline_8192_r384", "mlp_up_25600x5120_r384"])
-def test_norm_large_modules_sampled_rows(key):
-    w = synth.WORKLOADS[key]
+def test_norm_mlp_up_25600x5120_all_rows():
+    """Every row of the 25600 x 5120, r = 384 module (its norm spans many
+    pair tiles and stream-K segment boundaries), against the oracle's dense
+    norm taken over row blocks of 2048."""
+    w = synth.WORKLOADS["mlp_up_25600x5120_r384"]
     W0, A, B = synth.module_weights(w, device="cuda")
     m = synth.magnitude_from_base_rows(w, W0)
     s, eps = w.modules[0].s, synth.eps_for("bf16")
     n, g = dora.dora_factored_norm(W0, A, B, s, m, eps)
     torch.cuda.synchronize()
     d_out = W0.shape[0]
-    gen = torch.Generator().manual_seed(12)
-    rows = torch.cat([torch.arange(0, 130), torch.arange(d_out - 130, d_out),
-                      torch.randperm(d_out, generator=gen)[:256]]).unique().sort().values
-    rc = rows.cuda()
-    W, Aa, Bb = _np(W0[rc]), _np(A), _np(B[rc])
-    ref = oracle.rows_dense_row_norm(W, Aa, Bb, s)
-    check_rel(_np(n[rc]), ref, 1e-3, f"{key} n")
-    rg, _, _ = oracle.magnitude_scale(_np(m[rc]), ref, eps)
-    check_rel(_np(g[rc]), rg, 1e-3, f"{key} g")
-    assert torch.isfinite(n).all() and (n > 0).all()
+    Aa = _np(A)
+    ref = np.concatenate([oracle.rows_dense_row_norm(_np(W0[r0:r0 + 2048]), Aa,
+                                                     _np(B[r0:r0 + 2048]), s)
+                          for r0 in range(0, d_out, 2048)])
+    check_rel(_np(n), ref, 1e-3, "mlp_up n")
+    rg, _, _ = oracle.magnitude_scale(_np(m), ref, eps)
+    check_rel(_np(g), rg, 1e-3, "mlp_up g")
 
 
 def test_headline_norm_then_compose_full_path():

@@ -3,25 +3,35 @@ a workspace (a C host program without a device allocator, or a loop where
 cudaMalloc is not allowed because it can synchronise the device).  Its dm
 column partials live in the library's fixed device array instead.
 
-The test calls the entry point through the C ABI twice in a row, on
-different shapes and dtypes so that the second call reuses the array the
-first one wrote, and checks each result against dora_compose_bwd (the
-workspace entry point) with the same tolerances as the other parity tests.
-It also checks that a shape needing more scratch than the array holds is
-rejected before anything runs.  Collected last (file name) so that a run
-stopping at the first failure has run every other test first.
+The tests call the entry point through the C ABI several times in a row, on
+different shapes and dtypes so that each call reuses the array the one before
+wrote, and check every result against the fp64 oracle (the bars of the other
+parity tests) and against dora_compose_bwd (the workspace entry point).  The
+sequence includes T = 0, and a shape whose partial table is exactly as large
+as the array right after a call that used more row chunks (so a stale row
+would show).  A shape needing more scratch than the array holds is rejected
+before anything runs, and a first call made while its stream is being
+captured is refused.  Collected last (file name) so that a run stopping at
+the first failure has run every other test first.
 """
 import ctypes
+import os
+import subprocess
+import sys
 
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import dora_adapter_factored_b200 as dora
 from dora_adapter_factored_b200 import _abi
 from tolerances import check_bf16, check_dm, check_f32
 
 pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SCRATCH_BYTES = 4 << 20  # the array's size, as include/dora.h states it
 
 
 def _np(t):
@@ -38,32 +48,95 @@ def _inputs(T, d_out, dtype, seed):
     return dy, base, lora, m.cuda(), n.float().cuda()
 
 
-@pytest.mark.parametrize("calls", [[(300, 4096, torch.bfloat16, 1), (1000, 2048, torch.bfloat16, 2),
-                                    (77, 264, torch.float32, 3)]])
-def test_static_scratch_backward_matches_workspace_backward(calls):
-    s, eps = 2.0, 2.0 ** -7
+def _check_against_oracle_and_workspace_call(T, d_out, dtype, seed, s=2.0, eps=2.0 ** -7):
+    dy, base, lora, m, n = _inputs(T, d_out, dtype, seed)
+    got_db, got_dl, got_dm = dora.dora_compose_bwd_static(dy, base, lora, m, n, s, eps)
+    ws_db, ws_dl, ws_dm = dora.dora_compose_bwd(dy, base, lora, m, n, s, eps)
+    torch.cuda.synchronize()
+    assert dora.dora_get_device_status() == 0
+    d, b, l = _np(dy), _np(base), _np(lora)
+    mm, nn = _np(m), _np(n)
+    r_db, r_dl, r_dm = oracle.compose_bwd(d, b, l, mm, nn, s, eps)
+    nc = np.maximum(nn, eps)
+    chk = check_bf16 if dtype == torch.bfloat16 else check_f32
+    what = f"{T}x{d_out} {dtype}"
+    chk(_np(got_db), r_db, np.abs(r_db), f"d_base {what}")
+    chk(_np(got_dl), r_dl, np.abs(r_dl), f"d_lora {what}")
+    scale = np.sum(np.abs(d * (b + s * l)), axis=0) / nc
+    check_dm(_np(got_dm), r_dm, scale, f"dm {what}")
+    # The same computation as the workspace call, on the same inputs.
+    chk(_np(got_db), _np(ws_db), np.abs(_np(ws_db)), f"d_base vs workspace call {what}")
+    chk(_np(got_dl), _np(ws_dl), np.abs(_np(ws_dl)), f"d_lora vs workspace call {what}")
+    check_dm(_np(got_dm), _np(ws_dm), scale, f"dm vs workspace call {what}")
+    if T == 0:
+        assert torch.count_nonzero(got_dm) == 0
+
+
+def test_static_scratch_backward_matches_oracle_on_consecutive_calls():
+    # [4096, 1024] bf16 uses many row chunks; [8, 2^20] bf16 then needs
+    # exactly the whole array (one chunk of 2^20 fp32 partials); T = 0 and a
+    # ragged fp32 shape follow.
+    limit = (8, 1 << 20, torch.bfloat16)
+    assert dora.dora_compose_bwd_workspace_size(limit[0], limit[1], limit[2]) == SCRATCH_BYTES
+    assert dora.dora_compose_bwd_workspace_size(4096, 1024, torch.bfloat16) < SCRATCH_BYTES
+    calls = [(300, 4096, torch.bfloat16, 1), (4096, 1024, torch.bfloat16, 2),
+             (*limit, 3), (0, 4096, torch.bfloat16, 4), (1000, 2048, torch.bfloat16, 5),
+             (77, 264, torch.float32, 6)]
     for T, d_out, dtype, seed in calls:
-        dy, base, lora, m, n = _inputs(T, d_out, dtype, seed)
-        ref_db, ref_dl, ref_dm = dora.dora_compose_bwd(dy, base, lora, m, n, s, eps)
-        got_db, got_dl, got_dm = dora.dora_compose_bwd_static(dy, base, lora, m, n, s, eps)
-        torch.cuda.synchronize()
-        assert dora.dora_get_device_status() == 0
-        chk = check_bf16 if dtype == torch.bfloat16 else check_f32
-        chk(_np(got_db), _np(ref_db), np.abs(_np(ref_db)), f"d_base {T}x{d_out}")
-        chk(_np(got_dl), _np(ref_dl), np.abs(_np(ref_dl)), f"d_lora {T}x{d_out}")
-        d, b, l = _np(dy), _np(base), _np(lora)
-        nc = np.maximum(_np(n), eps)
-        check_dm(_np(got_dm), _np(ref_dm), np.sum(np.abs(d * (b + s * l)), axis=0) / nc,
-                 f"dm {T}x{d_out}")
+        _check_against_oracle_and_workspace_call(T, d_out, dtype, seed)
 
 
 def test_static_scratch_rejects_shapes_beyond_the_array():
     lib = dora.load_library()
     p = ctypes.c_void_p(0x10000)  # never dereferenced: the size check comes first
-    d_out = 1 << 21               # one chunk of 2^21 fp32 partials = 8 MiB > 4 MiB
-    st = lib.dora_compose_bwd_static(p, ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000), p, p,
-                                     2.0, 0.0, _abi.DORA_BF16, 64, d_out,
-                                     ctypes.c_void_p(0x40000), ctypes.c_void_p(0x50000),
-                                     ctypes.c_void_p(0x60000), None)
-    assert st == _abi.DORA_ERR_UNSUPPORTED
-    assert b"needs" in lib.dora_last_error()
+    for T, d_out in ((8, (1 << 20) + 8), (64, 1 << 21)):
+        assert dora.dora_compose_bwd_workspace_size(T, d_out, torch.bfloat16) > SCRATCH_BYTES
+        st = lib.dora_compose_bwd_static(p, ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000),
+                                         p, p, 2.0, 0.0, _abi.DORA_BF16, T, d_out,
+                                         ctypes.c_void_p(0x40000), ctypes.c_void_p(0x50000),
+                                         ctypes.c_void_p(0x60000), None)
+        assert st == _abi.DORA_ERR_UNSUPPORTED
+        assert b"needs" in lib.dora_last_error()
+
+
+_CAPTURE_SCRIPT = r"""
+import sys
+sys.path.insert(0, sys.argv[1])
+import torch
+import dora_adapter_factored_b200 as dora
+from dora_adapter_factored_b200 import _abi
+T, d = 64, 1024
+x = [torch.randn(T, d, device="cuda").bfloat16() for _ in range(3)]
+n = torch.ones(d, device="cuda")
+m = n * 1.001
+outs = [torch.empty(T, d, device="cuda", dtype=torch.bfloat16) for _ in range(2)]
+dm = torch.empty(d, device="cuda")
+lib = dora.load_library()
+def call(stream):
+    return lib.dora_compose_bwd_static(x[0].data_ptr(), x[1].data_ptr(), x[2].data_ptr(),
+                                       m.data_ptr(), n.data_ptr(), 2.0, 2.0 ** -7,
+                                       _abi.DORA_BF16, T, d, outs[0].data_ptr(),
+                                       outs[1].data_ptr(), dm.data_ptr(), stream)
+torch.cuda.synchronize()
+s = torch.cuda.Stream()
+g = torch.cuda.CUDAGraph()
+with torch.cuda.graph(g, stream=s):
+    first = call(s.cuda_stream)
+print("first", first, lib.dora_last_error().decode())
+second = call(torch.cuda.current_stream().cuda_stream)
+torch.cuda.synchronize()
+print("second", second)
+"""
+
+
+def test_static_scratch_first_call_refused_during_capture():
+    # A fresh process, so that this is the library's first static call on the
+    # device: made on a capturing stream it must be refused, launch nothing
+    # and leave the capture usable; the next call outside the capture works.
+    r = subprocess.run([sys.executable, "-c", _CAPTURE_SCRIPT, ROOT], capture_output=True,
+                       text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = {ln.split()[0]: ln.split() for ln in r.stdout.splitlines() if ln.strip()}
+    assert int(lines["first"][1]) == _abi.DORA_ERR_UNSUPPORTED, r.stdout
+    assert "capture" in r.stdout
+    assert int(lines["second"][1]) == _abi.DORA_OK, r.stdout
