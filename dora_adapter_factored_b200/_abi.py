@@ -37,7 +37,7 @@ EXPORTED = (
     "dora_compose_fwd_train", "dora_compose_bwd_inner", "dora_compose_bwd_frozen",
     "dora_compose_fwd_grouped", "dora_compose_bwd_grouped_workspace_size",
     "dora_compose_bwd_grouped", "dora_merge_weight_workspace_size", "dora_merge_weight",
-    "dora_factored_norm_sq", "dora_norm_finalize",
+    "dora_factored_norm_sq", "dora_norm_finalize", "dora_compose_fwd_delta",
 )
 
 
@@ -100,6 +100,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.dora_compose_fwd.argtypes = [c_vp, c_vp, c_vp, c_vp, c_f, c_f, c_i, c_i64, c_i64, c_vp,
                                          c_vp]
         lib.dora_compose_fwd.restype = c_i
+        lib.dora_compose_fwd_delta.argtypes = [c_vp, c_vp, c_vp, c_vp, c_f, c_f, c_i, c_i64, c_i64,
+                                               c_vp, c_vp]
+        lib.dora_compose_fwd_delta.restype = c_i
         lib.dora_compose_bwd_workspace_size.argtypes = [c_i64, c_i64, c_i]
         lib.dora_compose_bwd_workspace_size.restype = c_sz
         lib.dora_compose_bwd.argtypes = [c_vp, c_vp, c_vp, c_vp, c_vp, c_f, c_f, c_i, c_i64, c_i64,
@@ -324,6 +327,24 @@ def dora_compose_fwd(base: torch.Tensor, lora: torch.Tensor, m: torch.Tensor, n:
         float(eps), dt, T, d_out, _dev(y, "y", base.dtype, (T, d_out)), _stream(stream)),
         "dora_compose_fwd")
     return y
+
+
+def dora_compose_fwd_delta(base: torch.Tensor, lora: torch.Tensor, m: torch.Tensor,
+                           n: torch.Tensor, s: float, eps: float = 0.0,
+                           dy_out: Optional[torch.Tensor] = None, stream=None):
+    """dY = (g - 1) base + g s lora with g = m / max(n, eps) (the caller adds Y_base)."""
+    lib = load_library()
+    dt = _dtype_code(base)
+    T, d_out = base.shape
+    if dy_out is None:
+        dy_out = torch.empty_like(base)
+    _check(lib.dora_compose_fwd_delta(
+        _dev(base, "base", base.dtype), _dev(lora, "lora", base.dtype, (T, d_out)),
+        _dev(m, "m", torch.float32, (d_out,)), _dev(n, "n", torch.float32, (d_out,)), float(s),
+        float(eps), dt, T, d_out, _dev(dy_out, "dy_out", base.dtype, (T, d_out)),
+        _stream(stream)),
+        "dora_compose_fwd_delta")
+    return dy_out
 
 
 def dora_compose_bwd_workspace_size(T: int, d_out: int, dtype: torch.dtype) -> int:

@@ -162,8 +162,14 @@ __device__ __forceinline__ void fwd_coefficients(const float* __restrict__ m,
   }
 }
 
-// y = base + ((g - 1) base + (g s) lora); with kInner also inner = base + s lora.
-template <typename T, int VEC, typename Idx, bool kInner>
+// Outputs of the forward pass.
+enum FwdOut : int {
+  kFwdY = 0,       // y = base + ((g - 1) base + (g s) lora)
+  kFwdYInner = 1,  // y, and inner = base + s lora
+  kFwdDelta = 2,   // dY = (g - 1) base + (g s) lora only, for a caller that adds Y_base
+};
+
+template <typename T, int VEC, typename Idx, int kOut>
 __device__ __forceinline__ void fwd_rows(const T* __restrict__ base, const T* __restrict__ lora,
                                          const float (&gm1)[VEC], const float (&gs)[VEC], float s,
                                          long long t, long long stride, long long T_rows,
@@ -190,10 +196,13 @@ __device__ __forceinline__ void fwd_rows(const T* __restrict__ base, const T* __
         P::unpack(rb[u], b);
         P::unpack(rl[u], l);
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) o[e] = b[e] + fmaf(gm1[e], b[e], gs[e] * l[e]);
+        for (int e = 0; e < VEC; ++e) {
+          const float d = fmaf(gm1[e], b[e], gs[e] * l[e]);
+          o[e] = kOut == kFwdDelta ? d : b[e] + d;
+        }
         const Idx off = static_cast<Idx>(tt) * static_cast<Idx>(d_out) + static_cast<Idx>(col0);
         P::store(y + off, P::pack(o));
-        if (kInner) {
+        if (kOut == kFwdYInner) {
           float in[VEC];
 #pragma unroll
           for (int e = 0; e < VEC; ++e) in[e] = fmaf(s, l[e], b[e]);
@@ -304,10 +313,10 @@ __device__ __forceinline__ void colsum_column(const float* __restrict__ partial,
 // ---------------------------------------------------------------------------
 
 // y = base + ((g - 1) base + (g s) lora), (g - 1) = (m - n_c)/n_c, g = m/n_c;
-// with kInner also inner = base + s lora.  Idx is the element-offset type:
-// 32-bit when T * d_out < 2^31 (fewer live registers per in-flight row),
-// 64-bit otherwise.
-template <typename T, int VEC, typename Idx, bool kInner>
+// kOut adds inner = base + s lora, or writes dY = y - base alone (FwdOut).
+// Idx is the element-offset type: 32-bit when T * d_out < 2^31 (fewer live
+// registers per in-flight row), 64-bit otherwise.
+template <typename T, int VEC, typename Idx, int kOut>
 __global__ void __launch_bounds__(kStreamThreads, 2)
     compose_fwd_kernel(const T* __restrict__ base, const T* __restrict__ lora,
                        const float* __restrict__ m, const float* __restrict__ n, float s,
@@ -321,7 +330,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
   fwd_coefficients<VEC>(m, n, s, eps, col0, gm1, gs);
   const long long stride = static_cast<long long>(gridDim.y) * blockDim.y;
   const long long t = static_cast<long long>(blockIdx.y) * blockDim.y + threadIdx.y;
-  fwd_rows<T, VEC, Idx, kInner>(base, lora, gm1, gs, s, t, stride, T_rows, d_out, col0, y, inner);
+  fwd_rows<T, VEC, Idx, kOut>(base, lora, gm1, gs, s, t, stride, T_rows, d_out, col0, y, inner);
 }
 
 // d_base = g dy, d_lora = (g s) dy, and (unless frozen) per-block column
@@ -425,10 +434,10 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
   const T* base = static_cast<const T*>(it.in0);
   const T* lora = static_cast<const T*>(it.in1);
   if (it.out1 != nullptr)
-    fwd_rows<T, VEC, Idx, true>(base, lora, gm1, gs, it.s, t, stride, it.T, it.d_out, col0,
+    fwd_rows<T, VEC, Idx, kFwdYInner>(base, lora, gm1, gs, it.s, t, stride, it.T, it.d_out, col0,
                                 static_cast<T*>(it.out0), static_cast<T*>(it.out1));
   else
-    fwd_rows<T, VEC, Idx, false>(base, lora, gm1, gs, it.s, t, stride, it.T, it.d_out, col0,
+    fwd_rows<T, VEC, Idx, kFwdY>(base, lora, gm1, gs, it.s, t, stride, it.T, it.d_out, col0,
                                  static_cast<T*>(it.out0), nullptr);
 }
 

@@ -195,6 +195,38 @@ bool make_tmap_bf16_pairslab(CUtensorMap* map, const void* ptr, uint64_t h, uint
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// `parts` stacked row-major bf16 matrices [rows, cols] (`ld` elements per
+// row, rows x ld per part) as {cols, rows, parts}, loaded in boxes of
+// box_cols x box_rows x 1 with 128-byte swizzle; out-of-range elements read
+// as zero.
+bool make_tmap_bf16_parts(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols,
+                          uint64_t ld, uint64_t parts, uint32_t box_cols, uint32_t box_rows) {
+  auto enc = tmap_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {cols, rows, parts};
+  cuuint64_t strides[2] = {ld * 2, rows * ld * 2};
+  cuuint32_t box[3] = {box_cols, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The pair-slab view of `parts` stacked [4 h, cols] matrices: {cols, h, 2, 2,
+// parts}, box {box_cols, h, 1, 2, 1} (one CTA's halves of both chunks).
+bool make_tmap_bf16_pairslab_parts(CUtensorMap* map, const void* ptr, uint64_t h, uint64_t cols,
+                                   uint64_t ld, uint64_t parts, uint32_t box_cols) {
+  auto enc = tmap_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[5] = {cols, h, 2, 2, parts};
+  cuuint64_t strides[4] = {ld * 2, h * ld * 2, 2 * h * ld * 2, 4 * h * ld * 2};
+  cuuint32_t box[5] = {box_cols, static_cast<cuuint32_t>(h), 1, 2, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Row-major bf16 matrix [rows, cols] with `ld` elements per row, loaded in
 // boxes of box_cols x box_rows with 128-byte swizzle; out-of-range elements
 // read as zero.
@@ -219,10 +251,14 @@ struct ModulePlan {
   uint32_t b_region;
   // K and tiles (tiles of 256 rows; Gram pseudo-tiles of 256 rows of A)
   int kb_w, kb_r, tiles, pg_tiles, r8;
-  long long units[3];  // Gram, W0 and G units
+  // Gram blocks: nc columns of G each (gchunks MMA chunks of gn), gj0 of
+  // them for pseudo-tile 0; d_in is split into gkp parts (a job per block
+  // and part), and a job costs `gram_cost` W0 units in the schedule
+  int nc, gchunks, gn, gj0, gblocks, gkp, gram_cost;
+  long long units[3];  // Gram jobs, W0 units and G units
   // workspace (byte offsets from the workspace base) and counters (ints
   // from the start of the counter block)
-  size_t off_g, off_gp, off_np, off_tw, cnt_off;
+  size_t off_g, off_np, off_tw, cnt_off;
 };
 
 // One accumulator chunk up to N = 256, else two equal chunks; each chunk's
@@ -243,6 +279,22 @@ void plan_n_side(int r, ModulePlan& p) {
   p.tmem_cols = tc;
 }
 
+// What a Gram job costs in W0 units of its module: a k-block stages
+// 256 + nc rows of A against 256 + n_pad rows (W0 and A) for a W0 unit, and
+// the feed of a CTA's stages sets the pace; plus the job's epilogue.
+constexpr int kGramJobCharge = 3;
+constexpr int kMaxGramParts = 16;
+
+// Splits d_in into kp parts: kp jobs per Gram block, and the G units run
+// over every part of S.
+void set_gram_split(ModulePlan& p, int kp) {
+  p.gkp = kp;
+  p.units[kPhaseGram] = static_cast<long long>(p.gblocks) * kp;
+  p.units[kPhaseG] = static_cast<long long>(p.tiles) * 2 * p.kb_r * kp;
+  p.gram_cost = static_cast<int>(
+      ceil_div_ll(ceil_div_ll(p.kb_w, kp) * (256 + p.nc), 256 + p.n_pad) + kGramJobCharge);
+}
+
 void plan_module(int64_t d_out, int64_t d_in, int64_t r, ModulePlan& p) {
   plan_n_side(static_cast<int>(r), p);
   p.kb_w = static_cast<int>(ceil_div_ll(d_in, kBlockK));
@@ -250,32 +302,70 @@ void plan_module(int64_t d_out, int64_t d_in, int64_t r, ModulePlan& p) {
   p.tiles = static_cast<int>(ceil_div_ll(d_out, kPairM));
   p.pg_tiles = static_cast<int>(ceil_div_ll(r, kPairM));
   p.r8 = round_up_int(static_cast<int>(r), 8);
-  p.units[kPhaseGram] = static_cast<long long>(p.pg_tiles) * p.kb_w;
+  // Gram blocks of 256 columns as two chunks of 128 (one per MMA issuer)
+  // where the slab region holds them, else one chunk of up to 128.
+  if (p.n_pad >= 2 * kGramCols) {
+    p.nc = 2 * kGramCols;
+    p.gchunks = 2;
+  } else {
+    p.nc = std::min(kGramCols, p.n_pad);
+    p.gchunks = 1;
+  }
+  p.gn = p.nc / p.gchunks;
+  p.gj0 = gram_jobs_of_tile(static_cast<int>(r), p.nc, 0);
+  p.gblocks = p.gj0 + (p.pg_tiles > 1 ? gram_jobs_of_tile(static_cast<int>(r), p.nc, 1) : 0);
   p.units[kPhaseW0] = static_cast<long long>(p.tiles) * p.kb_w;
-  p.units[kPhaseG] = static_cast<long long>(p.tiles) * 2 * p.kb_r;
+  set_gram_split(p, 1);
 }
 
-int module_counters(const ModulePlan& p) { return p.tiles * 8 + p.pg_tiles * 2 + 1; }
+int module_counters(const ModulePlan& p) { return p.tiles * 2 + 1; }
 
-// Re-read operands (A and G') of one wave of the grouped norm: well inside
+// Re-read operands (A and S) of one wave of the grouped norm: well inside
 // the 126 MB L2, which also carries the W0 stream.
 constexpr size_t kWaveBudgetBytes = size_t(40) << 20;
 
+// Runs of equal Gram-job cost of modules [m0, m1), in order.
+int gram_runs(const std::vector<ModulePlan>& plans, int m0, int m1) {
+  int runs = 0, last = -1;
+  for (int i = m0; i < m1; ++i) {
+    if (plans[i].units[kPhaseGram] == 0) continue;
+    if (plans[i].gram_cost != last) ++runs;
+    last = plans[i].gram_cost;
+  }
+  return runs;
+}
+
 // Splits the modules, in order, into waves: a wave closes before a module
-// that would take its re-read operands (A, G'_hi, G'_lo) past `budget`
-// bytes, provided it already holds at least `min_w` W0 units; a last wave
-// with fewer joins the one before.  Returns the waves' first modules (and
-// the module count at the end).
+// that would take its re-read operands (A, S_hi, S_lo) past the budget,
+// provided it already holds at least `min_w` W0 units, and before one that
+// would give its Gram jobs more than kMaxGramRuns runs of equal cost; a last
+// wave with fewer W0 units joins the one before where it can.  The budget
+// is `budget` evened out over the waves it takes, so that no wave is left
+// with a small remainder.  Returns the waves' first modules (and the module
+// count at the end).
 std::vector<int> plan_waves(const std::vector<ModulePlan>& plans, const int64_t* d_in,
                             const int64_t* r, long long min_w, size_t budget) {
+  const int count = static_cast<int>(plans.size());
+  std::vector<size_t> mbytes(count);
+  size_t total = 0, largest = 0;
+  for (int i = 0; i < count; ++i) {
+    mbytes[i] = static_cast<size_t>(r[i]) * d_in[i] * 2 +
+                2 * static_cast<size_t>(r[i]) * plans[i].r8 * 2;
+    total += mbytes[i];
+    largest = std::max(largest, mbytes[i]);
+  }
+  if (budget != SIZE_MAX && total > budget) {
+    const size_t waves = (total + budget - 1) / budget;
+    budget = std::max(largest, total / waves + total / waves / 12);
+  }
   std::vector<int> begin{0};
   long long wunits = 0;
   size_t bytes = 0;
-  const int count = static_cast<int>(plans.size());
   for (int i = 0; i < count; ++i) {
-    const size_t mb = static_cast<size_t>(r[i]) * d_in[i] * 2 +
-                      2 * static_cast<size_t>(r[i]) * plans[i].r8 * 2;
-    if (wunits > 0 && bytes + mb > budget && wunits >= min_w) {
+    const size_t mb = mbytes[i];
+    const bool over_budget = bytes + mb > budget && wunits >= min_w;
+    const bool over_runs = gram_runs(plans, begin.back(), i + 1) > kMaxGramRuns;
+    if (wunits > 0 && (over_budget || over_runs)) {
       begin.push_back(i);
       wunits = 0;
       bytes = 0;
@@ -283,7 +373,9 @@ std::vector<int> plan_waves(const std::vector<ModulePlan>& plans, const int64_t*
     wunits += plans[i].units[kPhaseW0];
     bytes += mb;
   }
-  if (begin.size() > 1 && wunits < min_w) begin.pop_back();
+  if (begin.size() > 1 && wunits < min_w &&
+      gram_runs(plans, begin[begin.size() - 2], count) <= kMaxGramRuns)
+    begin.pop_back();
   begin.push_back(count);
   return begin;
 }
@@ -298,30 +390,67 @@ bool sched_valid(const WaveInfo& w, int pairs) {
   return true;
 }
 
-// Units a Gram pair's W0 share is cut by for each Gram segment it ends
-// (posting the partial and reducing its rows of G' take about that long).
-constexpr int kGramEpilogueUnits = 10;
+// The Gram jobs of a wave: one per pair while there are pairs enough (so
+// the Gram is done early), as runs of equal cost for the W0 split.
+// Units of slack between a Gram job's end (by the cost model) and the first
+// G units of any pair: the job's S still has to be published.
+constexpr int kGramSlackUnits = 4;
 
-// The Gram pairs of a wave: about half a pair's share of work each (so the
-// Gram is done early), more when the schedule needs them.
-bool choose_gram_pairs(WaveInfo& w, int pairs) {
-  const double share = static_cast<double>(w.n[0] + w.n[1] + w.n[2]) / pairs;
-  int J = static_cast<int>(std::ceil(2.0 * w.n[0] / std::max(1.0, share)));
-  J = std::min(std::max(J, 1), pairs);
-  for (; J <= pairs; ++J) {
-    w.J = J;
-    w.gw = w.n[0] + static_cast<long long>(J) * kGramEpilogueUnits;
-    if (sched_valid(w, pairs)) return true;
-    w.gw = w.n[0];
-    if (sched_valid(w, pairs)) return true;
+// Work of the wave (W0 units; Gram jobs at their cost; G units), with the
+// modules' current splits.
+long long wave_work(const WaveInfo& w, const std::vector<ModulePlan>& plans) {
+  long long work = 0;
+  for (int i = w.m0; i < w.m1; ++i)
+    work += plans[i].units[kPhaseW0] + plans[i].units[kPhaseG] +
+            plans[i].units[kPhaseGram] * plans[i].gram_cost;
+  return work;
+}
+
+bool plan_gram(WaveInfo& w, std::vector<ModulePlan>& plans, int pairs) {
+  // Each module's parts of d_in: the fewest (every part adds the module's G
+  // units once more) for which a job ends before any pair reaches its G
+  // units, with some slack.
+  for (int i = w.m0; i < w.m1; ++i) set_gram_split(plans[i], 1);
+  for (int i = w.m0; i < w.m1; ++i) {
+    ModulePlan& p = plans[i];
+    const int kp_max = std::max(1, std::min(kMaxGramParts, p.kb_w / 2));
+    for (int kp = 1; kp <= kp_max; ++kp) {
+      set_gram_split(p, kp);
+      long long g = 0;
+      for (int m = w.m0; m < w.m1; ++m) g += plans[m].units[kPhaseG];
+      const double share = static_cast<double>(wave_work(w, plans)) / pairs;
+      if (p.gram_cost + kGramSlackUnits <= share - static_cast<double>(g) / pairs) break;
+    }
   }
-  return false;
+  for (int ph = 0; ph < 3; ++ph) {
+    w.n[ph] = 0;
+    for (int i = w.m0; i < w.m1; ++i) w.n[ph] += plans[i].units[ph];
+  }
+  w.runs = 0;
+  w.gw = 0;
+  long long jobs = 0;
+  for (int i = w.m0; i < w.m1; ++i) {
+    const ModulePlan& p = plans[i];
+    if (p.units[kPhaseGram] == 0) continue;
+    if (w.runs > 0 && w.run_cost[w.runs - 1] == p.gram_cost) {
+      w.run_end[w.runs - 1] += static_cast<int>(p.units[kPhaseGram]);
+    } else {
+      if (w.runs == kMaxGramRuns) return false;
+      w.run_cost[w.runs] = p.gram_cost;
+      w.run_end[w.runs] = static_cast<int>(jobs + p.units[kPhaseGram]);
+      ++w.runs;
+    }
+    jobs += p.units[kPhaseGram];
+    w.gw += p.units[kPhaseGram] * p.gram_cost;
+  }
+  w.J = static_cast<int>(std::min<long long>(jobs, pairs));
+  return sched_valid(w, pairs);
 }
 
 struct GroupLayout {
   std::vector<ModulePlan> plans;
   NormSched sched;
-  int seg_slots = 1, gram_slots = 1;
+  int seg_slots = 1;
   uint32_t b_region = 0;
   int tmem_cols = 32;
   int stages = 0;
@@ -348,11 +477,13 @@ bool layout_group(const int64_t* d_out, const int64_t* d_in, const int64_t* r, i
   // epilogue), at most one per W0 unit; fewer if some wave cannot give every
   // pair a W0 range.
   long long total = 0;
-  for (const auto& p : L.plans) total += p.units[0] + p.units[1] + p.units[2];
+  for (const auto& p : L.plans)
+    total += p.units[kPhaseGram] * p.gram_cost + p.units[kPhaseW0] + p.units[kPhaseG];
   int pairs = static_cast<int>(std::min<long long>(
       std::max(1, workers), std::min<long long>(total_w, std::max(1ll, total / 12))));
   std::vector<int> wb;
   while (true) {
+    for (auto& p : L.plans) set_gram_split(p, 1);
     size_t budget = grouped ? kWaveBudgetBytes : SIZE_MAX;
     const long long min_w = 3ll * pairs;
     wb = plan_waves(L.plans, d_in, r, min_w, budget);
@@ -360,7 +491,7 @@ bool layout_group(const int64_t* d_out, const int64_t* d_in, const int64_t* r, i
       budget *= 2;
       wb = plan_waves(L.plans, d_in, r, min_w, budget);
     }
-    bool ok = true;
+    bool ok = static_cast<int>(wb.size()) - 1 <= kMaxWaves;
     NormSched& S = L.sched;
     S.waves = static_cast<int>(wb.size()) - 1;
     S.pairs = pairs;
@@ -371,38 +502,29 @@ bool layout_group(const int64_t* d_out, const int64_t* d_in, const int64_t* r, i
       wi.n[0] = wi.n[1] = wi.n[2] = 0;
       for (int i = wi.m0; i < wi.m1; ++i)
         for (int ph = 0; ph < 3; ++ph) wi.n[ph] += L.plans[i].units[ph];
-      if (wi.n[kPhaseW0] < pairs || !choose_gram_pairs(wi, pairs)) ok = false;
+      if (wi.n[kPhaseW0] < pairs || !plan_gram(wi, L.plans, pairs)) ok = false;
     }
     if (ok) break;
     if (pairs == 1) return false;
     pairs = std::max(1, pairs * 3 / 4);
   }
-  // Segment slots: the most segments any tile (W0 + G) or pseudo-tile has.
+  // Segment slots: the most segments any tile (W0 + G) has.
   const NormSched& S = L.sched;
   L.seg_slots = 1;
-  L.gram_slots = 1;
-  std::vector<long long> mb(3 * count);
   for (int w = 0; w < S.waves; ++w) {
     long long at[3] = {0, 0, 0};
     for (int i = S.w[w].m0; i < S.w[w].m1; ++i) {
       const ModulePlan& p = L.plans[i];
-      for (int ph = 0; ph < 3; ++ph) {
-        mb[3 * i + ph] = at[ph];
-        at[ph] += p.units[ph];
-      }
-      for (int t = 0; t < p.pg_tiles; ++t) {
-        const long long x0 = mb[3 * i] + static_cast<long long>(t) * p.kb_w;
-        L.gram_slots = std::max(L.gram_slots, sched_segments(S.w[w], S.pairs, kPhaseGram, x0,
-                                                             x0 + p.kb_w, -1, nullptr));
-      }
       for (int t = 0; t < p.tiles; ++t) {
-        const long long xw = mb[3 * i + 1] + static_cast<long long>(t) * p.kb_w;
-        const long long xg = mb[3 * i + 2] + static_cast<long long>(t) * 2 * p.kb_r;
+        const long long xw = at[kPhaseW0] + static_cast<long long>(t) * p.kb_w;
+        const long long gpt = p.units[kPhaseG] / p.tiles;  // G units per tile
+        const long long xg = at[kPhaseG] + static_cast<long long>(t) * gpt;
         L.seg_slots = std::max(
             L.seg_slots,
             sched_segments(S.w[w], S.pairs, kPhaseW0, xw, xw + p.kb_w, -1, nullptr) +
-                sched_segments(S.w[w], S.pairs, kPhaseG, xg, xg + 2 * p.kb_r, -1, nullptr));
+                sched_segments(S.w[w], S.pairs, kPhaseG, xg, xg + gpt, -1, nullptr));
       }
+      for (int ph = 0; ph < 3; ++ph) at[ph] += p.units[ph];
     }
   }
   const uint32_t stage_bytes = kTileABytes + L.b_region;
@@ -422,9 +544,8 @@ bool layout_group(const int64_t* d_out, const int64_t* d_in, const int64_t* r, i
   off += L.cnt_bytes;
   for (auto& p : L.plans) {
     p.off_g = off;
-    off += align_up(static_cast<size_t>(2) * p.n_pad * p.r8 * 2, 256);  // G'_hi^T, G'_lo^T
-    p.off_gp = off;
-    off += align_up(static_cast<size_t>(p.pg_tiles) * L.gram_slots * p.n_pad * kPairM * 4, 256);
+    off += align_up(static_cast<size_t>(2) * p.gkp * r[&p - L.plans.data()] * p.r8 * 2,
+                    256);  // S_hi, S_lo: gkp parts each
     p.off_np = off;
     off += align_up(static_cast<size_t>(p.tiles) * L.seg_slots * kPairM * 4, 256);
     p.off_tw = off;
@@ -489,10 +610,11 @@ bool fill_descriptor(const dora_norm_problem_t& pr, const GroupLayout& L, int i,
   const ModulePlan& p = L.plans[i];
   std::memset(&nd, 0, sizeof(nd));
   uint16_t* g_hi = reinterpret_cast<uint16_t*>(ws_base + p.off_g);
-  uint16_t* g_lo = g_hi + static_cast<size_t>(p.n_pad) * p.r8;
+  uint16_t* g_lo = g_hi + static_cast<size_t>(p.gkp) * pr.r * p.r8;
   bool ok = true;
   ok &= make_tmap_bf16(&nd.tm_w0, pr.W0, pr.d_out, pr.d_in, pr.d_in, kBlockK, kTileM);
   ok &= make_tmap_bf16(&nd.tm_arow, pr.A, pr.r, pr.d_in, pr.d_in, kBlockK, kTileM);
+  ok &= make_tmap_bf16(&nd.tm_agram, pr.A, pr.r, pr.d_in, pr.d_in, kBlockK, p.gn / 2);
   // The N-side slab half of a CTA in one 4-D box when the two chunks are
   // equal and cover r exactly (no dimension of the view then reaches past the
   // matrix); otherwise one 2-D box of h0 rows per chunk (rows past r read 0).
@@ -500,12 +622,12 @@ bool fill_descriptor(const dora_norm_problem_t& pr, const GroupLayout& L, int i,
   nd.slab4d = slab4d ? 1 : 0;
   if (slab4d) {
     ok &= make_tmap_bf16_pairslab(&nd.tm_a, pr.A, p.h0, pr.d_in, pr.d_in, kBlockK);
-    ok &= make_tmap_bf16_pairslab(&nd.tm_g, g_hi, p.h0, pr.r, p.r8, kBlockK);
-    ok &= make_tmap_bf16_pairslab(&nd.tm_glo, g_lo, p.h0, pr.r, p.r8, kBlockK);
+    ok &= make_tmap_bf16_pairslab_parts(&nd.tm_g, g_hi, p.h0, pr.r, p.r8, p.gkp, kBlockK);
+    ok &= make_tmap_bf16_pairslab_parts(&nd.tm_glo, g_lo, p.h0, pr.r, p.r8, p.gkp, kBlockK);
   } else {
     ok &= make_tmap_bf16(&nd.tm_a, pr.A, pr.r, pr.d_in, pr.d_in, kBlockK, p.h0);
-    ok &= make_tmap_bf16(&nd.tm_g, g_hi, pr.r, pr.r, p.r8, kBlockK, p.h0);
-    ok &= make_tmap_bf16(&nd.tm_glo, g_lo, pr.r, pr.r, p.r8, kBlockK, p.h0);
+    ok &= make_tmap_bf16_parts(&nd.tm_g, g_hi, pr.r, pr.r, p.r8, p.gkp, kBlockK, p.h0);
+    ok &= make_tmap_bf16_parts(&nd.tm_glo, g_lo, pr.r, pr.r, p.r8, p.gkp, kBlockK, p.h0);
   }
   ok &= make_tmap_bf16(&nd.tm_b, pr.B, pr.d_out, pr.r, pr.r, kBlockK, kTileM);
   int* cnt = reinterpret_cast<int*>(ws_base + L.table_bytes) + p.cnt_off;
@@ -513,10 +635,8 @@ bool fill_descriptor(const dora_norm_problem_t& pr, const GroupLayout& L, int i,
   nd.g_hi = g_hi;
   nd.g_lo = g_lo;
   nd.partial = reinterpret_cast<float*>(ws_base + p.off_np);
-  nd.gram_part = reinterpret_cast<float*>(ws_base + p.off_gp);
   nd.tile_cnt = cnt;
-  nd.gram_cnt = cnt + p.tiles * 8;
-  nd.g_ready = cnt + p.tiles * 8 + p.pg_tiles * 2;
+  nd.g_ready = cnt + p.tiles * 2;
   nd.tile_w = reinterpret_cast<int*>(ws_base + p.off_tw);
   nd.m = pr.m;
   nd.n_out = pr.n_out;
@@ -534,10 +654,18 @@ bool fill_descriptor(const dora_norm_problem_t& pr, const GroupLayout& L, int i,
   nd.tiles = p.tiles;
   nd.pg_tiles = p.pg_tiles;
   nd.seg_slots = L.seg_slots;
-  nd.gram_slots = L.gram_slots;
+  nd.nc = p.nc;
+  nd.gchunks = p.gchunks;
+  nd.gn = p.gn;
+  nd.gh = p.gn / 2;
+  nd.gj0 = p.gj0;
+  nd.gblocks = p.gblocks;
+  nd.gkp = p.gkp;
   nd.pair_tx = 2 * (kTileABytes + p.b_region);
+  nd.gram_tx = 2 * (kTileABytes + static_cast<uint32_t>(p.nc / 2) * 128u);  // gchunks x gh rows
   nd.idesc0 = idesc_bf16_f32(kPairM, p.n0);
   nd.idesc1 = p.n1 > 0 ? idesc_bf16_f32(kPairM, p.n1) : 0u;
+  nd.idesc_gram = idesc_bf16_f32(kPairM, p.gn);
   nd.two_s = 2.0f * pr.s;
   nd.half_s = 0.5f * pr.s;
   return ok;
@@ -642,7 +770,7 @@ namespace {
 template <typename E, int VEC>
 void launch_fwd(bool small, int64_t rows, int64_t d_out, const void* base, const void* lora,
                 const float* m, const float* n, float s, float eps, void* y, void* inner,
-                cudaStream_t cs) {
+                bool delta, cudaStream_t cs) {
   const StreamGrid g = stream_grid(rows, static_cast<int>(d_out / VEC), kFwdRowUnroll);
   const dim3 grid(g.gx, g.gy), block(g.bx, g.by);
   const E* b = static_cast<const E*>(base);
@@ -651,21 +779,21 @@ void launch_fwd(bool small, int64_t rows, int64_t d_out, const void* base, const
   E* io = static_cast<E*>(inner);
   const long long R = rows;
   const int D = static_cast<int>(d_out);
-  if (inner != nullptr) {
+  auto go = [&](auto out) {
+    constexpr int kOut = decltype(out)::value;
     if (small)
-      launch_pdl(compose_fwd_kernel<E, VEC, uint32_t, true>, grid, block, 0, cs, b, l, m, n, s,
+      launch_pdl(compose_fwd_kernel<E, VEC, uint32_t, kOut>, grid, block, 0, cs, b, l, m, n, s,
                  eps, R, D, yo, io);
     else
-      launch_pdl(compose_fwd_kernel<E, VEC, uint64_t, true>, grid, block, 0, cs, b, l, m, n, s,
+      launch_pdl(compose_fwd_kernel<E, VEC, uint64_t, kOut>, grid, block, 0, cs, b, l, m, n, s,
                  eps, R, D, yo, io);
-  } else {
-    if (small)
-      launch_pdl(compose_fwd_kernel<E, VEC, uint32_t, false>, grid, block, 0, cs, b, l, m, n, s,
-                 eps, R, D, yo, io);
-    else
-      launch_pdl(compose_fwd_kernel<E, VEC, uint64_t, false>, grid, block, 0, cs, b, l, m, n, s,
-                 eps, R, D, yo, io);
-  }
+  };
+  if (delta)
+    go(std::integral_constant<int, kFwdDelta>());
+  else if (inner != nullptr)
+    go(std::integral_constant<int, kFwdYInner>());
+  else
+    go(std::integral_constant<int, kFwdY>());
 }
 
 template <typename E, int VEC, int kMode>
@@ -850,7 +978,8 @@ namespace {
 // Forward with an optional second output.  Validation, then one launch.
 dora_status_t compose_fwd_impl(const void* base, const void* lora, const float* m, const float* n,
                                float s, float eps, dora_dtype_t dt, int64_t T, int64_t d_out,
-                               void* y, void* inner, bool want_inner, dora_stream_t stream) {
+                               void* y, void* inner, bool want_inner, dora_stream_t stream,
+                               bool delta = false) {
   if (dt != DORA_F32 && dt != DORA_BF16) return DORA_ERR_INVALID_ARG;
   if (T < 0 || d_out < 1) return DORA_ERR_INVALID_ARG;
   if (m == nullptr || n == nullptr) return DORA_ERR_INVALID_ARG;
@@ -881,14 +1010,14 @@ dora_status_t compose_fwd_impl(const void* base, const void* lora, const float* 
   if (dt == DORA_BF16) {
     using B16 = __nv_bfloat16;
     if (al && d_out % 8 == 0)
-      launch_fwd<B16, 8>(small, T, d_out, base, lora, m, n, s, eps, y, in_out, cs);
+      launch_fwd<B16, 8>(small, T, d_out, base, lora, m, n, s, eps, y, in_out, delta, cs);
     else
-      launch_fwd<B16, 1>(small, T, d_out, base, lora, m, n, s, eps, y, in_out, cs);
+      launch_fwd<B16, 1>(small, T, d_out, base, lora, m, n, s, eps, y, in_out, delta, cs);
   } else {
     if (al && d_out % 4 == 0)
-      launch_fwd<float, 4>(small, T, d_out, base, lora, m, n, s, eps, y, in_out, cs);
+      launch_fwd<float, 4>(small, T, d_out, base, lora, m, n, s, eps, y, in_out, delta, cs);
     else
-      launch_fwd<float, 1>(small, T, d_out, base, lora, m, n, s, eps, y, in_out, cs);
+      launch_fwd<float, 1>(small, T, d_out, base, lora, m, n, s, eps, y, in_out, delta, cs);
   }
   return launch_status();
 }
@@ -973,6 +1102,14 @@ dora_status_t dora_compose_fwd(const void* base, const void* lora, const float* 
                                float s, float eps, dora_dtype_t dt, int64_t T, int64_t d_out,
                                void* y, dora_stream_t stream) {
   return compose_fwd_impl(base, lora, m, n, s, eps, dt, T, d_out, y, nullptr, false, stream);
+}
+
+dora_status_t dora_compose_fwd_delta(const void* base, const void* lora, const float* m,
+                                     const float* n, float s, float eps, dora_dtype_t dt,
+                                     int64_t T, int64_t d_out, void* dy_out,
+                                     dora_stream_t stream) {
+  return compose_fwd_impl(base, lora, m, n, s, eps, dt, T, d_out, dy_out, nullptr, false, stream,
+                          true);
 }
 
 dora_status_t dora_compose_fwd_train(const void* base, const void* lora, const float* m,

@@ -98,10 +98,6 @@ __device__ __forceinline__ void bulk_wait_group_read0() {
 __device__ __forceinline__ void bulk_wait_group0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
-// Makes this thread's generic-proxy shared-memory writes visible to TMA.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 // At[j][k] = A[k][j]: 32 x 32 tiles through shared memory, block (32, 8).
 __global__ void __launch_bounds__(256)

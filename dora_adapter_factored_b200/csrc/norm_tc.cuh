@@ -7,32 +7,37 @@
 // One persistent kernel on CTA pairs (after a tiny kernel that zeroes its
 // counters) does the whole norm of one module, or of many (the grouped call):
 //
-//   Gram units   G = A A^T in pseudo-tiles of 256 rows of A: the A operand is
-//                256 rows of A, the N-side operand the whole of A, k-blocks
-//                over d_in.  A few pairs take these first; each posts its
-//                fp32 partial, and once all of a pseudo-tile's partials are
-//                posted, the pairs that posted them each sum a share of its
-//                rows in a fixed order, scale by s/2 and write G' = (s/2) G
-//                as two bf16 matrices, G'_hi = bf16(G') and
-//                G'_lo = bf16(G' - G'_hi), so that the Gram term keeps
-//                fp32-level accuracy (the pages' norm accumulates in fp32
-//                whatever the weight dtype).  They store them transposed,
-//                which the quadratic form B_i G' B_i^T does not see.
+//   Gram jobs    one block of G = A A^T each: 256 rows of A (a pseudo-tile)
+//                against nc (<= 256) rows of A, over one of the gkp equal
+//                parts of d_in.  A few pairs take one job each first; the
+//                job scales its sum by s/2 and writes it as part p of S, in
+//                two bf16 matrices S_hi = bf16(S_p) and S_lo = bf16(S_p -
+//                S_hi), so that the Gram term keeps fp32-level accuracy (the
+//                pages' norm accumulates in fp32 whatever the weight dtype).
+//                Since G is symmetric, only one triangle is computed and
+//                stored: S_p = G'_p on the diagonal, 2 G'_p below it and 0
+//                above it (row gr, column c: c < gr), for which
+//                B_i (sum_p S_p) B_i^T = B_i G' B_i^T, G' = (s/2) G.  The parts
+//                are never added up: the G units sum them in their
+//                accumulator, so no job waits for another.
 //   W0 units     per 256-row tile of W0, k-blocks over d_in: TMEM
 //                accumulator += W0_tile A^T, while the reduction warps square
 //                and sum the same W0 tile straight from shared memory
 //                (||W0_i||^2), so W0 crosses HBM exactly once.
-//   G units      per tile, k-blocks over r: accumulator += B_tile G'_hi, then
-//                B_tile G'_lo; they wait until the module's G' is written.
+//   G units      per tile, k-blocks over r, for every part p:
+//                accumulator += B_tile S_hi,p^T, then B_tile S_lo,p^T; they wait
+//                until every part of the module's S is written.
 //
 // A segment (one pair's run of units on one tile) ends with an epilogue that
-// drains TMEM, dots each row with B_i and posts the per-row partial
-// ||W0_i||^2_part + 2 s B_i.acc_i: every term is linear in a k-range, so the
+// drains TMEM and dots each row with B_i; the per-row value
+// ||W0_i||^2_part + 2 s B_i.acc_i is handed to a finisher warp, which posts it
+// as the segment's partial: every term is linear in a k-range, so the
 // partials of all segments of a tile simply add (B_i.acc_i over G units is
-// (s/2) B_i G B_i^T).  The segment that posts a tile's partials last (an
-// arrival counter per 32 rows) sums them in slot order and finalises those
-// rows: n_i = sqrt(max(sum, 0)) and g_i = m_i / max(n_i, eps) (section 4,
-// precision bullet).
+// (s/2) B_i G B_i^T).  The finisher of the segment that posts a tile's
+// partials last (an arrival counter per CTA half of the tile) sums them in
+// slot order and finalises those rows: n_i = sqrt(max(sum, 0)) and
+// g_i = m_i / max(n_i, eps) (section 4, precision bullet).  Global round
+// trips thus never hold up the warps that release pipeline stages.
 #pragma once
 
 #include "common.cuh"
@@ -45,11 +50,16 @@ constexpr int kPairM = 2 * kTileM;           // W0 rows per tile of a CTA pair
 constexpr int kBlockK = 64;                  // bf16 of K per stage: one 128-byte swizzle row
 constexpr int kMaxStages = 8;
 constexpr int kEpiWarps = 8;                 // warps 0-7: reduction + epilogue
-constexpr int kNormThreads = (kEpiWarps + 2) * 32;  // + warp 8 TMA, warp 9 MMA
+constexpr int kProducerWarp = kEpiWarps;     // warp 8: TMA producer
+constexpr int kMmaWarp = kEpiWarps + 1;      // warps 9, 10: MMA issuers, one per accumulator chunk
+constexpr int kFinisherWarp = kEpiWarps + 3; // warp 11: posts partials, finalises rows
+constexpr int kNormThreads = (kEpiWarps + 4) * 32;
 constexpr int kMaxChunksPerHalf = 8;         // 32-column TMEM chunks per epilogue half (r <= 512)
 constexpr int kPrefetchChunks = 6;           // of which B is prefetched into registers (r <= 384)
-// Registers are granted to a block in groups of four warps, so the 10-warp
-// kernel is charged as 12 warps: 65536 / 384 threads = 170 -> 168.
+constexpr int kPartBufs = 4;                 // epilogue -> finisher hand-over buffers
+constexpr int kFinBatch = 8;                 // partial slots loaded together when finalising
+constexpr int kGramCols = 128;               // columns of G per Gram job (at most)
+// 12 warps: 65536 / 384 threads = 170 -> 168 registers per thread.
 constexpr int kNormMaxRegs = 168;
 
 constexpr uint32_t kTileABytes = kTileM * kBlockK * 2;  // 16 KiB
@@ -64,61 +74,77 @@ enum NormPhase : int { kPhaseGram = 0, kPhaseW0 = 1, kPhaseG = 2 };
 // ---------------------------------------------------------------------------
 struct alignas(64) NormProblemDev {
   CUtensorMap tm_w0;     // W0 [d_out, d_in], box 64 x 128
-  CUtensorMap tm_arow;   // A  [r, d_in],     box 64 x 128: the Gram units' A operand
+  CUtensorMap tm_arow;   // A  [r, d_in],     box 64 x 128: the Gram jobs' A operand
+  CUtensorMap tm_agram;  // A  [r, d_in],     box 64 x gh: the Gram jobs' N-side slab
   CUtensorMap tm_a;      // A  as the N-side slab: box 64 x h0, or the 4-D view
                          //    {64, h0, 2 ranks, 2 chunks} with box {64, h0, 1, 2}
   CUtensorMap tm_b;      // B  [d_out, r],    box 64 x 128
-  CUtensorMap tm_g;      // G'_hi (transposed) [r, r], like tm_a
-  CUtensorMap tm_glo;    // G'_lo (transposed) [r, r], like tm_a
+  CUtensorMap tm_g;      // S_hi [gkp][r][r8] as {r8, r, gkp} (or the 5-D pair view), box like tm_a
+  CUtensorMap tm_glo;    // S_lo, like tm_g
   const uint16_t* B;     // bf16 bits of B, for the epilogue dot
-  uint16_t* g_hi;        // [r][r8] bf16 bits of (G'_hi)^T
-  uint16_t* g_lo;        // [r][r8] bf16 bits of (G'_lo)^T
+  uint16_t* g_hi;        // [gkp][r][r8] bf16 bits of S_hi: S_p[gr][c] = 2 G'_p (c < gr), G'_p (c = gr), 0
+  uint16_t* g_lo;        // [gkp][r][r8] bf16 bits of S_lo = bf16(S_p - S_hi)
   float* partial;        // [tiles][seg_slots][256] per-row partials
-  float* gram_part;      // [pg_tiles][gram_slots][n_pad][256] fp32 Gram partials
-  int* tile_cnt;         // [tiles * 8] segments posted per 32-row quarter of each CTA's half
-  int* gram_cnt;         // [pg_tiles * 2] Gram segments posted per pseudo-tile half
-  int* g_ready;          // [1] rows of G' written (256 per pseudo-tile when complete)
+  int* tile_cnt;         // [tiles * 2] segments posted per CTA half of each tile
+  int* g_ready;          // [1] CTA halves of Gram jobs whose rows of S are written
   int* tile_w;           // [tiles] first pair | (pairs << 16) of each tile's W0 units
   const float* m;        // [d_out] or null
   float* n_out;          // [d_out]
   float* g_out;          // [d_out] or null
-  long long begin[3];    // first unit of this module in its wave's Gram / W0 / G sequence
+  long long begin[3];    // first job (Gram) / unit (W0, G) of this module in its wave
   int d_out, r, r8, n_pad;
   int n0, n1;            // N of the two pair-MMA chunks (n1 = 0: single chunk; else n1 = n0)
   int h0;                // slab rows of each chunk that one CTA stages: n0 / 2
   int slab4d;            // tm_a / tm_g / tm_glo are the 4-D view: one box per slab half
   int emit_sq;           // write the squared-norm sum itself to n_out (no clamp, sqrt or g)
-  int kb_w, kb_r, tiles, pg_tiles, seg_slots, gram_slots;
-  uint32_t pair_tx;      // bytes landing per stage in both CTAs together
-  uint32_t idesc0, idesc1;
+  int kb_w, kb_r, tiles, pg_tiles, seg_slots;
+  int nc;                // columns of G per Gram block: gchunks MMA chunks of gn
+  int gchunks, gn, gh;   // each CTA stages gh = gn / 2 slab rows per chunk
+  int gj0, gblocks;      // Gram blocks of pseudo-tile 0, of the module
+  int gkp;               // parts of d_in (one job per block and part)
+  uint32_t pair_tx;      // bytes landing per W0 / G stage in both CTAs together
+  uint32_t gram_tx;      // bytes landing per Gram stage in both CTAs together
+  uint32_t idesc0, idesc1, idesc_gram;
   float two_s, half_s;
 };
 
-// Units of phase `ph` per tile (per pseudo-tile for the Gram).
+// Units of phase `ph` per tile (per job for the Gram).
 __host__ __device__ __forceinline__ int phase_per_tile(const NormProblemDev& P, int ph) {
-  return ph == kPhaseG ? 2 * P.kb_r : P.kb_w;
+  return ph == kPhaseG ? 2 * P.kb_r * P.gkp : P.kb_w;
+}
+
+// Gram jobs of pseudo-tile t of a module of rank r (nc columns each): the
+// column blocks that reach the lower triangle, c <= row < min(r, 256 (t + 1)).
+__host__ __device__ __forceinline__ int gram_jobs_of_tile(int r, int nc, int t) {
+  const int rows_end = r < kPairM * (t + 1) ? r : kPairM * (t + 1);
+  return (rows_end + nc - 1) / nc;
 }
 
 // ---------------------------------------------------------------------------
 // Schedule.  The grouped call splits its modules (in order) into waves whose
-// re-read operands (A, G') fit in L2 together; one module alone is one wave.
+// re-read operands (A, S) fit in L2 together; one module alone is one wave.
 // Within a wave every pair j takes, in this order, a contiguous range of the
-// wave's Gram units, of its W0 units and of its G units:
-//   Gram: pairs j < J share the n[0] Gram units evenly (the others have none),
+// wave's Gram jobs, of its W0 units and of its G units:
+//   Gram: pairs j < J share the n[0] jobs evenly by count (the others have
+//         none); a job is never split,
 //   G:    every pair gets an even share of the n[2] G units,
-//   W0:   the rest of an even share of all units, where the Gram units count
-//         as gw >= n[0] (the Gram pairs also post and reduce partials),
+//   W0:   the rest of an even share of all work, where a Gram job counts as
+//         its cost in W0 units (the jobs of a wave form runs of equal cost),
 // so every pair has about the same work, the Gram is done early by a few
-// pairs, and the G units (which need G') come last in every pair.  The
+// pairs, and the G units (which need S) come last in every pair.  The
 // boundaries are closed forms of j; the host checks that every pair's W0
 // range is non-empty and the ranges are ordered.
 // ---------------------------------------------------------------------------
 constexpr int kMaxWaves = 64;
+constexpr int kMaxGramRuns = 8;
 struct WaveInfo {
-  long long n[3];  // units of the wave in the Gram, W0 and G sequences
-  long long gw;    // what the Gram units weigh in the W0 split (>= n[0])
-  int J;           // pairs that share the Gram units
+  long long n[3];  // Gram jobs, W0 units and G units of the wave
+  long long gw;    // cost of all the wave's Gram jobs, in W0 units
+  int J;           // pairs that share the Gram jobs
   int m0, m1;      // modules [m0, m1) of the table
+  int runs;                      // runs of consecutive jobs of equal cost
+  int run_end[kMaxGramRuns];     // first job after each run
+  int run_cost[kMaxGramRuns];    // cost of one job of the run, in W0 units
 };
 struct NormSched {
   int waves;
@@ -126,16 +152,28 @@ struct NormSched {
   WaveInfo w[kMaxWaves];
 };
 
-// First unit of pair j's range of phase `ph` (j = pairs gives the total).
+// Cost, in W0 units, of the wave's first x Gram jobs.
+__host__ __device__ __forceinline__ long long gram_cost_prefix(const WaveInfo& w, long long x) {
+  long long c = 0, start = 0;
+  for (int i = 0; i < w.runs && start < x; ++i) {
+    const long long e = w.run_end[i];
+    c += ((x < e ? x : e) - start) * w.run_cost[i];
+    start = e;
+  }
+  return c;
+}
+
+// First unit (Gram: job) of pair j's range of phase `ph` (j = pairs gives
+// the total).
 __host__ __device__ __forceinline__ long long sched_begin(const WaveInfo& w, int pairs, int ph,
                                                           int j) {
   const long long jj = j;
   const long long jg = jj < w.J ? jj : w.J;
-  if (ph == kPhaseGram) return w.J > 0 ? jg * w.n[0] / w.J : 0;
+  const long long gj = w.J > 0 ? jg * w.n[0] / w.J : 0;
+  if (ph == kPhaseGram) return gj;
   const long long gp = jj * w.n[2] / pairs;
   if (ph == kPhaseG) return gp;
-  const long long gram_w = w.J > 0 ? jg * w.gw / w.J : 0;
-  return jj * (w.gw + w.n[1] + w.n[2]) / pairs - gram_w - gp;
+  return jj * (w.gw + w.n[1] + w.n[2]) / pairs - gram_cost_prefix(w, gj) - gp;
 }
 
 // The pair whose range of phase `ph` holds unit x (the last j with
@@ -174,8 +212,8 @@ __host__ __device__ __forceinline__ int even_segments(long long x0, long long x1
   return static_cast<int>(x1 - x0);
 }
 
-// The segments of units [x0, x1) of phase `ph`, in order: returns how many
-// there are and sets *ord to the position of pair `me`'s segment.
+// The segments of units [x0, x1) of phase `ph` (W0 or G), in order: returns
+// how many there are and sets *ord to the position of pair `me`'s segment.
 __host__ __device__ __forceinline__ int sched_segments(const WaveInfo& w, int pairs, int ph,
                                                        long long x0, long long x1, int me,
                                                        int* ord) {
@@ -190,7 +228,6 @@ __host__ __device__ __forceinline__ int sched_segments(const WaveInfo& w, int pa
   }
   return nseg;
 }
-
 __device__ __forceinline__ float sumsq_bf16x8(uint4 v) {
   float a = 0.f, b = 0.f;
   a = fmaf(bf16lo_to_f32(v.x), bf16lo_to_f32(v.x), a);
@@ -246,17 +283,20 @@ __device__ __forceinline__ void epi_bar_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
 }
 
+
 // Walks one pair's segments of one phase of one wave: its range [x, end) of
-// the wave's phase sequence, module by module, tile by tile.
+// the wave's phase sequence, module by module, tile by tile (Gram: job by
+// job).
 template <bool kGrouped>
 struct SegWalk {
   const NormProblemDev* single;
   const NormProblemDev* table;
   int m, m1, ph;
   long long x, end;
-  // current segment: tile (pseudo-tile for the Gram), first unit in the tile, units
+  // current segment: tile (pseudo-tile for the Gram), Gram block, its
+  // column block and K part, first unit in the tile, units
   const NormProblemDev* P;
-  int tile, k0, n;
+  int tile, blk, cb, kpart, k0, n;
   long long xs;  // the segment's first unit in the wave's phase sequence
 
   __device__ __forceinline__ void start(const WaveInfo& w, int pairs, int pair, int phase) {
@@ -275,13 +315,26 @@ struct SegWalk {
     } else {
       P = single;
     }
-    const int per = phase_per_tile(*P, ph);
     const long long local = x - P->begin[ph];
+    xs = x;
+    if (ph == kPhaseGram) {
+      const int q = static_cast<int>(local);
+      const int kp = P->gkp;
+      blk = q / kp;
+      kpart = q - blk * kp;
+      tile = blk < P->gj0 ? 0 : 1;
+      cb = blk - (tile ? P->gj0 : 0);
+      k0 = kpart * P->kb_w / kp;
+      n = (kpart + 1) * P->kb_w / kp - k0;
+      x += 1;
+      return true;
+    }
+    const int per = phase_per_tile(*P, ph);
     tile = static_cast<int>(local / per);
+    cb = 0;
     k0 = static_cast<int>(local % per);
     const long long left = end - x;
     n = static_cast<int>(left < per - k0 ? left : per - k0);
-    xs = x;
     x += n;
     return true;
   }
@@ -301,12 +354,14 @@ struct SegWalk {
 // Barriers (per CTA, same offsets in both):
 //   full[s]      rank 0 only: its producer's expected bytes plus the copies of
 //                both CTAs (the peer's copies signal rank 0's barrier).
-//   mma_done[s]  both: rank 0's commit after the MMAs reading stage s, sent to
-//                both CTAs; the reduction warps then read the W0 rows
+//   mma_done[s]  both: rank 0's commits after the MMAs reading stage s, sent
+//                to both CTAs; the reduction warps then read the W0 rows
 //                (||W0_i||^2) and release the stage.
 //   empty[s]     both: one arrival per reduction warp; the producer refills.
-//   acc_full     both: rank 0's commit at the end of a segment.
+//   acc_full     both: rank 0's commits at the end of a segment.
 //   acc_empty    rank 0 only: one arrival per epilogue warp of both CTAs.
+//   part_full[b] both: the epilogue threads have written hand-over buffer b.
+//   part_empty[b] both: the finisher has read it.
 // ---------------------------------------------------------------------------
 struct NormSmemTail {
   uint64_t full[kMaxStages];
@@ -314,12 +369,13 @@ struct NormSmemTail {
   uint64_t empty[kMaxStages];
   uint64_t acc_full;
   uint64_t acc_empty;
-  uint64_t drain;
-  uint64_t half_ready;         // upper epilogue half has posted its partial
-  float half_part[2][kTileM];  // double-buffered by segment parity
+  uint64_t drain[2];                   // one per MMA issuer
+  uint64_t part_full[kPartBufs];
+  uint64_t part_empty[kPartBufs];
+  float part[kPartBufs][2][kTileM];    // per buffer: the lower and upper half's value per row
+  uint4 xpose[kEpiWarps][32 * 4];      // per epilogue warp: 32 rows x 32 bf16, swizzled
   uint32_t tmem_slot;
   int abort_flag;
-  int gram_ok;                 // every Gram segment of the pseudo-tile has posted
 };
 
 // Sets this CTA's and the peer's abort flags and records the timeout.
@@ -340,9 +396,9 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
   // exit global time, MMA-issuer cycles waiting for data / for the
   // accumulator, issued k-blocks, segments, SM id, cycles waited for data
   // over the first four k-blocks; then global times: the MMA issuer starting
-  // its W0 and its G units, and (first Gram segment) the epilogue holding the
-  // accumulator, its partial posted, all partials posted, its rows of G'
-  // written.
+  // its W0 and its G units, the epilogue holding its first Gram job's
+  // accumulator and having written that block of S, and the finisher done
+  // with its last segment.
   const uint64_t t_entry = trace != nullptr ? global_timer_ns() : 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -363,13 +419,17 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&mma_done[s], 1);
+      mbar_init(&mma_done[s], 2);  // both issuers' commits
       mbar_init(&empty[s], kEpiWarps);
     }
-    mbar_init(&tail->acc_full, 1);
+    mbar_init(&tail->acc_full, 2);
     mbar_init(&tail->acc_empty, 2 * kEpiWarps);
-    mbar_init(&tail->drain, 1);
-    mbar_init(&tail->half_ready, kTileM);
+    mbar_init(&tail->drain[0], 1);
+    mbar_init(&tail->drain[1], 1);
+    for (int b = 0; b < kPartBufs; ++b) {
+      mbar_init(&tail->part_full[b], kEpiWarps * 32);
+      mbar_init(&tail->part_empty[b], 1);
+    }
     tail->abort_flag = 0;
     fence_mbar_init();
   }
@@ -377,9 +437,10 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
     tmem_alloc_pair(&tail->tmem_slot, tmem_cols);
     tmem_relinquish_pair();
   }
-  if (!kGrouped && warp == kEpiWarps && lane == 0) {
+  if (!kGrouped && warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&single.tm_w0);
     prefetch_tmap(&single.tm_arow);
+    prefetch_tmap(&single.tm_agram);
     prefetch_tmap(&single.tm_a);
     prefetch_tmap(&single.tm_b);
     prefetch_tmap(&single.tm_g);
@@ -396,7 +457,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
   sw.single = &single;
   sw.table = table;
 
-  if (warp == kEpiWarps) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint64_t pol_stream = policy_evict_first();
@@ -406,7 +467,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
       uint32_t phase = 0;
       long long issued = 0;
       bool dep_waited = false;
-      const NormProblemDev* ready = nullptr;  // module whose G' is known to be written
+      const NormProblemDev* ready = nullptr;  // module whose S is known to be written
       bool ok = true;
       for (int wv = 0; ok && wv < sched.waves; ++wv) {
         for (int ph = kPhaseGram; ok && ph <= kPhaseG; ++ph) {
@@ -414,14 +475,16 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
           while (ok && sw.next()) {
             const NormProblemDev* P = sw.P;
             if (ph == kPhaseG && P != ready) {
-              // G' of this module is written by the pairs that reduce its
-              // Gram; the count they raise was zeroed by the preceding kernel.
+              // S of this module is written by the pairs that run its Gram
+              // jobs (each CTA of a pair counts its half of each job); the
+              // count they raise was zeroed by the preceding kernel.
               if (!dep_waited) {
                 grid_dependency_wait();
                 grid_dependency_trigger();
                 dep_waited = true;
               }
-              if (!wait_counter_geq(P->g_ready, kPairM * P->pg_tiles, timeout_ns, abort_flag)) {
+              if (!wait_counter_geq(P->g_ready, 2 * P->gblocks * P->gkp, timeout_ns,
+                                    abort_flag)) {
                 give_up_pair(abort_flag, peer_abort);
                 ok = false;
                 break;
@@ -439,29 +502,45 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
               uint8_t* sa = smem + stage * stage_bytes;
               uint8_t* sb = sa + kTileABytes;
               const uint32_t bar = full0 + stage * static_cast<uint32_t>(sizeof(uint64_t));
-              if (rank == 0) mbar_arrive_expect_tx(&full[stage], P->pair_tx);
-              const CUtensorMap* slab;
-              int kx;
-              if (ph == kPhaseG) {
-                const bool lo = k >= P->kb_r;
-                kx = (k - (lo ? P->kb_r : 0)) * kBlockK;
-                tma_load_2d_pair(sa, &P->tm_b, bar, kx, row0, pol_keep);
-                slab = lo ? &P->tm_glo : &P->tm_g;
+              if (ph == kPhaseGram) {
+                if (rank == 0) mbar_arrive_expect_tx(&full[stage], P->gram_tx);
+                const int kx = k * kBlockK;
+                tma_load_2d_pair(sa, &P->tm_arow, bar, kx, row0, pol_keep);
+                for (int q = 0; q < P->gchunks; ++q)
+                  tma_load_2d_pair(sb + q * P->gh * 128, &P->tm_agram, bar, kx,
+                                   sw.cb * P->nc + q * P->gn + static_cast<int>(rank) * P->gh,
+                                   pol_keep);
               } else {
-                kx = k * kBlockK;
-                if (ph == kPhaseW0)
+                if (rank == 0) mbar_arrive_expect_tx(&full[stage], P->pair_tx);
+                const int rk = static_cast<int>(rank);
+                if (ph == kPhaseG) {
+                  // unit k: part p, then S_hi or S_lo, then the k-block of r
+                  const int p = k / (2 * P->kb_r);
+                  const int kk = k - p * 2 * P->kb_r;
+                  const bool lo = kk >= P->kb_r;
+                  const int kx = (kk - (lo ? P->kb_r : 0)) * kBlockK;
+                  tma_load_2d_pair(sa, &P->tm_b, bar, kx, row0, pol_keep);
+                  const CUtensorMap* slab = lo ? &P->tm_glo : &P->tm_g;
+                  if (P->slab4d) {
+                    tma_load_5d_pair(sb, slab, bar, kx, 0, rk, 0, p, pol_keep);
+                  } else {
+                    tma_load_3d_pair(sb, slab, bar, kx, rk * P->h0, p, pol_keep);
+                    if (P->n1 > 0)
+                      tma_load_3d_pair(sb + P->h0 * 128, slab, bar, kx, P->n0 + rk * P->h0, p,
+                                       pol_keep);
+                  }
+                } else {
+                  const int kx = k * kBlockK;
                   tma_load_2d_pair(sa, &P->tm_w0, bar, kx, row0, pol_stream);
-                else
-                  tma_load_2d_pair(sa, &P->tm_arow, bar, kx, row0, pol_keep);
-                slab = &P->tm_a;
-              }
-              if (P->slab4d) {
-                tma_load_4d_pair(sb, slab, bar, kx, 0, static_cast<int>(rank), 0, pol_keep);
-              } else {
-                tma_load_2d_pair(sb, slab, bar, kx, static_cast<int>(rank) * P->h0, pol_keep);
-                if (P->n1 > 0)
-                  tma_load_2d_pair(sb + P->h0 * 128, slab, bar, kx,
-                                   P->n0 + static_cast<int>(rank) * P->h0, pol_keep);
+                  if (P->slab4d) {
+                    tma_load_4d_pair(sb, &P->tm_a, bar, kx, 0, rk, 0, pol_keep);
+                  } else {
+                    tma_load_2d_pair(sb, &P->tm_a, bar, kx, rk * P->h0, pol_keep);
+                    if (P->n1 > 0)
+                      tma_load_2d_pair(sb + P->h0 * 128, &P->tm_a, bar, kx, P->n0 + rk * P->h0,
+                                       pol_keep);
+                  }
+                }
               }
               ++issued;
               if (++stage == stages) {
@@ -490,10 +569,15 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
           mbar_wait(&empty[j % stages], par, kDrainTimeoutNs, nullptr);
       }
     }
-  } else if (warp == kEpiWarps + 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+    // ------------------------------------------------------------ MMA issuers
+    // Issuer q drives accumulator chunk q: the two chains go to the tensor
+    // pipe from two threads, which halves the issue time per k-block.  Both
+    // commit after every stage and at the end of every segment (issuer 1
+    // without MMAs when there is a single chunk), so the barriers count two.
+    const int issuer = warp - kMmaWarp;
     if (lane == 0 && rank == 0) {
-      const bool tracing = trace != nullptr;
+      const bool tracing = trace != nullptr && issuer == 0;
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool issued_any = false;
@@ -515,9 +599,14 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
             if (tracing) wait_acc += clock64() - c0;
             ++nseg;
             tc_fence_after_sync();
-            const uint32_t idesc0 = P->idesc0, idesc1 = P->idesc1;
-            const int n0 = P->n0, n1 = P->n1;
-            const uint32_t b1_off = static_cast<uint32_t>(P->h0) * 128u;
+            // this issuer's chunk: accumulator columns, slab rows, shape
+            const bool gram = ph == kPhaseGram;
+            const bool active = issuer == 0 || (gram ? P->gchunks > 1 : P->n1 > 0);
+            const uint32_t d_col =
+                issuer == 0 ? 0u : static_cast<uint32_t>(gram ? P->gn : P->n0);
+            const uint32_t b_off =
+                issuer == 0 ? 0u : static_cast<uint32_t>(gram ? P->gh : P->h0) * 128u;
+            const uint32_t idesc = gram ? P->idesc_gram : (issuer == 0 ? P->idesc0 : P->idesc1);
             for (int i = 0; i < sw.n; ++i) {
               // The stage's copies completed on this barrier; the MMAs that
               // read it are issued straight after the wait.
@@ -532,24 +621,13 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
                 if (nkb < 4) wait_first = wait_data;
               }
               ++nkb;
-              const uint32_t a0 = smem_addr(smem + stage * stage_bytes);
-              const uint32_t b0 = a0 + kTileABytes;
-              // Two accumulator chains (chunks) when r > 256, interleaved per
-              // K step; the chunk test stays outside the issue loops.
-              if (n1 > 0) {
-#pragma unroll
-                for (int k = 0; k < kBlockK / 16; ++k) {
-                  const uint64_t ad = sw128_kmajor_desc(a0 + k * 32);
-                  const uint32_t acc = (i == 0 && k == 0) ? 0u : 1u;
-                  umma_bf16_pair(tmem_base, ad, sw128_kmajor_desc(b0 + k * 32), idesc0, acc);
-                  umma_bf16_pair(tmem_base + n0, ad, sw128_kmajor_desc(b0 + b1_off + k * 32),
-                                 idesc1, acc);
-                }
-              } else {
+              if (active) {
+                const uint32_t a0 = smem_addr(smem + stage * stage_bytes);
+                const uint32_t b0 = a0 + kTileABytes + b_off;
 #pragma unroll
                 for (int k = 0; k < kBlockK / 16; ++k)
-                  umma_bf16_pair(tmem_base, sw128_kmajor_desc(a0 + k * 32),
-                                 sw128_kmajor_desc(b0 + k * 32), idesc0,
+                  umma_bf16_pair(tmem_base + d_col, sw128_kmajor_desc(a0 + k * 32),
+                                 sw128_kmajor_desc(b0 + k * 32), idesc,
                                  (i == 0 && k == 0) ? 0u : 1u);
               }
               issued_any = true;
@@ -565,11 +643,12 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
           }
         }
       }
+      if (tracing) trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 15] = global_timer_ns();
       if (issued_any) {
-        umma_commit_pair(&tail->drain, 0x1);
-        mbar_wait(&tail->drain, 0, kDrainTimeoutNs, nullptr);
+        umma_commit_pair(&tail->drain[issuer], 0x1);
+        mbar_wait(&tail->drain[issuer], 0, kDrainTimeoutNs, nullptr);
       }
-      if (trace != nullptr) {
+      if (tracing) {
         unsigned long long* tr = trace + static_cast<size_t>(blockIdx.x) * kTraceWords;
         tr[2] = static_cast<unsigned long long>(wait_data);
         tr[3] = static_cast<unsigned long long>(wait_acc);
@@ -578,7 +657,127 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
         tr[7] = static_cast<unsigned long long>(wait_first);
       }
     }
-  } else {
+  } else if (warp == kFinisherWarp) {
+    // ------------------------------------------- partials and finalisation
+    // Gram jobs: once every epilogue thread has written its rows of S, make
+    // them visible and count this CTA's half of the job as written.
+    // W0 / G segments: lane l takes rows l, l + 32, l + 64, l + 96 of this
+    // CTA's half of the tile: it adds the two epilogue halves' values of each
+    // row (lower + upper), posts them as the segment's partial and, when this
+    // is the tile's last segment to post, sums every slot in slot order and
+    // writes n and g.
+    uint32_t seg_count = 0;
+    bool dep_waited = false;
+    bool gram_traced = false;
+    bool ok = true;
+    for (int wv = 0; ok && wv < sched.waves; ++wv) {
+      const WaveInfo& W = sched.w[wv];
+      for (int ph = kPhaseGram; ok && ph <= kPhaseG; ++ph) {
+        sw.start(W, pairs, pair, ph);
+        while (ok && sw.next()) {
+          const NormProblemDev* P = sw.P;
+          const int t = sw.tile;
+          const int buf = static_cast<int>(seg_count % kPartBufs);
+          const uint32_t par = (seg_count / kPartBufs) & 1u;
+          ++seg_count;
+          if (!mbar_wait(&tail->part_full[buf], par, timeout_ns, abort_flag)) {
+            give_up_pair(abort_flag, peer_abort);
+            ok = false;
+            break;
+          }
+          if (ph == kPhaseGram) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tail->part_empty[buf]);
+            if (!dep_waited) {  // the count was zeroed by the preceding kernel
+              grid_dependency_wait();
+              dep_waited = true;
+            }
+            if (lane == 0) {
+              __threadfence();
+              fence_proxy_async_global();
+              atomicAdd(P->g_ready, 1);
+              if (trace != nullptr && !gram_traced)
+                trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 11] = global_timer_ns();
+            }
+            gram_traced = true;
+            continue;
+          }
+          float v[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int row = lane + 32 * q;
+            v[q] = tail->part[buf][0][row] + tail->part[buf][1][row];
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tail->part_empty[buf]);
+          if (!dep_waited) {  // counters and the tile table come from the preceding kernel
+            grid_dependency_wait();
+            dep_waited = true;
+          }
+          // Where this segment's partial goes among the tile's segments: its
+          // W0 segments come from consecutive pairs (found by the preceding
+          // kernel), then the G segments, split evenly over all pairs.
+          const int g_per_tile = phase_per_tile(*P, kPhaseG);
+          const long long xg = P->begin[kPhaseG] + static_cast<long long>(t) * g_per_tile;
+          int ord = 0;
+          int nseg = even_segments(xg, xg + g_per_tile, sw.xs, W.n[kPhaseG], pairs, pair, &ord);
+          const int tw = __ldcg(P->tile_w + t);
+          const int nw = tw >> 16;
+          ord = ph == kPhaseW0 ? pair - (tw & 0xffff) : ord + nw;
+          nseg += nw;
+          const int row_base = t * kPairM + static_cast<int>(rank) * kTileM;
+          float* part_t = P->partial + static_cast<size_t>(t) * P->seg_slots * kPairM +
+                          static_cast<int>(rank) * kTileM;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (row_base + lane + 32 * q < P->d_out)
+              part_t[static_cast<size_t>(ord) * kPairM + lane + 32 * q] = v[q];
+          __threadfence();
+          __syncwarp();
+          int prev = 0;
+          if (lane == 0) prev = atomicAdd(P->tile_cnt + t * 2 + static_cast<int>(rank), 1);
+          prev = __shfl_sync(0xffffffffu, prev, 0);
+          if (prev == nseg - 1) {
+            __threadfence();
+            // All of a batch's loads (kFinBatch slots of the four rows) are in
+            // flight together; absent slots add zero, so the sum is the same
+            // fixed slot order whatever the batching.
+            float sum[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int c0 = 0; c0 < nseg; c0 += kFinBatch) {
+              float v[4][kFinBatch];
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int u = 0; u < kFinBatch; ++u)
+                  v[q][u] = c0 + u < nseg ? __ldcg(part_t + static_cast<size_t>(c0 + u) * kPairM +
+                                                   lane + 32 * q)
+                                          : 0.f;
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int u = 0; u < kFinBatch; ++u) sum[q] += v[q][u];
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int row = lane + 32 * q;
+              const int grow = row_base + row;
+              if (grow >= P->d_out) continue;
+              if (P->emit_sq) {
+                P->n_out[grow] = sum[q];
+              } else {
+                const float n = __fsqrt_rn(fmaxf(sum[q], 0.f));
+                P->n_out[grow] = n;
+                if (P->m != nullptr && P->g_out != nullptr)
+                  P->g_out[grow] = __fdiv_rn(__ldg(P->m + grow), fmaxf(n, eps));
+              }
+            }
+          }
+        }
+      }
+    }
+    if (trace != nullptr && lane == 0)
+      trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 12] = global_timer_ns();
+  } else if (warp < kEpiWarps) {
     // ------------------------------------ ||W0_i||^2 + epilogue (warps 0-7)
     // Thread (half h, row): TMEM lane `row`; half h of the row's 16-byte chunks
     // of each W0 stage and half h of the accumulator's 32-column chunks.
@@ -588,7 +787,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
     const uint32_t acc_empty0 = mapa_shared(smem_addr(&tail->acc_empty), 0);
     int stage = 0;
     uint32_t phase = 0, acc_phase = 0, seg_count = 0;
-    bool dep_waited = false;
+    bool gram_traced = false;
     bool ok = true;
     for (int wv = 0; ok && wv < sched.waves; ++wv) {
       const WaveInfo& W = sched.w[wv];
@@ -600,41 +799,25 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
           const int r = P->r;
           // the row of W0 (or, for the Gram, of A) this thread finishes
           const int grow = t * kPairM + static_cast<int>(rank) * kTileM + row;
-          const bool valid = grow < (ph == kPhaseGram ? r : P->d_out);
+          const bool gram = ph == kPhaseGram;
+          const bool valid = grow < (gram ? r : P->d_out);
           // this half's 32-column chunks of the accumulator
-          const int nchunks = (P->n0 + P->n1 + 31) / 32;
+          const int nchunks = gram ? (P->nc + 31) / 32 : (P->n0 + P->n1 + 31) / 32;
           const int c_lo = half == 0 ? 0 : (nchunks + 1) / 2;
           const int c_hi = half == 0 ? (nchunks + 1) / 2 : nchunks;
           // Prefetch B_i for (up to kPrefetchChunks of) those columns while
           // the MMAs of this segment run.
-          const bool dotted = ph != kPhaseGram;
-          const uint16_t* brow = P->B + static_cast<size_t>(dotted && valid ? grow : 0) * r;
+          const uint16_t* brow = P->B + static_cast<size_t>(!gram && valid ? grow : 0) * r;
           uint4 bq[kPrefetchChunks][4];
 #pragma unroll
           for (int c = 0; c < kPrefetchChunks; ++c)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const int col = (c_lo + c) * 32 + q * 8;
-              bq[c][q] = (dotted && valid && c_lo + c < c_hi && col < r)
+              bq[c][q] = (!gram && valid && c_lo + c < c_hi && col < r)
                              ? __ldg(reinterpret_cast<const uint4*>(brow + col))
                              : make_uint4(0u, 0u, 0u, 0u);
             }
-          // Where this segment's partial goes among the tile's segments
-          // (the Gram and G sequences are split evenly over their pairs; the
-          // W0 segments of each tile come from consecutive pairs, found by
-          // the preceding kernel).
-          int ord = 0, nseg = 0;
-          if (ph == kPhaseGram) {
-            const long long x0 = P->begin[kPhaseGram] + static_cast<long long>(t) * P->kb_w;
-            nseg = even_segments(x0, x0 + P->kb_w, sw.xs, W.n[kPhaseGram], W.J, pair, &ord);
-          } else {
-            const long long xg = P->begin[kPhaseG] + static_cast<long long>(t) * 2 * P->kb_r;
-            int ord_g = 0;
-            const int ng = even_segments(xg, xg + 2 * P->kb_r, sw.xs, W.n[kPhaseG], pairs, pair,
-                                         &ord_g);
-            nseg = ng;  // the W0 count and this pair's W0 slot follow once the table is visible
-            ord = ord_g;
-          }
           float ss = 0.f;
           for (int i = 0; i < sw.n; ++i) {
             // The MMAs that read this stage have completed, so its copies
@@ -668,117 +851,108 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
           }
           tc_fence_after_sync();
           acc_phase ^= 1u;
-          if (!dep_waited) {  // counters and the tile table come from the preceding kernel
-            grid_dependency_wait();
-            dep_waited = true;
-          }
-          if (ph != kPhaseGram) {
-            const int tw = __ldcg(P->tile_w + t);
-            const int nw = tw >> 16;
-            if (ph == kPhaseW0) {
-              ord = pair - (tw & 0xffff);
-              nseg += nw;
-            } else {
-              ord += nw;
-              nseg += nw;
-            }
-          }
 
-          const bool gtrace = trace != nullptr && threadIdx.x == 0 && ph == kPhaseGram &&
-                              trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 10] == 0;
-          if (gtrace) trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 10] = global_timer_ns();
-          if (ph == kPhaseGram) {
-            // ---- Gram segment: post the raw accumulator (this CTA's 128
-            // rows of G, all n_pad columns) as partial `ord`, column-major,
-            // so that each store of a warp covers 32 consecutive rows.
-            const int n_pad = P->n_pad;
-            const size_t slot = static_cast<size_t>(n_pad) * kPairM;
-            float* gbase = P->gram_part + static_cast<size_t>(t) * P->gram_slots * slot +
-                           static_cast<int>(rank) * kTileM;
-            float* gp = gbase + static_cast<size_t>(ord) * slot + row;
+          if (gram) {
+            // ---- Gram job: this CTA's 128 rows gr of the block of G
+            // (columns [cb nc, cb nc + nc)) over part kpart of d_in, scaled
+            // into S_kpart (row gr, column c): 2 G' for c < gr, G' for c = gr,
+            // 0 above.  A thread writes 8 consecutive columns of its row per
+            // 16-byte store.
+            const bool first = trace != nullptr && threadIdx.x == 0 && !gram_traced;
+            if (first) trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 10] = global_timer_ns();
+            const int col0 = sw.cb * P->nc;
+            const int col_end = min(r, col0 + P->nc);
+            const float hs = P->half_s;
+            // This warp's 32 rows of S_kpart (TMEM lanes (warp & 3) * 32 + i).
+            const int wrow0 = t * kPairM + static_cast<int>(rank) * kTileM + (warp & 3) * 32;
+            uint16_t* s_hi = P->g_hi + static_cast<size_t>(sw.kpart) * r * P->r8;
+            uint16_t* s_lo = P->g_lo + static_cast<size_t>(sw.kpart) * r * P->r8;
+            uint4* xp = tail->xpose[warp];
+            // Lane (i, piece): rows wrow0 + 8 j + lane / 4, 16-byte piece lane % 4
+            // of the 32 columns, after the transpose through shared memory
+            // (16-byte units swizzled by row, so that both sides are free of
+            // bank conflicts).
+            const int piece = lane & 3;
+            auto put_chunk = [&](int colc, const float (&acc)[32], bool lo_part) {
+              uint32_t w[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                float x[2];
+#pragma unroll
+                for (int f = 0; f < 2; ++f) {
+                  const int col = colc + 2 * e + f;
+                  const float g = acc[2 * e + f];
+                  x[f] = col < grow ? 2.f * hs * g : (col == grow ? hs * g : 0.f);
+                }
+                const uint16_t h0 = f32_to_bf16_rn(x[0]), h1 = f32_to_bf16_rn(x[1]);
+                uint16_t v0 = h0, v1 = h1;
+                if (lo_part) {
+                  v0 = f32_to_bf16_rn(x[0] - __uint_as_float(static_cast<uint32_t>(h0) << 16));
+                  v1 = f32_to_bf16_rn(x[1] - __uint_as_float(static_cast<uint32_t>(h1) << 16));
+                }
+                w[e] = static_cast<uint32_t>(v0) | (static_cast<uint32_t>(v1) << 16);
+              }
+              __syncwarp();
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                xp[lane * 4 + (j ^ ((lane >> 1) & 3))] =
+                    make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+              __syncwarp();
+              uint16_t* dst = lo_part ? s_lo : s_hi;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int rr = 8 * j + (lane >> 2);  // row within the warp's 32
+                const int col = colc + piece * 8;
+                const uint4 v = xp[rr * 4 + (piece ^ ((rr >> 1) & 3))];
+                if (wrow0 + rr < r && col < col_end)
+                  *reinterpret_cast<uint4*>(dst + static_cast<size_t>(wrow0 + rr) * P->r8 + col) = v;
+              }
+            };
 #pragma unroll 1
             for (int c = c_lo; c < c_hi; ++c) {
               float acc[32];
               tmem_load_32cols(tmem_base + lane_base + c * 32, acc);
-#pragma unroll
-              for (int q = 0; q < 32; ++q)
-                if (c * 32 + q < n_pad) __stcg(gp + static_cast<size_t>(c * 32 + q) * kPairM, acc[q]);
+              put_chunk(col0 + c * 32, acc, false);
+              put_chunk(col0 + c * 32, acc, true);
             }
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc_empty0);
-            // Once every segment of this pseudo-tile has posted (per CTA
-            // half: the segments end together, since the Gram pairs start
-            // at once), each sums a share of the rows over all partials in
-            // slot order and writes those rows of G'_hi and G'_lo.
-            __threadfence();
-            epi_bar_sync();
-            int* cnt = P->gram_cnt + t * 2 + static_cast<int>(rank);
-            if (threadIdx.x == 0) {
-              if (gtrace) trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 11] = global_timer_ns();
-              atomicAdd(cnt, 1);
-              tail->gram_ok = wait_counter_geq(cnt, nseg, timeout_ns, abort_flag) ? 1 : 0;
-              if (gtrace) trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 12] = global_timer_ns();
+            // The pseudo-tile's last block also zeroes the columns past it
+            // (all above the diagonal for these rows).
+            const int njt = gram_jobs_of_tile(r, P->nc, t);
+            if (sw.cb == njt - 1) {
+              // columns [z0, r) of the warp's 32 rows, 32 columns per step,
+              // split between the two halves
+              const int z0 = njt * P->nc;
+              const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+              for (int colc = z0 + half * 32; colc < r; colc += 64)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const int rr = 8 * j + (lane >> 2);
+                  const int col = colc + piece * 8;
+                  if (wrow0 + rr < r && col < r) {
+                    const size_t o = static_cast<size_t>(wrow0 + rr) * P->r8 + col;
+                    *reinterpret_cast<uint4*>(s_hi + o) = z;
+                    *reinterpret_cast<uint4*>(s_lo + o) = z;
+                  }
+                }
             }
-            epi_bar_sync();
-            if (!tail->gram_ok) {
+            // The finisher publishes these rows of S to the TMA reads of every
+            // pair's G units once all epilogue threads have handed over.
+            if (first) trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 13] = global_timer_ns();
+            fence_proxy_async_global();
+            if (first) trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 14] = global_timer_ns();
+            const int buf = static_cast<int>(seg_count % kPartBufs);
+            const uint32_t use = seg_count / kPartBufs;
+            ++seg_count;
+            if (!mbar_wait(&tail->part_empty[buf], (use & 1u) ^ 1u, timeout_ns, abort_flag)) {
               give_up_pair(abort_flag, peer_abort);
               ok = false;
               break;
             }
-            __threadfence();
-            // This segment's share: rows [rb, re) of the CTA half, every
-            // column.  Lanes take consecutive rows (32 at a time) and warps
-            // interleaved columns, so every load and store of a warp covers
-            // consecutive addresses; kU columns of every partial are in
-            // flight per thread.
-            const int rb = ord * kTileM / nseg, re = (ord + 1) * kTileM / nseg;
-            constexpr int kU = 12;
-            constexpr int kCs = kEpiWarps;  // column stride between a warp's columns
-#pragma unroll 1
-            for (int r0 = rb; r0 < re; r0 += 32) {
-              const int rr = r0 + lane;
-              const bool rv = rr < re;
-              const int gr = t * kPairM + static_cast<int>(rank) * kTileM + rr;
-              const float* src = gbase + rr;
-#pragma unroll 1
-              for (int c0 = warp; c0 < n_pad; c0 += kCs * kU) {
-                float sum[kU];
-#pragma unroll
-                for (int u = 0; u < kU; ++u) sum[u] = 0.f;
-#pragma unroll 1
-                for (int o = 0; o < nseg; ++o) {
-                  const float* so = src + static_cast<size_t>(o) * slot;
-                  float v[kU];
-#pragma unroll
-                  for (int u = 0; u < kU; ++u) {
-                    const int c = c0 + u * kCs;
-                    v[u] = (rv && c < n_pad) ? __ldcg(so + static_cast<size_t>(c) * kPairM) : 0.f;
-                  }
-#pragma unroll
-                  for (int u = 0; u < kU; ++u) sum[u] += v[u];
-                }
-                if (rv && gr < r) {
-#pragma unroll
-                  for (int u = 0; u < kU; ++u) {
-                    const int c = c0 + u * kCs;
-                    if (c >= r) break;
-                    const float x = P->half_s * sum[u];
-                    const uint16_t hi = f32_to_bf16_rn(x);
-                    const uint16_t lo =
-                        f32_to_bf16_rn(x - __uint_as_float(static_cast<uint32_t>(hi) << 16));
-                    P->g_hi[static_cast<size_t>(c) * P->r8 + gr] = hi;
-                    P->g_lo[static_cast<size_t>(c) * P->r8 + gr] = lo;
-                  }
-                }
-              }
-            }
-            // Publish these rows of G' to the TMA reads of every pair's G units.
-            __threadfence();
-            fence_proxy_async_global();
-            epi_bar_sync();
-            if (threadIdx.x == 0) atomicAdd(P->g_ready, re - rb);
-            if (gtrace) trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 13] = global_timer_ns();
+            mbar_arrive(&tail->part_full[buf]);
+            if (first) gram_traced = true;
             continue;
           }
 
@@ -805,57 +979,19 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
             }
           }
           tc_fence_before_sync();
-          // Combine the two halves of the row in a fixed order (lower +
-          // upper).  The lower half takes the upper half's value before it
-          // releases the accumulator, so the next segment cannot overwrite it
-          // early.
-          const float part = fmaf(P->two_s, dot, ss);
-          const int buf = seg_count & 1;
-          if (half == 1) {
-            tail->half_part[buf][row] = part;
-            mbar_arrive(&tail->half_ready);
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc_empty0);
-          } else {
-            const bool got_one =
-                mbar_wait(&tail->half_ready, seg_count & 1u, timeout_ns, abort_flag);
-            const float other = tail->half_part[buf][row];
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc_empty0);
-            if (!__all_sync(0xffffffffu, got_one)) {
-              give_up_pair(abort_flag, peer_abort);
-              ok = false;
-              break;
-            }
-            float* part_t = P->partial + static_cast<size_t>(t) * P->seg_slots * kPairM +
-                            static_cast<int>(rank) * kTileM + row;
-            if (valid) part_t[static_cast<size_t>(ord) * kPairM] = part + other;
-            // The last of the tile's segments to post its partials (per warp:
-            // 32 rows) sums every slot in slot order and writes n and g.
-            __threadfence();
-            __syncwarp();
-            int prev = 0;
-            if (lane == 0)
-              prev = atomicAdd(P->tile_cnt + (t * 2 + static_cast<int>(rank)) * 4 + warp, 1);
-            prev = __shfl_sync(0xffffffffu, prev, 0);
-            if (prev == nseg - 1) {
-              __threadfence();
-              if (valid) {
-                float sum = 0.f;
-                for (int c = 0; c < nseg; ++c)
-                  sum += __ldcg(part_t + static_cast<size_t>(c) * kPairM);
-                if (P->emit_sq) {
-                  P->n_out[grow] = sum;
-                } else {
-                  const float n = __fsqrt_rn(fmaxf(sum, 0.f));
-                  P->n_out[grow] = n;
-                  if (P->m != nullptr && P->g_out != nullptr)
-                    P->g_out[grow] = __fdiv_rn(__ldg(P->m + grow), fmaxf(n, eps));
-                }
-              }
-            }
-          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(acc_empty0);
+          // Hand this half's value of the row to the finisher warp.
+          const int buf = static_cast<int>(seg_count % kPartBufs);
+          const uint32_t use = seg_count / kPartBufs;
           ++seg_count;
+          if (!mbar_wait(&tail->part_empty[buf], (use & 1u) ^ 1u, timeout_ns, abort_flag)) {
+            give_up_pair(abort_flag, peer_abort);
+            ok = false;
+            break;
+          }
+          tail->part[buf][half][row] = fmaf(P->two_s, dot, ss);
+          mbar_arrive(&tail->part_full[buf]);
         }
       }
     }

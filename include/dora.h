@@ -159,6 +159,23 @@ dora_status_t dora_compose_fwd(const void *base, const void *lora, const float *
                                dora_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Compose forward, delta form  ["Scaling DoRA ...", Data Availability: the
+ * module's output is dY = g (s x A^T B^T) + (g - 1) Y_base, which the caller
+ * adds to its own Y_base]
+ *
+ *   dy_out[t, j] = (g_j - 1) base[t, j] + (g_j s) lora[t, j]
+ * with g and g - 1 formed as for dora_compose_fwd, evaluated in fp32 and
+ * rounded once to `dt`; y of dora_compose_fwd is base + dy_out before that
+ * rounding.  base, lora, dy_out: [T, d_out] in dtype `dt`; dy_out may equal
+ * base (same element, same thread), no other overlap.  One pass: two reads
+ * and one write per element.  T == 0 launches nothing.
+ * ---------------------------------------------------------------------- */
+dora_status_t dora_compose_fwd_delta(const void *base, const void *lora, const float *m,
+                                     const float *n, float s, float eps, dora_dtype_t dt,
+                                     int64_t T, int64_t d_out, void *dy_out,
+                                     dora_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Fused compose backward  ["Scaling DoRA ...", section 3 backward kernel]
  *
  *   d_base[t, j] = g_j dy[t, j],  d_lora[t, j] = (g_j s) dy[t, j]
@@ -364,8 +381,8 @@ void dora_set_timing_events(void *before, void *after);
  * operands and [3] for the accumulator, [4] k-blocks issued, [5] segments,
  * [6] SM id, [7] cycles waited for operands over the first four k-blocks,
  * then %globaltimer when [8] the MMA issuer starts its W0 units and [9] its
- * G units, and, for the first Gram segment of the CTA, when its epilogue
- * [10] holds the accumulator, [11] has posted its partial, [12] sees every
+ * G units, and, for the CTA's first Gram segment, when its epilogue [10]
+ * holds the accumulator, [11] has posted its partial, [12] sees every
  * partial of the pseudo-tile posted and [13] has written its rows of G'.
  * NULL turns it off.  The buffer must outlive every call made while it is
  * set. */

@@ -57,6 +57,7 @@ __all__ = [
     "factored_intermediate_elems",
     "magnitude_scale",
     "compose_fwd",
+    "compose_delta",
     "compose_bwd",
     "compose_inner",
     "compose_bwd_from_inner",
@@ -193,6 +194,15 @@ def compose_fwd(base, lora, m, n, s: float, eps: float) -> np.ndarray:
     base, lora = _f64(base), _f64(lora)
     g, gm1, _ = magnitude_scale(m, n, eps)
     return base + (gm1 * base + g * s * lora)
+
+
+def compose_delta(base, lora, m, n, s: float, eps: float) -> np.ndarray:
+    """dY = g * s * lora + (g - 1) * base, the module output of the composition
+    contract, which the caller adds to its Y_base  [ScalingDoRA, Data
+    Availability]; g - 1 formed as in ``magnitude_scale``."""
+    base, lora = _f64(base), _f64(lora)
+    g, gm1, _ = magnitude_scale(m, n, eps)
+    return g * s * lora + gm1 * base
 
 
 def compose_bwd(dy, base, lora, m, n, s: float, eps: float):

@@ -210,6 +210,33 @@ def test_compose_equals_dora_linear_forward():
     np.testing.assert_allclose(y, oracle.dora_linear_forward(x, W0, A, B, m, s), rtol=1e-12, atol=1e-13)
 
 
+def test_compose_delta_completes_the_dense_dora_forward():
+    # Y_base + dY must be the plain DoRALinear forward with the merged weight
+    # (the caller's side of the composition contract).
+    rng = np.random.default_rng(61)
+    d_out, d_in, r, T = 10, 7, 3, 6
+    W0, A, B = _rand_module(rng, d_out, d_in, r)
+    m = rng.uniform(0.5, 2.0, d_out)
+    s = 1.5
+    x = rng.standard_normal((T, d_in))
+    n = oracle.dense_row_norm(W0, A, B, s)
+    d = oracle.compose_delta(x @ W0.T, (x @ A.T) @ B.T, m, n, s, 1e-12)
+    np.testing.assert_allclose(x @ W0.T + d, oracle.dora_linear_forward(x, W0, A, B, m, s),
+                               rtol=1e-12, atol=1e-13)
+
+
+def test_compose_delta_special_cases():
+    rng = np.random.default_rng(62)
+    base = rng.standard_normal((4, 5)); lora = rng.standard_normal((4, 5))
+    n = rng.uniform(0.5, 2.0, 5)
+    # g = 1: the delta is the LoRA branch alone
+    np.testing.assert_allclose(oracle.compose_delta(base, lora, n, n, 2.0, 1e-12), 2.0 * lora,
+                               rtol=1e-15, atol=0)
+    # m = 2 n, lora = 0: the delta is base itself (g - 1 = 1)
+    np.testing.assert_allclose(oracle.compose_delta(base, np.zeros_like(lora), 2 * n, n, 2.0, 1e-12),
+                               base, rtol=1e-15, atol=0)
+
+
 def test_compose_g_equal_one_is_lora_forward():
     rng = np.random.default_rng(7)
     base = rng.standard_normal((5, 6)); lora = rng.standard_normal((5, 6))

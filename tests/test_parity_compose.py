@@ -63,6 +63,50 @@ def test_compose_fwd_small(dtype, T, d_out, near_unity):
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("T,d_out", SMALL)
+def test_compose_fwd_delta_small(dtype, T, d_out):
+    base, lora, _, m, n = _inputs(T, d_out, dtype, 20 + T * 3 + d_out, True)
+    eps = synth.eps_for("bf16" if dtype == torch.bfloat16 else "f32")
+    d = dora.dora_compose_fwd_delta(base.cuda(), lora.cuda(), m.cuda(), n.cuda(), S, eps)
+    torch.cuda.synchronize()
+    b, l, mm, nn = map(_np, (base, lora, m, n))
+    ref = oracle.compose_delta(b, l, mm, nn, S, eps)
+    g, gm1, _ = oracle.magnitude_scale(mm, nn, eps)
+    mag = np.abs(gm1 * b) + np.abs(g * S * l)
+    chk = check_bf16 if dtype == torch.bfloat16 else check_f32
+    chk(_np(d), ref, mag, f"dY {T}x{d_out}")
+
+
+def test_compose_fwd_delta_in_place_empty_and_headline():
+    eps = synth.eps_for("bf16")
+    # in place over base, and T = 0
+    base, lora, _, m, n = _inputs(9, 264, torch.bfloat16, 7)
+    b = base.cuda()
+    d = dora.dora_compose_fwd_delta(b, lora.cuda(), m.cuda(), n.cuda(), S, eps, dy_out=b)
+    torch.cuda.synchronize()
+    assert d.data_ptr() == b.data_ptr()
+    bb, l, mm, nn = map(_np, (base, lora, m, n))
+    g, gm1, _ = oracle.magnitude_scale(mm, nn, eps)
+    check_bf16(_np(d), oracle.compose_delta(bb, l, mm, nn, S, eps),
+               np.abs(gm1 * bb) + np.abs(g * S * l), "dY in place")
+    e = torch.empty(0, 264, dtype=torch.bfloat16, device="cuda")
+    dora.dora_compose_fwd_delta(e, e.clone(), m.cuda(), n.cuda(), S, eps)
+    # headline activations [4096, 8192] near g = 1: every element
+    T, d_out = 4096, 8192
+    w = synth.WORKLOADS["headline_8192_r384"]
+    s = w.modules[0].s
+    base, lora = synth.activations(w, T, d_out, which=("base", "lora"))
+    n = torch.empty(d_out).uniform_(1.2, 1.4, generator=torch.Generator().manual_seed(3))
+    m = synth.magnitude_near_unity(w, n)
+    d = dora.dora_compose_fwd_delta(base.cuda(), lora.cuda(), m.cuda(), n.cuda(), s, eps)
+    torch.cuda.synchronize()
+    bb, l, mm, nn = map(_np, (base, lora, m, n))
+    g, gm1, _ = oracle.magnitude_scale(mm, nn, eps)
+    check_bf16(_np(d), oracle.compose_delta(bb, l, mm, nn, s, eps),
+               np.abs(gm1 * bb) + np.abs(g * s * l), "dY headline")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("T,d_out", SMALL)
 def test_compose_bwd_small(dtype, T, d_out):
     base, lora, dy, m, n = _inputs(T, d_out, dtype, 99 + T * 5 + d_out)
     eps = synth.eps_for("bf16" if dtype == torch.bfloat16 else "f32")
