@@ -1021,7 +1021,7 @@ def run_suite(args):
 # --------------------------------------------------------------------------- single cases
 
 CASES = ("merge", "fwd_train", "bwd_inner", "bwd_frozen", "fwd_grouped", "bwd_grouped",
-         "norm_grouped", "norm_sq_shard")
+         "norm_grouped", "norm_sq_shard", "norm")
 
 
 def run_case(args):
@@ -1029,7 +1029,8 @@ def run_case(args):
     except where noted): the headline module / activations for the merge, the
     training and frozen compose variants and the d_in shard; one decoder
     layer (7 modules, [2048, d_out] activations) for the grouped compose;
-    one layer's 7 modules for the grouped norm."""
+    one layer's 7 modules for the grouped norm; the headline module's norm
+    (with g) for `norm`."""
     import torch
     import dora_adapter_factored_b200 as dora
     from dora_adapter_factored_b200 import synth
@@ -1038,10 +1039,18 @@ def run_case(args):
     w = synth.WORKLOADS[WORKLOAD]
     ms = w.modules[0]
     name = args.case
-    if name in ("merge", "norm_sq_shard"):
+    if name in ("merge", "norm_sq_shard", "norm"):
         W0, A, B = synth.module_weights(w, device=dev)
         sets = [(W0, A, B), (W0.flip(0).contiguous(), A, B.flip(0).contiguous())]
-        if name == "merge":
+        if name == "norm":
+            m = synth.magnitude_from_base_rows(w, W0)
+            n_out, g_out = torch.empty_like(m), torch.empty_like(m)
+            ws = torch.empty(dora.dora_factored_norm_workspace_size(ms.d_out, ms.d_in, ms.r,
+                                                                   torch.bfloat16),
+                             dtype=torch.uint8, device=dev)
+            fn = lambda i: dora.dora_factored_norm(*sets[i % 2], ms.s, m=m, eps=eps, n_out=n_out,
+                                                   g_out=g_out, ws=ws)
+        elif name == "merge":
             ns = [dora.dora_factored_norm(*x, ms.s)[0] for x in sets]
             out = torch.empty_like(W0)
             ws = torch.empty(dora.dora_merge_weight_workspace_size(ms.d_out, ms.d_in, ms.r),

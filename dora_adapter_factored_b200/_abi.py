@@ -20,7 +20,7 @@ import torch
 from . import build as _build
 
 DORA_OK, DORA_ERR_INVALID_ARG, DORA_ERR_UNSUPPORTED, DORA_ERR_WORKSPACE, DORA_ERR_CUDA, \
-    DORA_ERR_TIMEOUT = range(6)
+    DORA_ERR_TIMEOUT, DORA_ERR_BOUNDS = range(7)
 DORA_F32, DORA_BF16 = 0, 1
 DORA_MAX_RANK = 512
 DORA_MAX_GROUP = 1024

@@ -25,8 +25,14 @@ NVCC_FLAGS = [
 ]
 
 
-def library_path() -> str:
-    return os.path.join(PKG, LIB_NAME)
+DEBUG_LIB_NAME = "libdora_debug.so"
+
+
+def library_path(debug: bool = False) -> str:
+    """The in-tree library; `debug`: the DORA_DEBUG build, whose kernels check
+    the index of every computed-address global store, skip an out-of-range one
+    and record DORA_ERR_BOUNDS in the device status word."""
+    return os.path.join(PKG, DEBUG_LIB_NAME if debug else LIB_NAME)
 
 
 def _sources():
@@ -34,8 +40,8 @@ def _sources():
                   + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def is_stale() -> bool:
-    lib = library_path()
+def is_stale(debug: bool = False) -> bool:
+    lib = library_path(debug)
     if not os.path.exists(lib):
         return True
     t = os.path.getmtime(lib)
@@ -49,9 +55,11 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found: the CUDA toolkit is required to build libdora.so")
 
 
-def build(verbose: bool = False, extra_flags=()) -> str:
-    out = library_path()
+def build(verbose: bool = False, extra_flags=(), debug: bool = False) -> str:
+    out = library_path(debug)
     tmp = out + ".tmp"
+    if debug:
+        extra_flags = [*extra_flags, "-DDORA_DEBUG"]
     cmd = [nvcc(), *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC,
            os.path.join(CSRC, "dora.cu"), "-o", tmp]
     if verbose:
@@ -67,4 +75,5 @@ def build(verbose: bool = False, extra_flags=()) -> str:
 
 if __name__ == "__main__":
     print(build(verbose="--verbose" in sys.argv,
-                extra_flags=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else []))
+                extra_flags=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [],
+                debug="--debug" in sys.argv))

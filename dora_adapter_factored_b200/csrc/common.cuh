@@ -15,6 +15,19 @@ __device__ int g_device_status;
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_device_status, 0, code); }
 
+// DORA_DEBUG builds check the index of every computed-address global store:
+// an out-of-range one is skipped and recorded as DORA_ERR_BOUNDS (never a
+// trap or an assert).  Other builds compile the check away.
+#ifdef DORA_DEBUG
+__device__ __forceinline__ bool bounds_ok(bool ok) {
+  if (!ok) record_error(DORA_ERR_BOUNDS);
+  return ok;
+}
+#define DORA_BOUNDS_OK(cond) (::dora::bounds_ok(cond))
+#else
+#define DORA_BOUNDS_OK(cond) true
+#endif
+
 // A bound on waits that must end (draining copies or MMAs already issued),
 // independent of the configurable timeout.
 constexpr unsigned long long kDrainTimeoutNs = 200000000ull;  // 0.2 s

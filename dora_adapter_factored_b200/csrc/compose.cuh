@@ -201,6 +201,7 @@ __device__ __forceinline__ void fwd_rows(const T* __restrict__ base, const T* __
           o[e] = kOut == kFwdDelta ? d : b[e] + d;
         }
         const Idx off = static_cast<Idx>(tt) * static_cast<Idx>(d_out) + static_cast<Idx>(col0);
+        if (!DORA_BOUNDS_OK(col0 >= 0 && col0 + VEC <= d_out)) continue;
         P::store(y + off, P::pack(o));
         if (kOut == kFwdYInner) {
           float in[VEC];
@@ -260,6 +261,7 @@ __device__ __forceinline__ void bwd_rows(const T* dy, const T* __restrict__ x1,
           ol[e] = gs[e] * d[e];
         }
         const Idx off = static_cast<Idx>(tt) * static_cast<Idx>(d_out) + static_cast<Idx>(col0);
+        if (!DORA_BOUNDS_OK(col0 >= 0 && col0 + VEC <= d_out)) continue;
         P::store(d_base + off, P::pack(ob));
         P::store(d_lora + off, P::pack(ol));
       }

@@ -1594,29 +1594,13 @@ static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBy
 // address stays right after a device reset; the first lookup on a device can
 // load the module, which must not happen inside a stream capture, so that
 // first call is refused while `st` is capturing.
-void* static_scratch_address(cudaStream_t st) {
-  static bool seen[kMaxDevices] = {};
-  static std::mutex mu;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lk(mu);
-  if (!seen[dev]) {
-    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs != cudaStreamCaptureStatusNone) {
-      snprintf(t_last_error, sizeof(t_last_error),
-               "dora_compose_bwd_static: the first call on device %d looks up the scratch "
-               "array and must not be made during stream capture",
-               dev);
-      return nullptr;
-    }
-  }
+void* static_scratch_address() {
   void* p = nullptr;
   const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
   if (e != cudaSuccess) {
     note_error("cudaGetSymbolAddress(static scratch)", e);
     return nullptr;
   }
-  seen[dev] = true;
   return p;
 }
 }  // namespace
@@ -1640,14 +1624,8 @@ extern "C" dora_status_t dora_compose_bwd_static(const void* dy, const void* bas
   const DeviceInfo* di = device_info();
   if (di == nullptr) return DORA_ERR_CUDA;
   if (!di->supported) return DORA_ERR_UNSUPPORTED;
-  void* scratch = static_scratch_address(reinterpret_cast<cudaStream_t>(stream));
-  if (scratch == nullptr) {
-    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-    return (cudaStreamIsCapturing(reinterpret_cast<cudaStream_t>(stream), &cs) == cudaSuccess &&
-            cs != cudaStreamCaptureStatusNone)
-               ? DORA_ERR_UNSUPPORTED
-               : DORA_ERR_CUDA;
-  }
+  void* scratch = static_scratch_address();
+  if (scratch == nullptr) return DORA_ERR_CUDA;
   // Every slot of the partial table the kernels read is written by the same
   // call first, so nothing has to be cleared between calls.
   return dora_compose_bwd(dy, base, lora, m, n, s, eps, dt, T, d_out, d_base, d_lora, dm,
@@ -1677,6 +1655,7 @@ const char* dora_status_string(dora_status_t status) {
     case DORA_ERR_WORKSPACE: return "workspace missing, too small or not 256-byte aligned";
     case DORA_ERR_CUDA: return "CUDA runtime error";
     case DORA_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+    case DORA_ERR_BOUNDS: return "a kernel skipped an out-of-range store (debug build)";
   }
   return "unknown status";
 }

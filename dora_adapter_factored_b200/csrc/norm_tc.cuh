@@ -272,6 +272,14 @@ __device__ __forceinline__ bool wait_counter_geq(const int* flag, int target,
   }
 }
 
+// Atomic add with acquire-release semantics at GPU scope; returns the old value.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
+               : "memory");
+  return old;
+}
+
 // Orders this thread's generic-proxy accesses of global memory with its
 // async-proxy (TMA) ones.
 __device__ __forceinline__ void fence_proxy_async_global() {
@@ -730,15 +738,19 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
                           static_cast<int>(rank) * kTileM;
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            if (row_base + lane + 32 * q < P->d_out)
+            if (row_base + lane + 32 * q < P->d_out &&
+                DORA_BOUNDS_OK(ord >= 0 && ord < P->seg_slots && nseg <= P->seg_slots))
               part_t[static_cast<size_t>(ord) * kPairM + lane + 32 * q] = v[q];
-          __threadfence();
+          // One acquire-release arrival per warp: it publishes the lanes'
+          // partials (ordered before it by the warp barrier) and, for the
+          // last arrival, orders the other segments' partials before the
+          // loads below.
           __syncwarp();
           int prev = 0;
-          if (lane == 0) prev = atomicAdd(P->tile_cnt + t * 2 + static_cast<int>(rank), 1);
+          if (lane == 0) prev = atom_add_acq_rel_gpu(P->tile_cnt + t * 2 + static_cast<int>(rank), 1);
           prev = __shfl_sync(0xffffffffu, prev, 0);
           if (prev == nseg - 1) {
-            __threadfence();
+            __syncwarp();
             // All of a batch's loads (kFinBatch slots of the four rows) are in
             // flight together; absent slots add zero, so the sum is the same
             // fixed slot order whatever the batching.
@@ -904,7 +916,8 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
                 const int rr = 8 * j + (lane >> 2);  // row within the warp's 32
                 const int col = colc + piece * 8;
                 const uint4 v = xp[rr * 4 + (piece ^ ((rr >> 1) & 3))];
-                if (wrow0 + rr < r && col < col_end)
+                if (wrow0 + rr < r && col < col_end &&
+                    DORA_BOUNDS_OK(col + 8 <= P->r8 && sw.kpart < P->gkp))
                   *reinterpret_cast<uint4*>(dst + static_cast<size_t>(wrow0 + rr) * P->r8 + col) = v;
               }
             };
@@ -931,7 +944,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
                 for (int j = 0; j < 4; ++j) {
                   const int rr = 8 * j + (lane >> 2);
                   const int col = colc + piece * 8;
-                  if (wrow0 + rr < r && col < r) {
+                  if (wrow0 + rr < r && col < r && DORA_BOUNDS_OK(col + 8 <= P->r8)) {
                     const size_t o = static_cast<size_t>(wrow0 + rr) * P->r8 + col;
                     *reinterpret_cast<uint4*>(s_hi + o) = z;
                     *reinterpret_cast<uint4*>(s_lo + o) = z;

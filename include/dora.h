@@ -63,7 +63,9 @@ typedef enum {
   DORA_ERR_UNSUPPORTED = 2,   /* r > 512, not an sm_100 device, too many problems */
   DORA_ERR_WORKSPACE = 3,     /* workspace missing, too small or misaligned   */
   DORA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed         */
-  DORA_ERR_TIMEOUT = 5        /* a kernel gave up on a bounded wait           */
+  DORA_ERR_TIMEOUT = 5,       /* a kernel gave up on a bounded wait           */
+  DORA_ERR_BOUNDS = 6         /* DORA_DEBUG build only: a kernel skipped a
+                                 store whose computed index was out of range */
 } dora_status_t;
 
 typedef enum { DORA_F32 = 0, DORA_BF16 = 1 } dora_dtype_t;
@@ -326,12 +328,8 @@ dora_status_t dora_merge_weight(const void *W0, const void *A, const void *B, co
  *     DORA_ERR_UNSUPPORTED before anything is launched; dora_last_error()
  *     then says how much scratch the shape needs.
  *   - Every call looks up the array's device address (cudaGetSymbolAddress),
- *     so the call stays valid after a device reset.  The first lookup on a
- *     device can load the library's device code, which a stream capture does
- *     not allow: a first call made on a capturing stream returns
- *     DORA_ERR_UNSUPPORTED (dora_last_error() says why) and launches
- *     nothing; make the first call on each device, and the first after a
- *     device reset, outside any capture.
+ *     so the call stays valid after a device reset; a failed lookup returns
+ *     DORA_ERR_CUDA and launches nothing.
  *   - All calls share the one array: calls that overlap on the GPU (other
  *     streams, other host threads) race and give wrong results.  Nothing in
  *     the array needs to start at zero: each call writes every slot it
@@ -381,9 +379,10 @@ void dora_set_timing_events(void *before, void *after);
  * operands and [3] for the accumulator, [4] k-blocks issued, [5] segments,
  * [6] SM id, [7] cycles waited for operands over the first four k-blocks,
  * then %globaltimer when [8] the MMA issuer starts its W0 units and [9] its
- * G units, and, for the CTA's first Gram segment, when its epilogue [10]
- * holds the accumulator, [11] has posted its partial, [12] sees every
- * partial of the pseudo-tile posted and [13] has written its rows of G'.
+ * G units; for the CTA's first Gram job, when its epilogue [10] holds the
+ * accumulator, [13] has issued its stores of S and [14] has fenced them, and
+ * when [11] the finisher has published them; [12] when the finisher is done
+ * with its last segment and [15] when the MMA issuer has issued its last MMA.
  * NULL turns it off.  The buffer must outlive every call made while it is
  * set. */
 void dora_set_trace_buffer(void *buf);

@@ -28,3 +28,13 @@ def built_library():
     if not os.path.exists(path) or _build.is_stale():
         _build.build()
     return path
+
+
+@pytest.fixture(scope="session")
+def built_debug_library():
+    """Path of libdora_debug.so (the DORA_DEBUG build), building it if needed."""
+    from dora_adapter_factored_b200 import build as _build
+    path = _build.library_path(debug=True)
+    if not os.path.exists(path) or _build.is_stale(debug=True):
+        _build.build(debug=True)
+    return path
