@@ -227,6 +227,22 @@ bool make_tmap_bf16_pairslab_parts(CUtensorMap* map, const void* ptr, uint64_t h
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// `parts` stacked [rows, cols] bf16 matrices (ld elements per row) as the
+// destination of 32 x 32 tiled stores from shared memory staged in the
+// 64-byte swizzle; elements past rows or cols are not written.
+bool make_tmap_bf16_store32(CUtensorMap* map, void* ptr, uint64_t rows, uint64_t cols, uint64_t ld,
+                            uint64_t parts) {
+  auto enc = tmap_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {cols, rows, parts};
+  cuuint64_t strides[2] = {ld * 2, rows * ld * 2};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Row-major bf16 matrix [rows, cols] with `ld` elements per row, loaded in
 // boxes of box_cols x box_rows with 128-byte swizzle; out-of-range elements
 // read as zero.
@@ -255,7 +271,11 @@ struct ModulePlan {
   // them for pseudo-tile 0; d_in is split into gkp parts (a job per block
   // and part), and a job costs `gram_cost` W0 units in the schedule
   int nc, gchunks, gn, gj0, gblocks, gkp, gram_cost;
-  long long units[3];  // Gram jobs, W0 units and G units
+  long long units[3];  // Gram jobs, W0 units and G units (all of them)
+  // the pool: tiles [dyn_t0, tiles) go chunk by chunk (cpt chunks each), the
+  // others are split statically; every tile's G units are pool items
+  int dyn_t0, cpt, gpi, gipt;  // gpi parts of S per G item, gipt G items per tile
+  long long dyn_begin, g_item_begin;  // first W0-chunk item / G item in the wave's pool
   // workspace (byte offsets from the workspace base) and counters (ints
   // from the start of the counter block)
   size_t off_g, off_np, off_tw, cnt_off;
@@ -287,8 +307,14 @@ constexpr int kMaxGramParts = 16;
 
 // Splits d_in into kp parts: kp jobs per Gram block, and the G units run
 // over every part of S.
+// G items of at least kMinGItemKb k-blocks: one per part of S, parts grouped
+// where a part has fewer (each pool item costs an epilogue and a hand-over).
+constexpr int kMinGItemKb = 8;
+
 void set_gram_split(ModulePlan& p, int kp) {
   p.gkp = kp;
+  p.gpi = std::min(kp, std::max(1, (kMinGItemKb + 2 * p.kb_r - 1) / (2 * p.kb_r)));
+  p.gipt = (kp + p.gpi - 1) / p.gpi;
   p.units[kPhaseGram] = static_cast<long long>(p.gblocks) * kp;
   p.units[kPhaseG] = static_cast<long long>(p.tiles) * 2 * p.kb_r * kp;
   p.gram_cost = static_cast<int>(
@@ -316,6 +342,9 @@ void plan_module(int64_t d_out, int64_t d_in, int64_t r, ModulePlan& p) {
   p.gblocks = p.gj0 + (p.pg_tiles > 1 ? gram_jobs_of_tile(static_cast<int>(r), p.nc, 1) : 0);
   p.units[kPhaseW0] = static_cast<long long>(p.tiles) * p.kb_w;
   set_gram_split(p, 1);
+  p.dyn_t0 = p.tiles;
+  p.cpt = std::max(1, (p.kb_w + kChunkKb - 1) / kChunkKb);
+  p.dyn_begin = p.g_item_begin = 0;
 }
 
 int module_counters(const ModulePlan& p) { return p.tiles * 2 + 1; }
@@ -323,6 +352,9 @@ int module_counters(const ModulePlan& p) { return p.tiles * 2 + 1; }
 // Re-read operands (A and S) of one wave of the grouped norm: well inside
 // the 126 MB L2, which also carries the W0 stream.
 constexpr size_t kWaveBudgetBytes = size_t(40) << 20;
+
+// The static W0 units of a module (its tiles before the pool's).
+long long static_w0(const ModulePlan& p) { return static_cast<long long>(p.dyn_t0) * p.kb_w; }
 
 // Runs of equal Gram-job cost of modules [m0, m1), in order.
 int gram_runs(const std::vector<ModulePlan>& plans, int m0, int m1) {
@@ -380,18 +412,23 @@ std::vector<int> plan_waves(const std::vector<ModulePlan>& plans, const int64_t*
   return begin;
 }
 
-// Every pair's W0 range non-empty and every phase's ranges in order.
+// Every phase's ranges in order, and every non-Gram pair's static W0 range
+// non-empty when there are static W0 units (a tile's W0 segments then come
+// from consecutive pairs).
 bool sched_valid(const WaveInfo& w, int pairs) {
   for (int j = 0; j < pairs; ++j)
     for (int ph = kPhaseGram; ph <= kPhaseG; ++ph) {
       const long long a = sched_begin(w, pairs, ph, j), b = sched_begin(w, pairs, ph, j + 1);
-      if (b < a || (ph == kPhaseW0 && b == a)) return false;
+      if (b < a || (ph == kPhaseW0 && w.n[1] > 0 && j >= w.J && b == a)) return false;
     }
   return true;
 }
 
 // The Gram jobs of a wave: one per pair while there are pairs enough (so
 // the Gram is done early), as runs of equal cost for the W0 split.
+// The share of a wave's W0 units its pool takes (whole tiles from its end).
+constexpr double kPoolFraction = 0.25;
+
 // Units of slack between a Gram job's end (by the cost model) and the first
 // G units of any pair: the job's S still has to be published.
 constexpr int kGramSlackUnits = 4;
@@ -447,6 +484,48 @@ bool plan_gram(WaveInfo& w, std::vector<ModulePlan>& plans, int pairs) {
   return sched_valid(w, pairs);
 }
 
+// The wave's pool: the static W0 units are the wave's first whole tiles (in
+// module order) up to (1 - kPoolFraction) of its W0 units; the rest go to the
+// pool chunk by chunk, then the G items (by then S is written).  No static W0
+// at all when there would be less than one unit per non-Gram pair.
+bool plan_pool(WaveInfo& w, std::vector<ModulePlan>& plans, int pairs) {
+  long long w0_all = 0;
+  for (int i = w.m0; i < w.m1; ++i) w0_all += plans[i].units[kPhaseW0];
+  const long long q = pairs - w.J;
+  // A wave of one module keeps all its W0 units static (its pool holds the G
+  // items); a wave of several gives the pool the last kPoolFraction of them.
+  const double frac = w.m1 - w.m0 > 1 ? kPoolFraction : 0.0;
+  long long budget = q > 0 ? static_cast<long long>(w0_all * (1.0 - frac)) : 0;
+  long long w0 = 0;
+  bool open = true;  // static tiles are a prefix of the wave's tiles in module order
+  for (int i = w.m0; i < w.m1; ++i) {
+    ModulePlan& p = plans[i];
+    p.dyn_t0 = 0;
+    while (open && p.dyn_t0 < p.tiles && w0 + p.kb_w <= budget) {
+      ++p.dyn_t0;
+      w0 += p.kb_w;
+    }
+    if (p.dyn_t0 < p.tiles) open = false;
+  }
+  if (w0 < q) {  // too little for a static split: everything from the pool
+    for (int i = w.m0; i < w.m1; ++i) plans[i].dyn_t0 = 0;
+    w0 = 0;
+  }
+  long long items = 0, gitems = 0;
+  for (int i = w.m0; i < w.m1; ++i) {
+    ModulePlan& p = plans[i];
+    p.dyn_begin = items;
+    items += static_cast<long long>(p.tiles - p.dyn_t0) * p.cpt;
+    p.g_item_begin = gitems;
+    gitems += static_cast<long long>(p.tiles) * p.gipt;
+  }
+  w.n[kPhaseW0] = w0;
+  w.n[kPhaseG] = 0;
+  w.dyn_w0_items = items;
+  w.dyn_items = items + gitems;
+  return sched_valid(w, pairs);
+}
+
 struct GroupLayout {
   std::vector<ModulePlan> plans;
   NormSched sched;
@@ -458,6 +537,7 @@ struct GroupLayout {
   size_t table_bytes = 0;  // descriptor table at the start of the workspace (grouped)
   size_t cnt_bytes = 0;    // the counter block, right after it
   int cnt_ints = 0;
+  int queue_off = 0;       // the waves' pool counters, in ints from the counter block
   size_t total_bytes = 0;
 };
 
@@ -502,29 +582,32 @@ bool layout_group(const int64_t* d_out, const int64_t* d_in, const int64_t* r, i
       wi.n[0] = wi.n[1] = wi.n[2] = 0;
       for (int i = wi.m0; i < wi.m1; ++i)
         for (int ph = 0; ph < 3; ++ph) wi.n[ph] += L.plans[i].units[ph];
-      if (wi.n[kPhaseW0] < pairs || !plan_gram(wi, L.plans, pairs)) ok = false;
+      if (wi.n[kPhaseW0] < pairs || !plan_gram(wi, L.plans, pairs)) {
+        ok = false;
+        break;
+      }
+      if (!plan_pool(wi, L.plans, pairs)) ok = false;
     }
     if (ok) break;
     if (pairs == 1) return false;
     pairs = std::max(1, pairs * 3 / 4);
   }
-  // Segment slots: the most segments any tile (W0 + G) has.
+  // Segment slots: the most segments any tile has -- its W0 segments (the
+  // static pairs that share it, or its pool chunks) and one per part of S.
   const NormSched& S = L.sched;
   L.seg_slots = 1;
   for (int w = 0; w < S.waves; ++w) {
-    long long at[3] = {0, 0, 0};
+    long long at = 0;
     for (int i = S.w[w].m0; i < S.w[w].m1; ++i) {
       const ModulePlan& p = L.plans[i];
-      for (int t = 0; t < p.tiles; ++t) {
-        const long long xw = at[kPhaseW0] + static_cast<long long>(t) * p.kb_w;
-        const long long gpt = p.units[kPhaseG] / p.tiles;  // G units per tile
-        const long long xg = at[kPhaseG] + static_cast<long long>(t) * gpt;
+      for (int t = 0; t < p.dyn_t0; ++t) {
+        const long long xw = at + static_cast<long long>(t) * p.kb_w;
         L.seg_slots = std::max(
             L.seg_slots,
-            sched_segments(S.w[w], S.pairs, kPhaseW0, xw, xw + p.kb_w, -1, nullptr) +
-                sched_segments(S.w[w], S.pairs, kPhaseG, xg, xg + gpt, -1, nullptr));
+            sched_segments(S.w[w], S.pairs, kPhaseW0, xw, xw + p.kb_w, -1, nullptr) + p.gipt);
       }
-      for (int ph = 0; ph < 3; ++ph) at[ph] += p.units[ph];
+      if (p.dyn_t0 < p.tiles) L.seg_slots = std::max(L.seg_slots, p.cpt + p.gipt);
+      at += static_w0(p);
     }
   }
   const uint32_t stage_bytes = kTileABytes + L.b_region;
@@ -539,6 +622,8 @@ bool layout_group(const int64_t* d_out, const int64_t* d_in, const int64_t* r, i
     p.cnt_off = static_cast<size_t>(cnt);
     cnt += module_counters(p);
   }
+  L.queue_off = cnt;  // one pool counter per wave after the modules' counters
+  cnt += L.sched.waves;
   L.cnt_ints = cnt;
   L.cnt_bytes = align_up(static_cast<size_t>(cnt) * sizeof(int), 256);
   off += L.cnt_bytes;
@@ -630,6 +715,8 @@ bool fill_descriptor(const dora_norm_problem_t& pr, const GroupLayout& L, int i,
     ok &= make_tmap_bf16_parts(&nd.tm_glo, g_lo, pr.r, pr.r, p.r8, p.gkp, kBlockK, p.h0);
   }
   ok &= make_tmap_bf16(&nd.tm_b, pr.B, pr.d_out, pr.r, pr.r, kBlockK, kTileM);
+  ok &= make_tmap_bf16_store32(&nd.tm_ghi_st, g_hi, pr.r, pr.r, p.r8, p.gkp);
+  ok &= make_tmap_bf16_store32(&nd.tm_glo_st, g_lo, pr.r, pr.r, p.r8, p.gkp);
   int* cnt = reinterpret_cast<int*>(ws_base + L.table_bytes) + p.cnt_off;
   nd.B = static_cast<const uint16_t*>(pr.B);
   nd.g_hi = g_hi;
@@ -642,6 +729,12 @@ bool fill_descriptor(const dora_norm_problem_t& pr, const GroupLayout& L, int i,
   nd.n_out = pr.n_out;
   nd.g_out = pr.g_out;
   for (int ph = 0; ph < 3; ++ph) nd.begin[ph] = phase_begin[ph];
+  nd.dyn_t0 = p.dyn_t0;
+  nd.cpt = p.cpt;
+  nd.gpi = p.gpi;
+  nd.gipt = p.gipt;
+  nd.dyn_begin = p.dyn_begin;
+  nd.g_item_begin = p.g_item_begin;
   nd.d_out = static_cast<int>(pr.d_out);
   nd.r = static_cast<int>(pr.r);
   nd.r8 = p.r8;
@@ -712,7 +805,8 @@ dora_status_t run_tc_group(const dora_norm_problem_t* probs, int count, bool gro
     for (int i = W.m0; i < W.m1; ++i) {
       if (!fill_descriptor(probs[i], L, i, at, base, nds[i])) return DORA_ERR_INVALID_ARG;
       nds[i].emit_sq = emit_sq ? 1 : 0;
-      for (int ph = 0; ph < 3; ++ph) at[ph] += L.plans[i].units[ph];
+      at[kPhaseGram] += L.plans[i].units[kPhaseGram];
+      at[kPhaseW0] += static_w0(L.plans[i]);
     }
   }
   const unsigned long long tmo = g_timeout_ns.load();
@@ -741,11 +835,11 @@ dora_status_t run_tc_group(const dora_norm_problem_t* probs, int count, bool gro
   if (grouped)
     launch_pdl(norm_main_kernel<true>, dim3(2 * L.sched.pairs), dim3(kNormThreads),
                L.smem_bytes, st, nds[0], table, L.sched, L.stages, L.b_region,
-               static_cast<uint32_t>(L.tmem_cols), eps, tmo, g_trace);
+               static_cast<uint32_t>(L.tmem_cols), eps, tmo, cnt + L.queue_off, g_trace);
   else
     launch_pdl(norm_main_kernel<false>, dim3(2 * L.sched.pairs), dim3(kNormThreads),
                L.smem_bytes, st, nds[0], table, L.sched, L.stages, L.b_region,
-               static_cast<uint32_t>(L.tmem_cols), eps, tmo, g_trace);
+               static_cast<uint32_t>(L.tmem_cols), eps, tmo, cnt + L.queue_off, g_trace);
   return launch_status();
 }
 

@@ -79,26 +79,6 @@ __device__ __forceinline__ void merge_give_up(volatile int* abort_flag) {
   record_error(DORA_ERR_TIMEOUT);
 }
 
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t x,
-                                             int32_t y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(smem_addr(src)), "r"(x), "r"(y)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_commit_group() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-// Waits until the bulk store groups committed so far have finished reading
-// shared memory.
-__device__ __forceinline__ void bulk_wait_group_read0() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_group0() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
 // At[j][k] = A[k][j]: 32 x 32 tiles through shared memory, block (32, 8).
 __global__ void __launch_bounds__(256)
     transpose_bf16_kernel(const uint16_t* __restrict__ A, int rows, int cols,

@@ -58,6 +58,11 @@ constexpr int kMaxChunksPerHalf = 8;         // 32-column TMEM chunks per epilog
 constexpr int kPrefetchChunks = 6;           // of which B is prefetched into registers (r <= 384)
 constexpr int kPartBufs = 4;                 // epilogue -> finisher hand-over buffers
 constexpr int kFinBatch = 8;                 // partial slots loaded together when finalising
+constexpr int kChunkKb = 16;                 // k-blocks per W0 chunk of the pool (at most)
+constexpr int kItemRing = 8;                 // pool items in flight between the roles of a pair
+// Roles that read each pool item: rank 0's two MMA issuers, eight epilogue
+// warps and finisher; rank 1's producer, eight epilogue warps and finisher.
+constexpr int kItemConsumers = 2 + kEpiWarps + 1 + 1 + kEpiWarps + 1;
 constexpr int kGramCols = 128;               // columns of G per Gram job (at most)
 // 12 warps: 65536 / 384 threads = 170 -> 168 registers per thread.
 constexpr int kNormMaxRegs = 168;
@@ -81,6 +86,8 @@ struct alignas(64) NormProblemDev {
   CUtensorMap tm_b;      // B  [d_out, r],    box 64 x 128
   CUtensorMap tm_g;      // S_hi [gkp][r][r8] as {r8, r, gkp} (or the 5-D pair view), box like tm_a
   CUtensorMap tm_glo;    // S_lo, like tm_g
+  CUtensorMap tm_ghi_st; // S_hi as {r, r, gkp}, box 32 x 32 x 1, 64-byte swizzle: the Gram jobs' stores
+  CUtensorMap tm_glo_st; // S_lo, like tm_ghi_st
   const uint16_t* B;     // bf16 bits of B, for the epilogue dot
   uint16_t* g_hi;        // [gkp][r][r8] bf16 bits of S_hi: S_p[gr][c] = 2 G'_p (c < gr), G'_p (c = gr), 0
   uint16_t* g_lo;        // [gkp][r][r8] bf16 bits of S_lo = bf16(S_p - S_hi)
@@ -91,7 +98,12 @@ struct alignas(64) NormProblemDev {
   const float* m;        // [d_out] or null
   float* n_out;          // [d_out]
   float* g_out;          // [d_out] or null
-  long long begin[3];    // first job (Gram) / unit (W0, G) of this module in its wave
+  long long begin[3];    // first job (Gram) / static W0 unit of this module in its wave
+  long long dyn_begin;   // first W0-chunk item of this module in its wave's pool
+  long long g_item_begin;  // first G item of this module among the wave's G items
+  int dyn_t0;            // tiles [0, dyn_t0) are scheduled statically, the rest chunk by chunk
+  int cpt;               // W0 chunks per pool tile
+  int gpi, gipt;         // parts of S per G item, G items per tile
   int d_out, r, r8, n_pad;
   int n0, n1;            // N of the two pair-MMA chunks (n1 = 0: single chunk; else n1 = n0)
   int h0;                // slab rows of each chunk that one CTA stages: n0 / 2
@@ -123,22 +135,24 @@ __host__ __device__ __forceinline__ int gram_jobs_of_tile(int r, int nc, int t) 
 // ---------------------------------------------------------------------------
 // Schedule.  The grouped call splits its modules (in order) into waves whose
 // re-read operands (A, S) fit in L2 together; one module alone is one wave.
-// Within a wave every pair j takes, in this order, a contiguous range of the
-// wave's Gram jobs, of its W0 units and of its G units:
-//   Gram: pairs j < J share the n[0] jobs evenly by count (the others have
-//         none); a job is never split,
-//   G:    every pair gets an even share of the n[2] G units,
-//   W0:   the rest of an even share of all work, where a Gram job counts as
-//         its cost in W0 units (the jobs of a wave form runs of equal cost),
-// so every pair has about the same work, the Gram is done early by a few
-// pairs, and the G units (which need S) come last in every pair.  The
-// boundaries are closed forms of j; the host checks that every pair's W0
-// range is non-empty and the ranges are ordered.
+// Within a wave:
+//   Gram: pairs j < J share the n[0] jobs evenly by count (a job is never
+//         split), first;
+//   W0:   the other pairs share the n[1] static W0 units (the wave's first
+//         tiles) evenly;
+//   pool: then every pair takes items from the wave's pool until it is
+//         empty: the W0 units of the remaining tiles in chunks, then one item
+//         per tile and part of S with its G units (which need S, written by
+//         then),
+// so the Gram is done early by a few pairs, and the pool evens out whatever
+// the static split did not (the Gram pairs' work, segment overheads, slower
+// pairs).  The static boundaries are closed forms of j.
 // ---------------------------------------------------------------------------
 constexpr int kMaxWaves = 64;
 constexpr int kMaxGramRuns = 8;
 struct WaveInfo {
-  long long n[3];  // Gram jobs, W0 units and G units of the wave
+  long long n[3];  // Gram jobs, static W0 units and (static) G units of the wave
+  long long dyn_w0_items, dyn_items;  // pool: W0 chunks, then G items (gipt per tile)
   long long gw;    // cost of all the wave's Gram jobs, in W0 units
   int J;           // pairs that share the Gram jobs
   int m0, m1;      // modules [m0, m1) of the table
@@ -163,17 +177,21 @@ __host__ __device__ __forceinline__ long long gram_cost_prefix(const WaveInfo& w
   return c;
 }
 
-// First unit (Gram: job) of pair j's range of phase `ph` (j = pairs gives
-// the total).
+// First unit (Gram: job) of pair j's static range of phase `ph` (j = pairs
+// gives the total).  The Gram pairs j < J share the Gram jobs and take no
+// static W0 units (they go on to the pool); the other pairs share the static
+// W0 units evenly.  There are no static G units.
 __host__ __device__ __forceinline__ long long sched_begin(const WaveInfo& w, int pairs, int ph,
                                                           int j) {
   const long long jj = j;
-  const long long jg = jj < w.J ? jj : w.J;
-  const long long gj = w.J > 0 ? jg * w.n[0] / w.J : 0;
-  if (ph == kPhaseGram) return gj;
-  const long long gp = jj * w.n[2] / pairs;
-  if (ph == kPhaseG) return gp;
-  return jj * (w.gw + w.n[1] + w.n[2]) / pairs - gram_cost_prefix(w, gj) - gp;
+  if (ph == kPhaseGram) {
+    const long long jg = jj < w.J ? jj : w.J;
+    return w.J > 0 ? jg * w.n[0] / w.J : 0;
+  }
+  if (ph == kPhaseG) return 0;
+  const long long q = pairs - w.J;
+  if (q <= 0 || jj <= w.J) return 0;
+  return (jj - w.J) * w.n[1] / q;
 }
 
 // The pair whose range of phase `ph` holds unit x (the last j with
@@ -370,8 +388,13 @@ struct SegWalk {
 //   acc_empty    rank 0 only: one arrival per epilogue warp of both CTAs.
 //   part_full[b] both: the epilogue threads have written hand-over buffer b.
 //   part_empty[b] both: the finisher has read it.
+//   item_full[i] both: rank 0's producer has written pool item slot i.
+//   item_empty[i] rank 0 only: every role of both CTAs has read it.
 // ---------------------------------------------------------------------------
 struct NormSmemTail {
+  // per epilogue warp: 32 rows x 32 bf16 of S for one tiled store, in the
+  // 64-byte swizzle of the store's tensor map (first, so 1024-byte aligned)
+  alignas(1024) uint4 xpose[kEpiWarps][32 * 4];
   uint64_t full[kMaxStages];
   uint64_t mma_done[kMaxStages];
   uint64_t empty[kMaxStages];
@@ -381,7 +404,9 @@ struct NormSmemTail {
   uint64_t part_full[kPartBufs];
   uint64_t part_empty[kPartBufs];
   float part[kPartBufs][2][kTileM];    // per buffer: the lower and upper half's value per row
-  uint4 xpose[kEpiWarps][32 * 4];      // per epilogue warp: 32 rows x 32 bf16, swizzled
+  uint64_t item_full[kItemRing];
+  uint64_t item_empty[kItemRing];
+  int item[kItemRing];                 // pool items (-1: the wave's pool is empty)
   uint32_t tmem_slot;
   int abort_flag;
 };
@@ -393,20 +418,237 @@ __device__ __forceinline__ void give_up_pair(volatile int* abort_flag, uint32_t 
   record_error(DORA_ERR_TIMEOUT);
 }
 
+// One segment of a pair's work: a static range of one phase on one tile (or a
+// Gram job), or an item of the wave's pool.
+struct Seg {
+  const NormProblemDev* P;
+  int wv, ph, tile, blk, cb, kpart, k0, n;
+  int chunk;  // pool items: the W0 chunk of the tile, or the tile's G item; -1: static
+};
+
+// A pair's segments in order, as one role sees them: per wave its static
+// Gram jobs, its static W0 range, then pool items until the wave's pool is
+// empty.  Rank 0's producer takes the items from the wave's queue counter
+// (one taken ahead, so the round trip overlaps the copies) and writes each
+// into both CTAs' item rings; every other role of either CTA reads them
+// there, in the same order.  Items are handed out in order: a wave's W0
+// chunks (tile by tile), then its G items, so a pair that runs fast takes
+// more and the pairs end together.
+template <bool kGrouped>
+struct SegSource {
+  SegWalk<kGrouped> sw;
+  const NormSched* sched;
+  const NormProblemDev* single;
+  const NormProblemDev* table;
+  NormSmemTail* tail;
+  int* queues;
+  int pairs, pair;
+  bool grabber;     // rank 0's producer
+  bool rank1;       // this CTA is rank 1: arrivals go to rank 0's item_empty
+  bool warp_wide;   // the whole warp runs this source (one arrival per warp)
+  uint32_t peer_item, peer_full, empty0;  // cluster addresses
+  unsigned long long timeout_ns;
+  const volatile int* abort;
+  int wv, stage;    // stage: 0 static Gram, 1 static W0, 2 pool, 3 wave done
+  bool started, have_nxt;
+  int nxt;
+  uint32_t d;       // item-ring slots used so far
+  bool* dep;        // grabber: whether the preceding kernel is known to be done
+  Seg s;
+
+  __device__ __forceinline__ void init(const NormSched* sc, const NormProblemDev* sg,
+                                       const NormProblemDev* tb, NormSmemTail* t, int* q, int pr,
+                                       bool grab, uint32_t rank, bool ww,
+                                       unsigned long long tmo, const volatile int* ab) {
+    sched = sc;
+    single = sg;
+    table = tb;
+    sw.single = sg;
+    sw.table = tb;
+    tail = t;
+    queues = q;
+    pairs = sc->pairs;
+    pair = pr;
+    grabber = grab;
+    rank1 = rank != 0;
+    warp_wide = ww;
+    peer_item = mapa_shared(smem_addr(&t->item[0]), rank ^ 1u);
+    peer_full = mapa_shared(smem_addr(&t->item_full[0]), rank ^ 1u);
+    empty0 = mapa_shared(smem_addr(&t->item_empty[0]), 0);
+    timeout_ns = tmo;
+    abort = ab;
+    wv = 0;
+    stage = 0;
+    started = false;
+    have_nxt = false;
+    d = 0;
+    dep = nullptr;
+  }
+
+  // Takes the next item of the current wave's pool ahead (rank 0's producer;
+  // after the counters were zeroed by the preceding kernel).
+  __device__ __forceinline__ void take_ahead() {
+    if (grabber && !have_nxt && wv < sched->waves) {
+      if (!*dep) {
+        grid_dependency_wait();
+        grid_dependency_trigger();
+        *dep = true;
+      }
+      nxt = atomicAdd(queues + wv, 1);
+      have_nxt = true;
+    }
+  }
+
+  // The pool item at position idx of wave W: a W0 chunk or a G item.
+  __device__ __forceinline__ void decode(const WaveInfo& W, long long idx) {
+    s.wv = wv;
+    s.blk = s.cb = s.kpart = 0;
+    if (idx < W.dyn_w0_items) {
+      const NormProblemDev* P = single;
+      if (kGrouped) {
+        int m = W.m0;
+        while (m + 1 < W.m1 && table[m + 1].dyn_begin <= idx) ++m;
+        P = &table[m];
+      }
+      const int local = static_cast<int>(idx - P->dyn_begin);
+      const int c = local % P->cpt;
+      s.P = P;
+      s.ph = kPhaseW0;
+      s.tile = P->dyn_t0 + local / P->cpt;
+      s.chunk = c;
+      s.k0 = c * P->kb_w / P->cpt;
+      s.n = (c + 1) * P->kb_w / P->cpt - s.k0;
+    } else {
+      const long long j = idx - W.dyn_w0_items;
+      const NormProblemDev* P = single;
+      if (kGrouped) {
+        int m = W.m0;
+        while (m + 1 < W.m1 && table[m + 1].g_item_begin <= j) ++m;
+        P = &table[m];
+      }
+      const int local = static_cast<int>(j - P->g_item_begin);
+      const int gi = local % P->gipt;
+      const int p0 = gi * P->gpi;
+      const int p1 = p0 + P->gpi < P->gkp ? p0 + P->gpi : P->gkp;
+      s.P = P;
+      s.ph = kPhaseG;
+      s.tile = local / P->gipt;
+      s.chunk = gi;
+      s.k0 = p0 * 2 * P->kb_r;
+      s.n = (p1 - p0) * 2 * P->kb_r;
+    }
+  }
+
+  // Writes v into ring slot d of both CTAs (rank 0's producer).
+  __device__ __forceinline__ bool publish(int v) {
+    const int i = static_cast<int>(d % kItemRing);
+    const uint32_t par = (d / kItemRing) & 1u;
+    ++d;
+    if (!mbar_wait(&tail->item_empty[i], par ^ 1u, timeout_ns, abort)) return false;
+    tail->item[i] = v;
+    st_cluster_u32(peer_item + 4u * i, static_cast<uint32_t>(v));
+    mbar_arrive(&tail->item_full[i]);
+    mbar_arrive_cluster(peer_full + 8u * i);
+    return true;
+  }
+
+  // Reads ring slot d (every other role).
+  __device__ __forceinline__ bool consume(int* v) {
+    const int i = static_cast<int>(d % kItemRing);
+    const uint32_t par = (d / kItemRing) & 1u;
+    ++d;
+    if (!mbar_wait_cluster(&tail->item_full[i], par, timeout_ns, abort)) return false;
+    *v = *reinterpret_cast<volatile int*>(&tail->item[i]);
+    if (warp_wide) __syncwarp();
+    if (!warp_wide || (threadIdx.x & 31) == 0) {
+      if (rank1)
+        mbar_arrive_cluster(empty0 + 8u * i);
+      else
+        mbar_arrive(&tail->item_empty[i]);
+    }
+    return true;
+  }
+
+  // Moves to the next segment; false at the end, or with *ok = false after a
+  // bounded wait gave up.
+  __device__ __forceinline__ bool next(bool* ok) {
+    while (wv < sched->waves) {
+      const WaveInfo& W = sched->w[wv];
+      if (stage < 2) {
+        if (!started) {
+          sw.start(W, pairs, pair, stage == 0 ? kPhaseGram : kPhaseW0);
+          started = true;
+        }
+        if (sw.next()) {
+          s.P = sw.P;
+          s.wv = wv;
+          s.ph = sw.ph;
+          s.tile = sw.tile;
+          s.blk = sw.blk;
+          s.cb = sw.cb;
+          s.kpart = sw.kpart;
+          s.k0 = sw.k0;
+          s.n = sw.n;
+          s.chunk = -1;
+          return true;
+        }
+        ++stage;
+        started = false;
+        continue;
+      }
+      if (stage == 2) {
+        int idx;
+        if (grabber) {
+          take_ahead();
+          idx = nxt;
+          have_nxt = false;
+          const bool end = idx >= W.dyn_items;
+          if (!publish(end ? -1 : idx)) {
+            *ok = false;
+            return false;
+          }
+          if (!end) {
+            take_ahead();
+          } else if (wv + 1 < sched->waves) {
+            ++wv;          // take the next wave's first item ahead, then come back
+            take_ahead();
+            --wv;
+          }
+          if (end) idx = -1;
+        } else if (!consume(&idx)) {
+          *ok = false;
+          return false;
+        }
+        if (idx < 0) {
+          stage = 3;
+          continue;
+        }
+        decode(W, idx);
+        return true;
+      }
+      ++wv;
+      stage = 0;
+      started = false;
+    }
+    return false;
+  }
+};
+
 template <bool kGrouped>
 __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
     norm_main_kernel(const __grid_constant__ NormProblemDev single,
                      const NormProblemDev* __restrict__ table,
                      const __grid_constant__ NormSched sched, int stages, uint32_t b_region,
                      uint32_t tmem_cols, float eps, unsigned long long timeout_ns,
-                     unsigned long long* __restrict__ trace) {
+                     int* __restrict__ queues, unsigned long long* __restrict__ trace) {
+  // queues: one pool counter per wave, zeroed by the preceding kernel.
   // trace (optional, diagnostics): per CTA kTraceWords words -- entry and
   // exit global time, MMA-issuer cycles waiting for data / for the
   // accumulator, issued k-blocks, segments, SM id, cycles waited for data
   // over the first four k-blocks; then global times: the MMA issuer starting
-  // its W0 and its G units, the epilogue holding its first Gram job's
-  // accumulator and having written that block of S, and the finisher done
-  // with its last segment.
+  // its static W0 range and its first pool item, the epilogue holding its
+  // first Gram job's accumulator and having written that block of S, and the
+  // finisher done with its last segment.
   const uint64_t t_entry = trace != nullptr ? global_timer_ns() : 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -438,6 +680,10 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
       mbar_init(&tail->part_full[b], kEpiWarps * 32);
       mbar_init(&tail->part_empty[b], 1);
     }
+    for (int i = 0; i < kItemRing; ++i) {
+      mbar_init(&tail->item_full[i], 1);  // rank 0's producer (locally, or from the peer)
+      mbar_init(&tail->item_empty[i], kItemConsumers);
+    }
     tail->abort_flag = 0;
     fence_mbar_init();
   }
@@ -453,6 +699,8 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
     prefetch_tmap(&single.tm_b);
     prefetch_tmap(&single.tm_g);
     prefetch_tmap(&single.tm_glo);
+    prefetch_tmap(&single.tm_ghi_st);
+    prefetch_tmap(&single.tm_glo_st);
   }
   // Both CTAs' barriers are initialised (and their TMEM allocated) before
   // either CTA signals the other.
@@ -461,9 +709,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
   tc_fence_after_sync();
   const uint32_t tmem_base = tail->tmem_slot;
 
-  SegWalk<kGrouped> sw;
-  sw.single = &single;
-  sw.table = table;
+  SegSource<kGrouped> src;
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ TMA producer
@@ -476,12 +722,33 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
       long long issued = 0;
       bool dep_waited = false;
       const NormProblemDev* ready = nullptr;  // module whose S is known to be written
+      const NormProblemDev* fetched = nullptr;  // module whose tensor maps were prefetched
       bool ok = true;
-      for (int wv = 0; ok && wv < sched.waves; ++wv) {
-        for (int ph = kPhaseGram; ok && ph <= kPhaseG; ++ph) {
-          sw.start(sched.w[wv], pairs, pair, ph);
-          while (ok && sw.next()) {
-            const NormProblemDev* P = sw.P;
+      src.init(&sched, &single, table, tail, queues, pair, rank == 0, rank, false, timeout_ns,
+               abort_flag);
+      src.dep = &dep_waited;
+      while (ok && src.next(&ok)) {
+            const Seg& sg = src.s;
+            const NormProblemDev* P = sg.P;
+            const int ph = sg.ph;
+            if (kGrouped && P != fetched) {
+              // Each module has its own tensor maps in the table: fetch this
+              // module's and the next one's into the TMA unit's descriptor
+              // cache ahead of their copies.
+              const NormProblemDev* Q[2] = {
+                  P, static_cast<int>(P - table) + 1 < sched.w[sg.wv].m1 ? P + 1 : P};
+              for (int i = 0; i < 2; ++i) {
+                prefetch_tmap(&Q[i]->tm_w0);
+                prefetch_tmap(&Q[i]->tm_a);
+                prefetch_tmap(&Q[i]->tm_arow);
+                prefetch_tmap(&Q[i]->tm_agram);
+                prefetch_tmap(&Q[i]->tm_b);
+                prefetch_tmap(&Q[i]->tm_g);
+                prefetch_tmap(&Q[i]->tm_glo);
+              }
+              // (the Gram jobs' store maps are fetched by the epilogue's own stores)
+              fetched = P;
+            }
             if (ph == kPhaseG && P != ready) {
               // S of this module is written by the pairs that run its Gram
               // jobs (each CTA of a pair counts its half of each job); the
@@ -500,8 +767,8 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
               fence_proxy_async_global();
               ready = P;
             }
-            const int row0 = sw.tile * kPairM + static_cast<int>(rank) * kTileM;
-            for (int k = sw.k0; k < sw.k0 + sw.n; ++k) {
+            const int row0 = sg.tile * kPairM + static_cast<int>(rank) * kTileM;
+            for (int k = sg.k0; k < sg.k0 + sg.n; ++k) {
               if (!mbar_wait(&empty[stage], phase ^ 1u, timeout_ns, abort_flag)) {
                 give_up_pair(abort_flag, peer_abort);
                 ok = false;
@@ -516,7 +783,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
                 tma_load_2d_pair(sa, &P->tm_arow, bar, kx, row0, pol_keep);
                 for (int q = 0; q < P->gchunks; ++q)
                   tma_load_2d_pair(sb + q * P->gh * 128, &P->tm_agram, bar, kx,
-                                   sw.cb * P->nc + q * P->gn + static_cast<int>(rank) * P->gh,
+                                   sg.cb * P->nc + q * P->gn + static_cast<int>(rank) * P->gh,
                                    pol_keep);
               } else {
                 if (rank == 0) mbar_arrive_expect_tx(&full[stage], P->pair_tx);
@@ -555,10 +822,13 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
                 stage = 0;
                 phase ^= 1u;
               }
+              // Once the first stages are in flight: wait for the preceding
+              // kernel (it zeroes the counters) and take the first pool item
+              // ahead.
+              if (issued == stages) src.take_ahead();
             }
-          }
-        }
       }
+      if (!ok) give_up_pair(abort_flag, peer_abort);
       if (!dep_waited) {
         grid_dependency_wait();
         grid_dependency_trigger();
@@ -591,13 +861,21 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
       bool issued_any = false;
       long long wait_data = 0, wait_first = 0, wait_acc = 0, nseg = 0, nkb = 0;
       bool ok = true;
-      for (int wv = 0; ok && wv < sched.waves; ++wv) {
-        for (int ph = kPhaseGram; ok && ph <= kPhaseG; ++ph) {
-          sw.start(sched.w[wv], pairs, pair, ph);
-          if (tracing && wv == 0 && ph > kPhaseGram)
-            trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 7 + ph] = global_timer_ns();
-          while (ok && sw.next()) {
-            const NormProblemDev* P = sw.P;
+      bool seen_w0 = false, seen_pool = false;
+      src.init(&sched, &single, table, tail, queues, pair, false, rank, false, timeout_ns,
+               abort_flag);
+      while (ok && src.next(&ok)) {
+            const Seg& sg = src.s;
+            const NormProblemDev* P = sg.P;
+            const int ph = sg.ph;
+            if (tracing && !seen_w0 && sg.chunk < 0 && ph == kPhaseW0) {
+              trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 8] = global_timer_ns();
+              seen_w0 = true;
+            }
+            if (tracing && !seen_pool && sg.chunk >= 0) {
+              trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 9] = global_timer_ns();
+              seen_pool = true;
+            }
             const long long c0 = tracing ? clock64() : 0;
             if (!mbar_wait(&tail->acc_empty, acc_phase ^ 1u, timeout_ns, abort_flag)) {
               give_up_pair(abort_flag, peer_abort);
@@ -615,7 +893,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
             const uint32_t b_off =
                 issuer == 0 ? 0u : static_cast<uint32_t>(gram ? P->gh : P->h0) * 128u;
             const uint32_t idesc = gram ? P->idesc_gram : (issuer == 0 ? P->idesc0 : P->idesc1);
-            for (int i = 0; i < sw.n; ++i) {
+            for (int i = 0; i < sg.n; ++i) {
               // The stage's copies completed on this barrier; the MMAs that
               // read it are issued straight after the wait.
               const long long c1 = tracing ? clock64() : 0;
@@ -648,9 +926,8 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
             if (!ok) break;
             umma_commit_pair(&tail->acc_full, 0x3);
             acc_phase ^= 1u;
-          }
-        }
       }
+      if (!ok) give_up_pair(abort_flag, peer_abort);
       if (tracing) trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 15] = global_timer_ns();
       if (issued_any) {
         umma_commit_pair(&tail->drain[issuer], 0x1);
@@ -671,122 +948,145 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
     // them visible and count this CTA's half of the job as written.
     // W0 / G segments: lane l takes rows l, l + 32, l + 64, l + 96 of this
     // CTA's half of the tile: it adds the two epilogue halves' values of each
-    // row (lower + upper), posts them as the segment's partial and, when this
-    // is the tile's last segment to post, sums every slot in slot order and
-    // writes n and g.
+    // row (lower + upper), posts them as the segment's partial and counts the
+    // arrival; when that was the tile's last arrival, it sums every slot in
+    // slot order and writes n and g.  The arrival's result is looked at one
+    // segment later (or at the end), so its round trip overlaps the next
+    // segment's instead of holding up the hand-over buffers.
     uint32_t seg_count = 0;
     bool dep_waited = false;
     bool gram_traced = false;
     bool ok = true;
-    for (int wv = 0; ok && wv < sched.waves; ++wv) {
-      const WaveInfo& W = sched.w[wv];
-      for (int ph = kPhaseGram; ok && ph <= kPhaseG; ++ph) {
-        sw.start(W, pairs, pair, ph);
-        while (ok && sw.next()) {
-          const NormProblemDev* P = sw.P;
-          const int t = sw.tile;
-          const int buf = static_cast<int>(seg_count % kPartBufs);
-          const uint32_t par = (seg_count / kPartBufs) & 1u;
-          ++seg_count;
-          if (!mbar_wait(&tail->part_full[buf], par, timeout_ns, abort_flag)) {
-            give_up_pair(abort_flag, peer_abort);
-            ok = false;
-            break;
-          }
-          if (ph == kPhaseGram) {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tail->part_empty[buf]);
-            if (!dep_waited) {  // the count was zeroed by the preceding kernel
-              grid_dependency_wait();
-              dep_waited = true;
-            }
-            if (lane == 0) {
-              __threadfence();
-              fence_proxy_async_global();
-              atomicAdd(P->g_ready, 1);
-              if (trace != nullptr && !gram_traced)
-                trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 11] = global_timer_ns();
-            }
-            gram_traced = true;
-            continue;
-          }
-          float v[4];
+    // the previous segment, whose arrival count is still in flight
+    bool pend = false;
+    int pend_prev = 0, pend_nseg = 0, pend_row_base = 0;
+    const NormProblemDev* pend_P = nullptr;
+    const float* pend_part = nullptr;
+    auto finish_pending = [&]() {
+      if (!pend) return;
+      pend = false;
+      const int prev = __shfl_sync(0xffffffffu, pend_prev, 0);
+      if (prev != pend_nseg - 1) return;
+      __syncwarp();
+      // All of a batch's loads (kFinBatch slots of the four rows) are in
+      // flight together; absent slots add zero, so the sum is the same
+      // fixed slot order whatever the batching.
+      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int c0 = 0; c0 < pend_nseg; c0 += kFinBatch) {
+        float v[4][kFinBatch];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int row = lane + 32 * q;
-            v[q] = tail->part[buf][0][row] + tail->part[buf][1][row];
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tail->part_empty[buf]);
-          if (!dep_waited) {  // counters and the tile table come from the preceding kernel
-            grid_dependency_wait();
-            dep_waited = true;
-          }
-          // Where this segment's partial goes among the tile's segments: its
-          // W0 segments come from consecutive pairs (found by the preceding
-          // kernel), then the G segments, split evenly over all pairs.
-          const int g_per_tile = phase_per_tile(*P, kPhaseG);
-          const long long xg = P->begin[kPhaseG] + static_cast<long long>(t) * g_per_tile;
-          int ord = 0;
-          int nseg = even_segments(xg, xg + g_per_tile, sw.xs, W.n[kPhaseG], pairs, pair, &ord);
-          const int tw = __ldcg(P->tile_w + t);
-          const int nw = tw >> 16;
-          ord = ph == kPhaseW0 ? pair - (tw & 0xffff) : ord + nw;
-          nseg += nw;
-          const int row_base = t * kPairM + static_cast<int>(rank) * kTileM;
-          float* part_t = P->partial + static_cast<size_t>(t) * P->seg_slots * kPairM +
-                          static_cast<int>(rank) * kTileM;
+        for (int q = 0; q < 4; ++q)
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (row_base + lane + 32 * q < P->d_out &&
-                DORA_BOUNDS_OK(ord >= 0 && ord < P->seg_slots && nseg <= P->seg_slots))
-              part_t[static_cast<size_t>(ord) * kPairM + lane + 32 * q] = v[q];
-          // One acquire-release arrival per warp: it publishes the lanes'
-          // partials (ordered before it by the warp barrier) and, for the
-          // last arrival, orders the other segments' partials before the
-          // loads below.
-          __syncwarp();
-          int prev = 0;
-          if (lane == 0) prev = atom_add_acq_rel_gpu(P->tile_cnt + t * 2 + static_cast<int>(rank), 1);
-          prev = __shfl_sync(0xffffffffu, prev, 0);
-          if (prev == nseg - 1) {
-            __syncwarp();
-            // All of a batch's loads (kFinBatch slots of the four rows) are in
-            // flight together; absent slots add zero, so the sum is the same
-            // fixed slot order whatever the batching.
-            float sum[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int c0 = 0; c0 < nseg; c0 += kFinBatch) {
-              float v[4][kFinBatch];
+          for (int u = 0; u < kFinBatch; ++u)
+            v[q][u] = c0 + u < pend_nseg
+                          ? __ldcg(pend_part + static_cast<size_t>(c0 + u) * kPairM + lane + 32 * q)
+                          : 0.f;
 #pragma unroll
-              for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < 4; ++q)
 #pragma unroll
-                for (int u = 0; u < kFinBatch; ++u)
-                  v[q][u] = c0 + u < nseg ? __ldcg(part_t + static_cast<size_t>(c0 + u) * kPairM +
-                                                   lane + 32 * q)
-                                          : 0.f;
+          for (int u = 0; u < kFinBatch; ++u) sum[q] += v[q][u];
+      }
+      const NormProblemDev* Q = pend_P;
 #pragma unroll
-              for (int q = 0; q < 4; ++q)
-#pragma unroll
-                for (int u = 0; u < kFinBatch; ++u) sum[q] += v[q][u];
-            }
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int row = lane + 32 * q;
-              const int grow = row_base + row;
-              if (grow >= P->d_out) continue;
-              if (P->emit_sq) {
-                P->n_out[grow] = sum[q];
-              } else {
-                const float n = __fsqrt_rn(fmaxf(sum[q], 0.f));
-                P->n_out[grow] = n;
-                if (P->m != nullptr && P->g_out != nullptr)
-                  P->g_out[grow] = __fdiv_rn(__ldg(P->m + grow), fmaxf(n, eps));
-              }
-            }
-          }
+      for (int q = 0; q < 4; ++q) {
+        const int grow = pend_row_base + lane + 32 * q;
+        if (grow >= Q->d_out) continue;
+        if (Q->emit_sq) {
+          Q->n_out[grow] = sum[q];
+        } else {
+          const float n = __fsqrt_rn(fmaxf(sum[q], 0.f));
+          Q->n_out[grow] = n;
+          if (Q->m != nullptr && Q->g_out != nullptr)
+            Q->g_out[grow] = __fdiv_rn(__ldg(Q->m + grow), fmaxf(n, eps));
         }
       }
+    };
+    src.init(&sched, &single, table, tail, queues, pair, false, rank, true, timeout_ns,
+             abort_flag);
+    while (ok && src.next(&ok)) {
+      const Seg& sg = src.s;
+      const NormProblemDev* P = sg.P;
+      const int ph = sg.ph;
+      const int t = sg.tile;
+      const int buf = static_cast<int>(seg_count % kPartBufs);
+      const uint32_t par = (seg_count / kPartBufs) & 1u;
+      ++seg_count;
+      // A static tile's W0 segment table, requested before the hand-over wait
+      // (it comes from the preceding kernel, waited for once before).
+      const bool static_tile = ph != kPhaseGram && t < P->dyn_t0;
+      int tw = 0;
+      if (static_tile && dep_waited) tw = __ldcg(P->tile_w + t);
+      if (!mbar_wait(&tail->part_full[buf], par, timeout_ns, abort_flag)) {
+        ok = false;
+        break;
+      }
+      if (ph == kPhaseGram) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tail->part_empty[buf]);
+        if (!dep_waited) {  // the count was zeroed by the preceding kernel
+          grid_dependency_wait();
+          dep_waited = true;
+        }
+        if (lane == 0) {
+          __threadfence();
+          fence_proxy_async_global();
+          atomicAdd(P->g_ready, 1);
+          if (trace != nullptr && !gram_traced)
+            trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 11] = global_timer_ns();
+        }
+        gram_traced = true;
+        continue;
+      }
+      float v[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int row = lane + 32 * q;
+        v[q] = tail->part[buf][0][row] + tail->part[buf][1][row];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tail->part_empty[buf]);
+      if (!dep_waited) {  // counters and the tile table come from the preceding kernel
+        grid_dependency_wait();
+        dep_waited = true;
+        if (static_tile) tw = __ldcg(P->tile_w + t);
+      }
+      // Where this segment's partial goes among the tile's segments: first
+      // its W0 segments -- on a static tile, consecutive pairs (found by the
+      // preceding kernel), on a pool tile one per chunk -- then its G items.
+      int nw, ord;
+      if (static_tile) {
+        nw = tw >> 16;
+        ord = sg.chunk < 0 ? pair - (tw & 0xffff) : nw + sg.chunk;
+      } else {
+        nw = P->cpt;
+        ord = ph == kPhaseW0 ? sg.chunk : nw + sg.chunk;
+      }
+      const int nseg = nw + P->gipt;
+      const int row_base = t * kPairM + static_cast<int>(rank) * kTileM;
+      float* part_t = P->partial + static_cast<size_t>(t) * P->seg_slots * kPairM +
+                      static_cast<int>(rank) * kTileM;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (row_base + lane + 32 * q < P->d_out &&
+            DORA_BOUNDS_OK(ord >= 0 && ord < P->seg_slots && nseg <= P->seg_slots))
+          part_t[static_cast<size_t>(ord) * kPairM + lane + 32 * q] = v[q];
+      // One acquire-release arrival per warp: it publishes the lanes'
+      // partials (ordered before it by the warp barrier) and, for the last
+      // arrival, orders the other segments' partials before the loads of the
+      // finalisation.  The previous segment's arrival is looked at first.
+      __syncwarp();
+      int prev = 0;
+      if (lane == 0) prev = atom_add_acq_rel_gpu(P->tile_cnt + t * 2 + static_cast<int>(rank), 1);
+      finish_pending();
+      pend = true;
+      pend_prev = prev;
+      pend_nseg = nseg;
+      pend_row_base = row_base;
+      pend_P = P;
+      pend_part = part_t;
     }
+    if (ok) finish_pending();
+    if (!ok) give_up_pair(abort_flag, peer_abort);
     if (trace != nullptr && lane == 0)
       trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 12] = global_timer_ns();
   } else if (warp < kEpiWarps) {
@@ -801,13 +1101,13 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
     uint32_t phase = 0, acc_phase = 0, seg_count = 0;
     bool gram_traced = false;
     bool ok = true;
-    for (int wv = 0; ok && wv < sched.waves; ++wv) {
-      const WaveInfo& W = sched.w[wv];
-      for (int ph = kPhaseGram; ok && ph <= kPhaseG; ++ph) {
-        sw.start(W, pairs, pair, ph);
-        while (ok && sw.next()) {
-          const NormProblemDev* P = sw.P;
-          const int t = sw.tile;
+    src.init(&sched, &single, table, tail, queues, pair, false, rank, true, timeout_ns,
+             abort_flag);
+    while (ok && src.next(&ok)) {
+          const Seg& sg = src.s;
+          const NormProblemDev* P = sg.P;
+          const int ph = sg.ph;
+          const int t = sg.tile;
           const int r = P->r;
           // the row of W0 (or, for the Gram, of A) this thread finishes
           const int grow = t * kPairM + static_cast<int>(rank) * kTileM + row;
@@ -831,7 +1131,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
                              : make_uint4(0u, 0u, 0u, 0u);
             }
           float ss = 0.f;
-          for (int i = 0; i < sw.n; ++i) {
+          for (int i = 0; i < sg.n; ++i) {
             // The MMAs that read this stage have completed, so its copies
             // (completed on rank 0's barrier) have landed here too.
             if (!mbar_wait(&mma_done[stage], phase, timeout_ns, abort_flag)) {
@@ -868,25 +1168,43 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
             // ---- Gram job: this CTA's 128 rows gr of the block of G
             // (columns [cb nc, cb nc + nc)) over part kpart of d_in, scaled
             // into S_kpart (row gr, column c): 2 G' for c < gr, G' for c = gr,
-            // 0 above.  A thread writes 8 consecutive columns of its row per
-            // 16-byte store.
+            // 0 above.
             const bool first = trace != nullptr && threadIdx.x == 0 && !gram_traced;
             if (first) trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 10] = global_timer_ns();
-            const int col0 = sw.cb * P->nc;
+            const int col0 = sg.cb * P->nc;
             const int col_end = min(r, col0 + P->nc);
             const float hs = P->half_s;
-            // This warp's 32 rows of S_kpart (TMEM lanes (warp & 3) * 32 + i).
+            // This warp's 32 rows of S_kpart (TMEM lanes (warp & 3) * 32 + i):
+            // per 32 columns, hi then lo, the warp writes the 32 x 32 block
+            // into its staging tile (16-byte units swizzled by row, the
+            // store's 64-byte swizzle: no bank conflicts) and one lane stores
+            // it with TMA; rows and columns past r are clipped by the store.
             const int wrow0 = t * kPairM + static_cast<int>(rank) * kTileM + (warp & 3) * 32;
-            uint16_t* s_hi = P->g_hi + static_cast<size_t>(sw.kpart) * r * P->r8;
-            uint16_t* s_lo = P->g_lo + static_cast<size_t>(sw.kpart) * r * P->r8;
             uint4* xp = tail->xpose[warp];
-            // Lane (i, piece): rows wrow0 + 8 j + lane / 4, 16-byte piece lane % 4
-            // of the 32 columns, after the transpose through shared memory
-            // (16-byte units swizzled by row, so that both sides are free of
-            // bank conflicts).
-            const int piece = lane & 3;
-            auto put_chunk = [&](int colc, const float (&acc)[32], bool lo_part) {
-              uint32_t w[16];
+            bool pending = false;  // a store may still be reading the staging tile
+            auto stage_store = [&](const uint32_t (&w)[16], const CUtensorMap* map, int colc) {
+              if (pending) {
+                if (lane == 0) bulk_wait_group_read0();
+                __syncwarp();
+              }
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                xp[lane * 4 + (j ^ ((lane >> 1) & 3))] =
+                    make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0 && DORA_BOUNDS_OK(colc % 8 == 0 && sg.kpart < P->gkp)) {
+                tma_store_3d(map, xp, colc, wrow0, sg.kpart);
+                bulk_commit_group();
+              }
+              pending = true;
+            };
+#pragma unroll 1
+            for (int c = c_lo; c < c_hi; ++c) {
+              float acc[32];
+              tmem_load_32cols(tmem_base + lane_base + c * 32, acc);
+              const int colc = col0 + c * 32;
+              uint32_t wh[16], wl[16];
 #pragma unroll
               for (int e = 0; e < 16; ++e) {
                 float x[2];
@@ -897,63 +1215,39 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
                   x[f] = col < grow ? 2.f * hs * g : (col == grow ? hs * g : 0.f);
                 }
                 const uint16_t h0 = f32_to_bf16_rn(x[0]), h1 = f32_to_bf16_rn(x[1]);
-                uint16_t v0 = h0, v1 = h1;
-                if (lo_part) {
-                  v0 = f32_to_bf16_rn(x[0] - __uint_as_float(static_cast<uint32_t>(h0) << 16));
-                  v1 = f32_to_bf16_rn(x[1] - __uint_as_float(static_cast<uint32_t>(h1) << 16));
-                }
-                w[e] = static_cast<uint32_t>(v0) | (static_cast<uint32_t>(v1) << 16);
+                const uint16_t l0 = f32_to_bf16_rn(x[0] - __uint_as_float(static_cast<uint32_t>(h0) << 16));
+                const uint16_t l1 = f32_to_bf16_rn(x[1] - __uint_as_float(static_cast<uint32_t>(h1) << 16));
+                wh[e] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+                wl[e] = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
               }
-              __syncwarp();
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                xp[lane * 4 + (j ^ ((lane >> 1) & 3))] =
-                    make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-              __syncwarp();
-              uint16_t* dst = lo_part ? s_lo : s_hi;
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int rr = 8 * j + (lane >> 2);  // row within the warp's 32
-                const int col = colc + piece * 8;
-                const uint4 v = xp[rr * 4 + (piece ^ ((rr >> 1) & 3))];
-                if (wrow0 + rr < r && col < col_end &&
-                    DORA_BOUNDS_OK(col + 8 <= P->r8 && sw.kpart < P->gkp))
-                  *reinterpret_cast<uint4*>(dst + static_cast<size_t>(wrow0 + rr) * P->r8 + col) = v;
+              if (colc < col_end) {
+                stage_store(wh, &P->tm_ghi_st, colc);
+                stage_store(wl, &P->tm_glo_st, colc);
               }
-            };
-#pragma unroll 1
-            for (int c = c_lo; c < c_hi; ++c) {
-              float acc[32];
-              tmem_load_32cols(tmem_base + lane_base + c * 32, acc);
-              put_chunk(col0 + c * 32, acc, false);
-              put_chunk(col0 + c * 32, acc, true);
             }
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc_empty0);
             // The pseudo-tile's last block also zeroes the columns past it
-            // (all above the diagonal for these rows).
+            // (all above the diagonal for these rows), 32 at a time, split
+            // between the two halves.
             const int njt = gram_jobs_of_tile(r, P->nc, t);
-            if (sw.cb == njt - 1) {
-              // columns [z0, r) of the warp's 32 rows, 32 columns per step,
-              // split between the two halves
-              const int z0 = njt * P->nc;
-              const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-              for (int colc = z0 + half * 32; colc < r; colc += 64)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  const int rr = 8 * j + (lane >> 2);
-                  const int col = colc + piece * 8;
-                  if (wrow0 + rr < r && col < r && DORA_BOUNDS_OK(col + 8 <= P->r8)) {
-                    const size_t o = static_cast<size_t>(wrow0 + rr) * P->r8 + col;
-                    *reinterpret_cast<uint4*>(s_hi + o) = z;
-                    *reinterpret_cast<uint4*>(s_lo + o) = z;
-                  }
-                }
+            if (sg.cb == njt - 1) {
+              const uint32_t zero[16] = {};
+              for (int colc = njt * P->nc + half * 32; colc < r; colc += 64) {
+                stage_store(zero, &P->tm_ghi_st, colc);
+                stage_store(zero, &P->tm_glo_st, colc);
+              }
             }
+            // Every store of this warp has written global memory before the
+            // hand-over below.
+            if (lane == 0) {
+              bulk_wait_group0();
+              fence_proxy_async_global();
+            }
+            __syncwarp();
             // The finisher publishes these rows of S to the TMA reads of every
             // pair's G units once all epilogue threads have handed over.
-            if (first) trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 13] = global_timer_ns();
             fence_proxy_async_global();
             if (first) trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 14] = global_timer_ns();
             const int buf = static_cast<int>(seg_count % kPartBufs);
@@ -998,16 +1292,20 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
           const int buf = static_cast<int>(seg_count % kPartBufs);
           const uint32_t use = seg_count / kPartBufs;
           ++seg_count;
-          if (!mbar_wait(&tail->part_empty[buf], (use & 1u) ^ 1u, timeout_ns, abort_flag)) {
+          const long long cw = trace != nullptr ? clock64() : 0;
+          const bool handed =
+              mbar_wait(&tail->part_empty[buf], (use & 1u) ^ 1u, timeout_ns, abort_flag);
+          if (trace != nullptr && threadIdx.x == 0)
+            trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 13] += clock64() - cw;
+          if (!handed) {
             give_up_pair(abort_flag, peer_abort);
             ok = false;
             break;
           }
           tail->part[buf][half][row] = fmaf(P->two_s, dot, ss);
           mbar_arrive(&tail->part_full[buf]);
-        }
-      }
     }
+    if (!ok) give_up_pair(abort_flag, peer_abort);
   }
 
   // Neither CTA leaves (or frees TMEM) while the other may still signal it,
@@ -1048,7 +1346,7 @@ __global__ void __launch_bounds__(256)
     const WaveInfo& W = sched.w[w];
     for (int m = W.m0; m < W.m1; ++m) {
       const NormProblemDev* P = kGrouped ? &table[m] : &single;
-      for (int t = tid; t < P->tiles; t += stride) {
+      for (int t = tid; t < P->dyn_t0; t += stride) {
         const long long x0 = P->begin[kPhaseW0] + static_cast<long long>(t) * P->kb_w;
         const int f = sched_pair_of(W, sched.pairs, kPhaseW0, x0);
         const int l = sched_pair_of(W, sched.pairs, kPhaseW0, x0 + P->kb_w - 1);
