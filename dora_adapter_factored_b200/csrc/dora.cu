@@ -429,10 +429,6 @@ bool sched_valid(const WaveInfo& w, int pairs) {
 // The share of a wave's W0 units its pool takes (whole tiles from its end).
 constexpr double kPoolFraction = 0.25;
 
-// Units of slack between a Gram job's end (by the cost model) and the first
-// G units of any pair: the job's S still has to be published.
-constexpr int kGramSlackUnits = 4;
-
 // Work of the wave (W0 units; Gram jobs at their cost; G units), with the
 // modules' current splits.
 long long wave_work(const WaveInfo& w, const std::vector<ModulePlan>& plans) {
@@ -445,18 +441,25 @@ long long wave_work(const WaveInfo& w, const std::vector<ModulePlan>& plans) {
 
 bool plan_gram(WaveInfo& w, std::vector<ModulePlan>& plans, int pairs) {
   // Each module's parts of d_in: the fewest (every part adds the module's G
-  // units once more) for which a job ends before any pair reaches its G
-  // units, with some slack.
-  for (int i = w.m0; i < w.m1; ++i) set_gram_split(plans[i], 1);
+  // units once more) for which a job ends, by the cost model, before the
+  // other pairs finish their static W0 units (the G items that need S come
+  // after those).
+  const double frac = w.m1 - w.m0 > 1 ? kPoolFraction : 0.0;
+  long long w0_all = 0;
+  for (int i = w.m0; i < w.m1; ++i) {
+    set_gram_split(plans[i], 1);
+    w0_all += plans[i].units[kPhaseW0];
+  }
   for (int i = w.m0; i < w.m1; ++i) {
     ModulePlan& p = plans[i];
     const int kp_max = std::max(1, std::min(kMaxGramParts, p.kb_w / 2));
     for (int kp = 1; kp <= kp_max; ++kp) {
       set_gram_split(p, kp);
-      long long g = 0;
-      for (int m = w.m0; m < w.m1; ++m) g += plans[m].units[kPhaseG];
-      const double share = static_cast<double>(wave_work(w, plans)) / pairs;
-      if (p.gram_cost + kGramSlackUnits <= share - static_cast<double>(g) / pairs) break;
+      long long jobs = 0;
+      for (int m = w.m0; m < w.m1; ++m) jobs += plans[m].units[kPhaseGram];
+      const long long q = std::max<long long>(1, pairs - std::min<long long>(jobs, pairs));
+      const double static_per_pair = static_cast<double>(w0_all) * (1.0 - frac) / q;
+      if (p.gram_cost <= static_per_pair) break;
     }
   }
   for (int ph = 0; ph < 3; ++ph) {
@@ -819,15 +822,18 @@ dora_status_t run_tc_group(const dora_norm_problem_t* probs, int count, bool gro
       return DORA_ERR_CUDA;
     table = ntab;
   }
-  int max_tiles = 1;
-  for (const auto& p : L.plans) max_tiles = std::max(max_tiles, p.tiles);
-  const unsigned prep_blocks = static_cast<unsigned>(
-      std::min<long long>(64, ceil_div_ll(std::max(L.cnt_ints, max_tiles), 256)));
+  // One-warp blocks (each fits beside a fused-kernel CTA), as many as the
+  // counters and static tiles need at about 8 items per lane.
+  long long static_tiles = 0;
+  for (const auto& p : L.plans) static_tiles += p.dyn_t0;
+  const unsigned prep_blocks = static_cast<unsigned>(std::min<long long>(
+      64, std::max<long long>(1, ceil_div_ll(std::max<long long>(L.cnt_ints, static_tiles),
+                                             32 * 8))));
   if (grouped)
-    launch_pdl(norm_prep_kernel<true>, dim3(prep_blocks), dim3(256), 0, st, cnt, L.cnt_ints,
+    launch_pdl(norm_prep_kernel<true>, dim3(prep_blocks), dim3(32), 0, st, cnt, L.cnt_ints,
                nds[0], table, count, L.sched);
   else
-    launch_pdl(norm_prep_kernel<false>, dim3(prep_blocks), dim3(256), 0, st, cnt, L.cnt_ints,
+    launch_pdl(norm_prep_kernel<false>, dim3(prep_blocks), dim3(32), 0, st, cnt, L.cnt_ints,
                nds[0], table, count, L.sched);
   dora_status_t s;
   if ((s = launch_status()) != DORA_OK) return s;

@@ -1331,9 +1331,11 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
 // its counters (every module's counters form one block of ints) and writes
 // each tile's W0 segment table (first pair, number of pairs: the W0 ranges
 // are not an even split, so this takes a search per tile), then lets the
-// fused kernel launch; it waits for this grid before it reads either.
+// fused kernel launch; it waits for this grid before it reads either.  One
+// warp of at most 32 registers: it fits beside a fused-kernel CTA on the same
+// SM (which leaves 1024 registers free), so no pair waits for it to finish.
 template <bool kGrouped>
-__global__ void __launch_bounds__(256)
+__global__ void __maxnreg__(32)
     norm_prep_kernel(int* __restrict__ cnt, int n_cnt, const __grid_constant__ NormProblemDev single,
                      const NormProblemDev* __restrict__ table, int count,
                      const __grid_constant__ NormSched sched) {
