@@ -93,7 +93,7 @@ struct alignas(64) NormProblemDev {
   uint16_t* g_lo;        // [gkp][r][r8] bf16 bits of S_lo = bf16(S_p - S_hi)
   float* partial;        // [tiles][seg_slots][256] per-row partials
   int* tile_cnt;         // [tiles * 2] segments posted per CTA half of each tile
-  int* g_ready;          // [1] CTA halves of Gram jobs whose rows of S are written
+  int* g_ready;          // [1] epilogue warps of Gram jobs whose rows of S are written
   int* tile_w;           // [tiles] first pair | (pairs << 16) of each tile's W0 units
   const float* m;        // [d_out] or null
   float* n_out;          // [d_out]
@@ -272,6 +272,14 @@ __device__ __forceinline__ float dot_bf16x8(const float* acc, uint4 v) {
   return s;
 }
 
+// Splits two fp32 values into bf16 hi (round to nearest even) and bf16 lo
+// (the residual, rounded the same way), each pair packed low half first.
+__device__ __forceinline__ void split_bf16_hi_lo(float x0, float x1, uint32_t* hi, uint32_t* lo) {
+  const uint32_t h = pack_bf16x2_rn(x0, x1);
+  *hi = h;
+  *lo = pack_bf16x2_rn(x0 - __uint_as_float(h << 16), x1 - __uint_as_float(h & 0xffff0000u));
+}
+
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
@@ -288,6 +296,11 @@ __device__ __forceinline__ bool wait_counter_geq(const int* flag, int target,
     if (global_timer_ns() - t0 > timeout_ns) return false;
     __nanosleep(64);
   }
+}
+
+// Atomic add with release semantics at GPU scope (no result).
+__device__ __forceinline__ void red_add_release_gpu(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 // Atomic add with acquire-release semantics at GPU scope; returns the old value.
@@ -751,14 +764,14 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
             }
             if (ph == kPhaseG && P != ready) {
               // S of this module is written by the pairs that run its Gram
-              // jobs (each CTA of a pair counts its half of each job); the
-              // count they raise was zeroed by the preceding kernel.
+              // jobs (each epilogue warp of both CTAs counts its rows of each
+              // job); the count they raise was zeroed by the preceding kernel.
               if (!dep_waited) {
                 grid_dependency_wait();
                 grid_dependency_trigger();
                 dep_waited = true;
               }
-              if (!wait_counter_geq(P->g_ready, 2 * P->gblocks * P->gkp, timeout_ns,
+              if (!wait_counter_geq(P->g_ready, 2 * kEpiWarps * P->gblocks * P->gkp, timeout_ns,
                                     abort_flag)) {
                 give_up_pair(abort_flag, peer_abort);
                 ok = false;
@@ -944,8 +957,8 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
     }
   } else if (warp == kFinisherWarp) {
     // ------------------------------------------- partials and finalisation
-    // Gram jobs: once every epilogue thread has written its rows of S, make
-    // them visible and count this CTA's half of the job as written.
+    // Gram jobs: only the hand-over buffer is passed on (the epilogue warps
+    // publish their rows of S themselves).
     // W0 / G segments: lane l takes rows l, l + 32, l + 64, l + 96 of this
     // CTA's half of the tile: it adds the two epilogue halves' values of each
     // row (lower + upper), posts them as the segment's partial and counts the
@@ -955,7 +968,6 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
     // segment's instead of holding up the hand-over buffers.
     uint32_t seg_count = 0;
     bool dep_waited = false;
-    bool gram_traced = false;
     bool ok = true;
     // the previous segment, whose arrival count is still in flight
     bool pend = false;
@@ -1020,21 +1032,9 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
         ok = false;
         break;
       }
-      if (ph == kPhaseGram) {
+      if (ph == kPhaseGram) {  // published by the epilogue warps themselves
         __syncwarp();
         if (lane == 0) mbar_arrive(&tail->part_empty[buf]);
-        if (!dep_waited) {  // the count was zeroed by the preceding kernel
-          grid_dependency_wait();
-          dep_waited = true;
-        }
-        if (lane == 0) {
-          __threadfence();
-          fence_proxy_async_global();
-          atomicAdd(P->g_ready, 1);
-          if (trace != nullptr && !gram_traced)
-            trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 11] = global_timer_ns();
-        }
-        gram_traced = true;
         continue;
       }
       float v[4];
@@ -1174,6 +1174,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
             const int col0 = sg.cb * P->nc;
             const int col_end = min(r, col0 + P->nc);
             const float hs = P->half_s;
+            const float two_hs = 2.f * hs;
             // This warp's 32 rows of S_kpart (TMEM lanes (warp & 3) * 32 + i):
             // per 32 columns, hi then lo, the warp writes the 32 x 32 block
             // into its staging tile (16-byte units swizzled by row, the
@@ -1205,20 +1206,29 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
               tmem_load_32cols(tmem_base + lane_base + c * 32, acc);
               const int colc = col0 + c * 32;
               uint32_t wh[16], wl[16];
+              // The warp's 32 rows are wrow0 .. wrow0 + 31: a block of
+              // columns wholly left of all of them is scaled by 2 G' as a
+              // whole, one wholly right of them is zero, and the block that
+              // holds the diagonal goes element by element.
+              if (colc + 31 < wrow0) {
 #pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                float x[2];
+                for (int e = 0; e < 16; ++e)
+                  split_bf16_hi_lo(two_hs * acc[2 * e], two_hs * acc[2 * e + 1], &wh[e], &wl[e]);
+              } else if (colc > wrow0 + 31) {
 #pragma unroll
-                for (int f = 0; f < 2; ++f) {
-                  const int col = colc + 2 * e + f;
-                  const float g = acc[2 * e + f];
-                  x[f] = col < grow ? 2.f * hs * g : (col == grow ? hs * g : 0.f);
+                for (int e = 0; e < 16; ++e) wh[e] = wl[e] = 0u;
+              } else {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                  float x[2];
+#pragma unroll
+                  for (int f = 0; f < 2; ++f) {
+                    const int col = colc + 2 * e + f;
+                    const float g = acc[2 * e + f];
+                    x[f] = col < grow ? two_hs * g : (col == grow ? hs * g : 0.f);
+                  }
+                  split_bf16_hi_lo(x[0], x[1], &wh[e], &wl[e]);
                 }
-                const uint16_t h0 = f32_to_bf16_rn(x[0]), h1 = f32_to_bf16_rn(x[1]);
-                const uint16_t l0 = f32_to_bf16_rn(x[0] - __uint_as_float(static_cast<uint32_t>(h0) << 16));
-                const uint16_t l1 = f32_to_bf16_rn(x[1] - __uint_as_float(static_cast<uint32_t>(h1) << 16));
-                wh[e] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
-                wl[e] = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
               }
               if (colc < col_end) {
                 stage_store(wh, &P->tm_ghi_st, colc);
@@ -1239,17 +1249,17 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
                 stage_store(zero, &P->tm_glo_st, colc);
               }
             }
-            // Every store of this warp has written global memory before the
-            // hand-over below.
+            // Once every store of this warp has written global memory, its
+            // rows of S are published to the TMA reads of every pair's G
+            // units: a release add on the count their producers wait for.
             if (lane == 0) {
               bulk_wait_group0();
               fence_proxy_async_global();
+              if (first) trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 14] = global_timer_ns();
+              red_add_release_gpu(P->g_ready, 1);
+              if (first) trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 11] = global_timer_ns();
             }
             __syncwarp();
-            // The finisher publishes these rows of S to the TMA reads of every
-            // pair's G units once all epilogue threads have handed over.
-            fence_proxy_async_global();
-            if (first) trace[static_cast<size_t>(blockIdx.x) * kTraceWords + 14] = global_timer_ns();
             const int buf = static_cast<int>(seg_count % kPartBufs);
             const uint32_t use = seg_count / kPartBufs;
             ++seg_count;

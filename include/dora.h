@@ -378,11 +378,12 @@ void dora_set_timing_events(void *before, void *after);
  * [0] entry and [1] exit %globaltimer, cycles the MMA issuer waited [2] for
  * operands and [3] for the accumulator, [4] k-blocks issued, [5] segments,
  * [6] SM id, [7] cycles waited for operands over the first four k-blocks,
- * then %globaltimer when [8] the MMA issuer starts its W0 units and [9] its
- * G units; for the CTA's first Gram job, when its epilogue [10] holds the
- * accumulator, [13] has issued its stores of S and [14] has fenced them, and
- * when [11] the finisher has published them; [12] when the finisher is done
- * with its last segment and [15] when the MMA issuer has issued its last MMA.
+ * then %globaltimer when [8] the MMA issuer starts its static W0 units and
+ * [9] its first pool item; for the CTA's first Gram job, when its epilogue's
+ * first warp [10] holds the accumulator, [14] has its stores of S written
+ * and [11] has published them; [12] when the finisher is done with its last
+ * segment and [15] when the MMA issuer has issued its last MMA; [13] cycles
+ * the first epilogue thread waited for a free hand-over buffer, summed.
  * NULL turns it off.  The buffer must outlive every call made while it is
  * set. */
 void dora_set_trace_buffer(void *buf);
