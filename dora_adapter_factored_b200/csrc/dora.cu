@@ -429,16 +429,6 @@ bool sched_valid(const WaveInfo& w, int pairs) {
 // The share of a wave's W0 units its pool takes (whole tiles from its end).
 constexpr double kPoolFraction = 0.25;
 
-// Work of the wave (W0 units; Gram jobs at their cost; G units), with the
-// modules' current splits.
-long long wave_work(const WaveInfo& w, const std::vector<ModulePlan>& plans) {
-  long long work = 0;
-  for (int i = w.m0; i < w.m1; ++i)
-    work += plans[i].units[kPhaseW0] + plans[i].units[kPhaseG] +
-            plans[i].units[kPhaseGram] * plans[i].gram_cost;
-  return work;
-}
-
 bool plan_gram(WaveInfo& w, std::vector<ModulePlan>& plans, int pairs) {
   // Each module's parts of d_in: the fewest (every part adds the module's G
   // units once more) for which a job ends, by the cost model, before the
@@ -1306,10 +1296,11 @@ bool merge_layout(int64_t d_out, int64_t d_in, int64_t r, MergeLayout& L) {
   if (d_out < 1 || d_in < 1 || r < 1 || r > DORA_MAX_RANK) return false;
   L.kb = static_cast<int>(ceil_div_ll(r, kMergeK));
   L.r8 = round_up_int(static_cast<int>(r), 8);
-  L.tiles_m = static_cast<int>(ceil_div_ll(d_out, kMergeM));
+  L.tiles_m = static_cast<int>(ceil_div_ll(d_out, kMergePairM));
   L.tiles_n = static_cast<int>(ceil_div_ll(d_in, kMergeN));
-  // Shared memory: two W0 / W' staging tiles and as many 32 KiB k-block
-  // stages (A^T, or B while a row block starts) as fit: three.
+  // Shared memory: two W0 / W' staging tiles and as many 16 KiB k-block
+  // stages (this CTA's half of A^T, or its B rows while a row block
+  // starts) as fit: six.
   const size_t tail = align_up(sizeof(MergeSmemTail), 128);
   const size_t fixed = 1024 + static_cast<size_t>(kMergeWBufs) * kMergeTileBytes + tail;
   if (fixed + 2 * kMergeStageBytes > static_cast<size_t>(kMaxDynSmem)) return false;
@@ -1364,7 +1355,7 @@ dora_status_t dora_merge_weight(const void* W0, const void* A, const void* B, co
   ok &= make_tmap_bf16(&P.tm_w0, W0, d_out, d_in, d_in, 64, kMergeM);
   ok &= make_tmap_bf16(&P.tm_out, W_out, d_out, d_in, d_in, 64, 32);
   ok &= make_tmap_bf16(&P.tm_b, B, d_out, r, r, kMergeK, kMergeM);
-  ok &= make_tmap_bf16(&P.tm_at, At, d_in, r, L.r8, kMergeK, kMergeN);  // 256-row boxes
+  ok &= make_tmap_bf16(&P.tm_at, At, d_in, r, L.r8, kMergeK, kMergeM);  // a CTA's 128 rows
   if (!ok) return DORA_ERR_INVALID_ARG;
   P.m = m;
   P.n = n;
@@ -1376,16 +1367,16 @@ dora_status_t dora_merge_weight(const void* W0, const void* A, const void* B, co
   P.kb = L.kb;
   P.tiles_n = L.tiles_n;
   P.tiles = L.tiles_m * L.tiles_n;
-  P.idesc = idesc_bf16_f32(kMergeM, kMergeN);
+  P.idesc = idesc_bf16_f32(kMergePairM, kMergeN);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   launch_pdl(transpose_bf16_kernel, dim3((unsigned)ceil_div_ll(d_in, 32), (unsigned)ceil_div_ll(r, 32)),
              dim3(32, 8), 0, cs, static_cast<const uint16_t*>(A), static_cast<int>(r),
              static_cast<int>(d_in), At, L.r8);
   dora_status_t st = launch_status();
   if (st != DORA_OK) return st;
-  const int ctas = std::min(di->sms, P.tiles);
+  const int pairs = std::max(1, std::min(di->sms / 2, P.tiles));
   TimedLaunch tl(cs);
-  launch_pdl(merge_kernel, dim3(ctas), dim3(kMergeThreads), L.smem_bytes, cs, P, L.stages,
+  launch_pdl(merge_kernel, dim3(2 * pairs), dim3(kMergeThreads), L.smem_bytes, cs, P, L.stages,
              g_timeout_ns.load());
   return launch_status();
 }

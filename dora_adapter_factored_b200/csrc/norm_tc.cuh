@@ -675,7 +675,6 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
-  const int pairs = sched.pairs;
   const int pair = blockIdx.x >> 1;
   const uint32_t peer_abort = mapa_shared(smem_addr(&tail->abort_flag), rank ^ 1u);
 
@@ -1237,7 +1236,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
             }
             tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc_empty0);
+            if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty0);
             // The pseudo-tile's last block also zeroes the columns past it
             // (all above the diagonal for these rows), 32 at a time, split
             // between the two halves.
@@ -1297,7 +1296,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(kNormMaxRegs)
           }
           tc_fence_before_sync();
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(acc_empty0);
+          if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty0);
           // Hand this half's value of the row to the finisher warp.
           const int buf = static_cast<int>(seg_count % kPartBufs);
           const uint32_t use = seg_count / kPartBufs;
