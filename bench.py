@@ -695,6 +695,33 @@ def _device_time(fn, iters, flush):
     return statistics.median(a.elapsed_time(b) for a, b in evs) * 1e-3
 
 
+def _back_to_back_time(fn, K=10, R=5):
+    """Device time (s) per call of fn(i) in a stream of such calls: K calls
+    (input sets alternating, the two sets together larger than L2, so each
+    call reads its inputs from HBM) captured in a CUDA graph and replayed R
+    times between a pair of CUDA events; no L2 flush between calls, so no
+    write-back of a flush buffer runs under the call either."""
+    import torch
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        for i in range(K):
+            fn(i)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    for _ in range(R):
+        g.replay()
+    b.record(st)
+    torch.cuda.synchronize()
+    del g
+    return a.elapsed_time(b) * 1e-3 / (R * K)
+
+
 def _oracle_seconds(fn, scale, budget_s=2.0):
     """Mean wall time of the oracle sample fn(), times `scale` (the sample's
     share of the full call), over about budget_s seconds."""
@@ -727,7 +754,8 @@ def run_suite(args):
     iters = max(5, min(args.steps, 30))
     cores = blas_threads()
 
-    def emit(name, workload, t_gpu, flops, nbytes, oracle_s=None, sample=None, extra=None):
+    def emit(name, workload, t_gpu, flops, nbytes, oracle_s=None, sample=None, extra=None,
+             t_b2b=None):
         t_roof = max(flops / TC, nbytes / HBM)
         bound = "tensor" if flops / TC >= nbytes / HBM else "hbm"
         line = {"suite": name, "workload": workload, "us": t_gpu * 1e6,
@@ -741,6 +769,9 @@ def run_suite(args):
             line["cpu_baseline"] = {"kind": "oracle", "seconds_per_call": oracle_s,
                                     "cores": cores, "sample": sample,
                                     "gpu_speedup": oracle_s / t_gpu}
+        if t_b2b is not None:
+            line["us_back_to_back"] = t_b2b * 1e6
+            line["frac_back_to_back"] = t_roof / t_b2b
         if extra:
             line.update(extra)
         print(json.dumps(line), flush=True)
@@ -762,6 +793,7 @@ def run_suite(args):
         for i in range(3):
             fn(i)
         t = _device_time(fn, iters, flush)
+        tb = _back_to_back_time(fn)
         W0h, Ah, Bh = (x.float().cpu().numpy() for x in sets[0])
         rows = 16
         o_s, reps = _oracle_seconds(lambda: oracle.rows_dense_row_norm(
@@ -769,7 +801,8 @@ def run_suite(args):
             ms.s), ms.d_out / rows)
         emit("factored_norm", key, t, 2.0 * ms.d_out * ms.d_in * ms.r,
              2.0 * (ms.d_out * ms.d_in + ms.r * ms.d_in + ms.d_out * ms.r), o_s,
-             f"fp64 dense norm of {rows} of {ms.d_out} rows ({reps} repeats), scaled")
+             f"fp64 dense norm of {rows} of {ms.d_out} rows ({reps} repeats), scaled",
+             t_b2b=tb if ms.d_out * ms.d_in * 2 * 2 > (126 << 20) else None)
         del sets, ws
 
     # ---- grouped norm over the 56-module layer stack
@@ -904,9 +937,10 @@ def run_suite(args):
         for i in range(3):
             fn(i)
         t = _device_time(fn, iters, flush)
+        tb = _back_to_back_time(fn)
         o_s, reps = _oracle_seconds(samples[name], T / 64)
         emit(name, "headline [4096, 8192] bf16", t, 0.0, passes * act, o_s,
-             f"fp64 on 64 of {T} tokens ({reps} repeats), scaled")
+             f"fp64 on 64 of {T} tokens ({reps} repeats), scaled", t_b2b=tb)
     del sets
 
     # ---- compose sweep: fused vs eager over the layer-stack shapes
@@ -971,6 +1005,7 @@ def run_suite(args):
         for i in range(3):
             fn(i)
         t = _device_time(fn, iters, flush)
+        tb = _back_to_back_time(fn)
         W0h, Ah, Bh = (x.float().cpu().numpy().astype(np.float64) for x in sets[0])
         mh, nh = ns[0][1].double().cpu().numpy(), ns[0][0].double().cpu().numpy()
         rows = 16
@@ -978,7 +1013,7 @@ def run_suite(args):
             W0h[:rows], Ah, Bh[:rows], mh[:rows], nh[:rows], ms.s, eps), ms.d_out / rows)
         emit("merge_weight", key, t, 2.0 * ms.d_out * ms.d_in * ms.r,
              2.0 * (2 * ms.d_out * ms.d_in + ms.r * ms.d_in + ms.d_out * ms.r), o_s,
-             f"fp64 merge of {rows} of {ms.d_out} rows ({reps} repeats), scaled")
+             f"fp64 merge of {rows} of {ms.d_out} rows ({reps} repeats), scaled", t_b2b=tb)
         del sets, ws, out
 
     # ---- one column shard of the headline module (d_in-sharded norm, 2 ranks)
@@ -997,9 +1032,11 @@ def run_suite(args):
     for i in range(3):
         fn(i)
     t = _device_time(fn, iters, flush)
+    tb = _back_to_back_time(fn)
     wd = b0 - a0
     emit("factored_norm_sq_shard", f"headline module, columns [{a0}, {b0}) of 2 shards", t,
-         2.0 * ms.d_out * wd * ms.r, 2.0 * (ms.d_out * wd + ms.r * wd + ms.d_out * ms.r))
+         2.0 * ms.d_out * wd * ms.r, 2.0 * (ms.d_out * wd + ms.r * wd + ms.d_out * ms.r),
+         t_b2b=tb)
     # ---- stable compose against a naive bf16 evaluation near g = 1 ("Scaling
     # DoRA", section 3: about 3.0x lower peak error at d_out = 8192, d_in =
     # 2048, against fp64); read as [2048, 8192] activations, g = 1 + N(0, 0.0015)
