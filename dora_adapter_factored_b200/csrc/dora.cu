@@ -328,15 +328,16 @@ void plan_module(int64_t d_out, int64_t d_in, int64_t r, ModulePlan& p) {
   p.tiles = static_cast<int>(ceil_div_ll(d_out, kPairM));
   p.pg_tiles = static_cast<int>(ceil_div_ll(r, kPairM));
   p.r8 = round_up_int(static_cast<int>(r), 8);
-  // Gram blocks of 256 columns as two chunks of 128 (one per MMA issuer)
-  // where the slab region holds them, else one chunk of up to 128.
-  if (p.n_pad >= 2 * kGramCols) {
-    p.nc = 2 * kGramCols;
-    p.gchunks = 2;
-  } else {
-    p.nc = std::min(kGramCols, p.n_pad);
-    p.gchunks = 1;
-  }
+  // Gram blocks of up to 128 columns, one chunk (one MMA issuer).  At
+  // r = 384 that is five blocks (two on the first pseudo-tile, three on the
+  // second) where 256-column blocks made three: a job's k-block stages
+  // 24 KiB instead of 32, the second pseudo-tile's padded rows cost
+  // 128-column blocks instead of 256, and the jobs spread over more pairs,
+  // so S is written sooner (headline: by ~32 us of the call against ~40 us,
+  // the kernel 60 us against 64 us).  The kernel also runs two chunks of
+  // 128 (gchunks = 2) should a block be made 256 wide.
+  p.nc = std::min(kGramCols, p.n_pad);
+  p.gchunks = 1;
   p.gn = p.nc / p.gchunks;
   p.gj0 = gram_jobs_of_tile(static_cast<int>(r), p.nc, 0);
   p.gblocks = p.gj0 + (p.pg_tiles > 1 ? gram_jobs_of_tile(static_cast<int>(r), p.nc, 1) : 0);
