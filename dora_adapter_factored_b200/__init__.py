@@ -13,7 +13,8 @@ from ._abi import (  # noqa: F401
     dora_compose_bwd_workspace_size, dora_compose_fwd, dora_compose_fwd_grouped,
     dora_compose_fwd_train, dora_compose_fwd_delta, dora_debug_unsignalled_wait, dora_factored_norm,
     dora_factored_norm_grouped, dora_factored_norm_grouped_workspace_size,
-    dora_factored_norm_sq, dora_factored_norm_workspace_size, dora_norm_finalize, dora_get_device_status, dora_launch_count,
+    dora_factored_norm_sq, dora_factored_norm_workspace_size, dora_norm_finalize, dora_norm_plan_check,
+    dora_get_device_status, dora_launch_count,
     dora_merge_weight, dora_merge_weight_workspace_size, dora_set_timing_events, dora_set_trace_buffer, dora_set_wait_timeout_ns, dora_version,
     load_library, status_string,
 )

@@ -20,7 +20,7 @@ import torch
 from . import build as _build
 
 DORA_OK, DORA_ERR_INVALID_ARG, DORA_ERR_UNSUPPORTED, DORA_ERR_WORKSPACE, DORA_ERR_CUDA, \
-    DORA_ERR_TIMEOUT, DORA_ERR_BOUNDS = range(7)
+    DORA_ERR_TIMEOUT, DORA_ERR_BOUNDS, DORA_ERR_INTERNAL = range(8)
 DORA_F32, DORA_BF16 = 0, 1
 DORA_MAX_RANK = 512
 DORA_MAX_GROUP = 1024
@@ -38,6 +38,7 @@ EXPORTED = (
     "dora_compose_fwd_grouped", "dora_compose_bwd_grouped_workspace_size",
     "dora_compose_bwd_grouped", "dora_merge_weight_workspace_size", "dora_merge_weight",
     "dora_factored_norm_sq", "dora_norm_finalize", "dora_compose_fwd_delta",
+    "dora_norm_plan_check",
 )
 
 
@@ -45,7 +46,7 @@ class DoraError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
         detail = ""
-        if status == DORA_ERR_CUDA:
+        if status in (DORA_ERR_CUDA, DORA_ERR_INTERNAL):
             detail = " [" + load_library().dora_last_error().decode() + "]"
         super().__init__(f"{where}: {status_string(status)} (status {status}){detail}")
 
@@ -126,6 +127,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.dora_last_error.restype = ctypes.c_char_p
         lib.dora_set_trace_buffer.argtypes = [c_vp]
         lib.dora_set_trace_buffer.restype = None
+        lib.dora_norm_plan_check.argtypes = [ctypes.POINTER(c_i64)] * 3 + [c_i, c_i, c_i]
+        lib.dora_norm_plan_check.restype = c_i
         lib.dora_compose_bwd_static.argtypes = [c_vp, c_vp, c_vp, c_vp, c_vp, c_f, c_f, c_i,
                                                 c_i64, c_i64, c_vp, c_vp, c_vp, c_vp]
         lib.dora_compose_bwd_static.restype = c_i
@@ -234,6 +237,17 @@ def dora_set_timing_events(before: Optional[torch.cuda.Event], after: Optional[t
 def dora_set_trace_buffer(buf: Optional[torch.Tensor]) -> None:
     """Diagnostics: per-CTA trace of the fused norm GEMM (see include/dora.h)."""
     load_library().dora_set_trace_buffer(_dev(buf, "trace", torch.int64) if buf is not None else None)
+
+
+def dora_norm_plan_check(shapes: Sequence[Sequence[int]], grouped: bool = False,
+                         pairs: int = 74) -> None:
+    """Host-only self-check of the fused norm's schedule for modules of
+    `shapes` [(d_out, d_in, r), ...] on `pairs` CTA pairs (see include/dora.h);
+    raises DoraError naming the first invariant that fails."""
+    n = len(shapes)
+    arr = [(ctypes.c_int64 * n)(*[int(x[k]) for x in shapes]) for k in range(3)]
+    _check(load_library().dora_norm_plan_check(arr[0], arr[1], arr[2], n, int(bool(grouped)),
+                                               int(pairs)), "dora_norm_plan_check")
 
 
 def dora_debug_unsignalled_wait(timeout_ns: int, stream=None) -> None:

@@ -11,6 +11,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <string>
 #include <utility>
 #include <vector>
 
@@ -990,6 +991,163 @@ dora_status_t norm_impl(const void* W0, const void* A, const void* B, dora_dtype
   }
   return launch_status();
 }
+
+// The schedule self-check behind dora_norm_plan_check: walks every segment
+// the kernel's roles take (the same closed forms and item decoding) and
+// checks coverage and partial-slot numbering.  Returns "" when every
+// invariant holds, else the first one that failed.
+std::string check_norm_plan(const GroupLayout& L) {
+  char msg[256];
+  const NormSched& S = L.sched;
+  const int P = S.pairs;
+  for (int w = 0; w < S.waves; ++w) {
+    const WaveInfo& W = S.w[w];
+    const int nm = W.m1 - W.m0;
+    std::vector<long long> bw(nm), bg(nm);
+    long long aw = 0, ag = 0;
+    for (int i = 0; i < nm; ++i) {
+      const ModulePlan& p = L.plans[W.m0 + i];
+      bw[i] = aw;
+      bg[i] = ag;
+      aw += static_w0(p);
+      if (W.n[kPhaseG] > 0) ag += p.units[kPhaseG];
+    }
+    if (aw != W.n[kPhaseW0] || ag != W.n[kPhaseG]) {
+      snprintf(msg, sizeof(msg), "wave %d: static W0 / G totals %lld / %lld against %lld / %lld",
+               w, aw, ag, W.n[kPhaseW0], W.n[kPhaseG]);
+      return msg;
+    }
+    // Gram jobs: consecutive ranges of the wave's jobs, in pair order.
+    long long gx = 0;
+    for (int j = 0; j < P; ++j) {
+      const long long a = sched_begin(W, P, kPhaseGram, j), b = sched_begin(W, P, kPhaseGram, j + 1);
+      if (a != gx || b < a) {
+        snprintf(msg, sizeof(msg), "wave %d: Gram range of pair %d is [%lld, %lld)", w, j, a, b);
+        return msg;
+      }
+      gx = b;
+    }
+    if (gx != W.n[kPhaseGram]) {
+      snprintf(msg, sizeof(msg), "wave %d: Gram ranges cover %lld of %lld jobs", w, gx,
+               W.n[kPhaseGram]);
+      return msg;
+    }
+    // Per tile of each module: (nseg, slot) of every segment; units covered.
+    std::vector<std::vector<std::vector<std::pair<int, int>>>> slots(nm);
+    std::vector<std::vector<long long>> cov_w(nm), cov_g(nm);
+    for (int i = 0; i < nm; ++i) {
+      const ModulePlan& p = L.plans[W.m0 + i];
+      slots[i].assign(p.tiles, {});
+      cov_w[i].assign(p.tiles, 0);
+      cov_g[i].assign(p.tiles, 0);
+    }
+    auto module_of = [&](long long x, bool g) {
+      int i = 0;
+      while (i + 1 < nm && (g ? bg[i + 1] : bw[i + 1]) <= x) ++i;
+      return i;
+    };
+    auto g_segments = [&](int i, int t, int me, int* gord) {
+      const ModulePlan& p = L.plans[W.m0 + i];
+      if (W.n[kPhaseG] > 0) {
+        const int per = 2 * p.kb_r * p.gkp;
+        const long long xg = bg[i] + static_cast<long long>(t) * per;
+        return sched_segments(W, P, kPhaseG, xg, xg + per, me, gord);
+      }
+      return p.gipt;
+    };
+    auto w0_segments = [&](int i, int t, int* first) {
+      const ModulePlan& p = L.plans[W.m0 + i];
+      const long long xw = bw[i] + static_cast<long long>(t) * p.kb_w;
+      const int f = sched_pair_of(W, P, kPhaseW0, xw);
+      *first = f;
+      return sched_pair_of(W, P, kPhaseW0, xw + p.kb_w - 1) - f + 1;
+    };
+    // each pair's static W0 and G ranges
+    for (int j = 0; j < P; ++j) {
+      for (int ph : {kPhaseW0, kPhaseG}) {
+        long long x = sched_begin(W, P, ph, j);
+        const long long e = sched_begin(W, P, ph, j + 1);
+        while (x < e) {
+          const int i = module_of(x, ph == kPhaseG);
+          const ModulePlan& p = L.plans[W.m0 + i];
+          const int per = ph == kPhaseG ? 2 * p.kb_r * p.gkp : p.kb_w;
+          const long long local = x - (ph == kPhaseG ? bg[i] : bw[i]);
+          const int t = static_cast<int>(local / per);
+          const int k0 = static_cast<int>(local % per);
+          const int len = static_cast<int>(std::min<long long>(e - x, per - k0));
+          if (t >= p.tiles || (ph == kPhaseW0 && t >= p.dyn_t0)) {
+            snprintf(msg, sizeof(msg), "wave %d pair %d: static unit %lld lands on tile %d", w,
+                     j, x, t);
+            return msg;
+          }
+          int gord = -1, f = 0;
+          const int ng = g_segments(i, t, j, &gord);
+          const int nw = w0_segments(i, t, &f);
+          slots[i][t].push_back({nw + ng, ph == kPhaseW0 ? j - f : nw + gord});
+          (ph == kPhaseG ? cov_g : cov_w)[i][t] += len;
+          x += len;
+        }
+      }
+    }
+    // the pool items
+    for (long long idx = 0; idx < W.dyn_items; ++idx) {
+      if (idx < W.dyn_w0_items) {
+        int i = 0;
+        while (i + 1 < nm && L.plans[W.m0 + i + 1].dyn_begin <= idx) ++i;
+        const ModulePlan& p = L.plans[W.m0 + i];
+        const int local = static_cast<int>(idx - p.dyn_begin);
+        const int c = local % p.cpt, t = p.dyn_t0 + local / p.cpt;
+        if (t >= p.tiles) {
+          snprintf(msg, sizeof(msg), "wave %d: pool item %lld lands on tile %d", w, idx, t);
+          return msg;
+        }
+        int gord;
+        slots[i][t].push_back({p.cpt + g_segments(i, t, -1, &gord), c});
+        cov_w[i][t] += (c + 1) * p.kb_w / p.cpt - c * p.kb_w / p.cpt;
+      } else {
+        const long long jj = idx - W.dyn_w0_items;
+        int i = 0;
+        while (i + 1 < nm && L.plans[W.m0 + i + 1].g_item_begin <= jj) ++i;
+        const ModulePlan& p = L.plans[W.m0 + i];
+        const int local = static_cast<int>(jj - p.g_item_begin);
+        const int gi = local % p.gipt, t = local / p.gipt;
+        if (t >= p.tiles || W.n[kPhaseG] > 0) {
+          snprintf(msg, sizeof(msg), "wave %d: G item %lld (tile %d) not expected", w, jj, t);
+          return msg;
+        }
+        int f = 0;
+        const int nw = t < p.dyn_t0 ? w0_segments(i, t, &f) : p.cpt;
+        const int p0 = gi * p.gpi, p1 = std::min(p0 + p.gpi, p.gkp);
+        slots[i][t].push_back({nw + p.gipt, nw + gi});
+        cov_g[i][t] += static_cast<long long>(p1 - p0) * 2 * p.kb_r;
+      }
+    }
+    for (int i = 0; i < nm; ++i) {
+      const ModulePlan& p = L.plans[W.m0 + i];
+      for (int t = 0; t < p.tiles; ++t) {
+        const auto& v = slots[i][t];
+        if (cov_w[i][t] != p.kb_w || cov_g[i][t] != 2LL * p.kb_r * p.gkp) {
+          snprintf(msg, sizeof(msg), "wave %d module %d tile %d: %lld of %d W0 and %lld of %d G "
+                   "units covered", w, W.m0 + i, t, cov_w[i][t], p.kb_w, cov_g[i][t],
+                   2 * p.kb_r * p.gkp);
+          return msg;
+        }
+        const int nseg = v.empty() ? 0 : v[0].first;
+        std::vector<int> seen(std::max(nseg, 1), 0);
+        bool ok = static_cast<int>(v.size()) == nseg && nseg <= L.seg_slots;
+        for (const auto& q : v) {
+          if (q.first != nseg || q.second < 0 || q.second >= nseg || seen[q.second]++) ok = false;
+        }
+        if (!ok) {
+          snprintf(msg, sizeof(msg), "wave %d module %d tile %d: %zu segments, nseg %d, %d slots",
+                   w, W.m0 + i, t, v.size(), nseg, L.seg_slots);
+          return msg;
+        }
+      }
+    }
+  }
+  return "";
+}
 }  // namespace
 
 extern "C" {
@@ -1748,6 +1906,7 @@ const char* dora_status_string(dora_status_t status) {
     case DORA_ERR_CUDA: return "CUDA runtime error";
     case DORA_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
     case DORA_ERR_BOUNDS: return "a kernel skipped an out-of-range store (debug build)";
+    case DORA_ERR_INTERNAL: return "a schedule invariant does not hold";
   }
   return "unknown status";
 }
@@ -1769,6 +1928,30 @@ uint64_t dora_launch_count(void) { return g_launches.load(); }
 const char* dora_last_error(void) { return t_last_error; }
 
 void dora_set_trace_buffer(void* buf) { g_trace = static_cast<unsigned long long*>(buf); }
+
+dora_status_t dora_norm_plan_check(const int64_t* d_out, const int64_t* d_in, const int64_t* r,
+                                   int count, int grouped, int pairs) {
+  if (d_out == nullptr || d_in == nullptr || r == nullptr || count < 1 || pairs < 1 ||
+      pairs > 512 || (!grouped && count != 1))
+    return DORA_ERR_INVALID_ARG;
+  if (count > DORA_MAX_GROUP) return DORA_ERR_UNSUPPORTED;
+  for (int i = 0; i < count; ++i) {
+    if (d_out[i] < 1 || d_in[i] < 1 || r[i] < 1) return DORA_ERR_INVALID_ARG;
+    if (r[i] > DORA_MAX_RANK || d_out[i] > (1ll << 31) - 1 || d_in[i] > (1ll << 31) - 1)
+      return DORA_ERR_UNSUPPORTED;
+  }
+  static thread_local dora::GroupLayout L;
+  if (!dora::layout_group(d_out, d_in, r, count, grouped != 0, pairs, L)) {
+    snprintf(dora::t_last_error, sizeof(dora::t_last_error), "no schedule for these sizes");
+    return DORA_ERR_UNSUPPORTED;
+  }
+  const std::string err = check_norm_plan(L);
+  if (!err.empty()) {
+    snprintf(dora::t_last_error, sizeof(dora::t_last_error), "%s", err.c_str());
+    return DORA_ERR_INTERNAL;
+  }
+  return DORA_OK;
+}
 
 void dora_set_timing_events(void* before, void* after) {
   t_ev_before = static_cast<cudaEvent_t>(before);

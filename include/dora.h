@@ -64,8 +64,10 @@ typedef enum {
   DORA_ERR_WORKSPACE = 3,     /* workspace missing, too small or misaligned   */
   DORA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed         */
   DORA_ERR_TIMEOUT = 5,       /* a kernel gave up on a bounded wait           */
-  DORA_ERR_BOUNDS = 6         /* DORA_DEBUG build only: a kernel skipped a
+  DORA_ERR_BOUNDS = 6,        /* DORA_DEBUG build only: a kernel skipped a
                                  store whose computed index was out of range */
+  DORA_ERR_INTERNAL = 7       /* dora_norm_plan_check: a schedule invariant
+                                 does not hold (a library defect)            */
 } dora_status_t;
 
 typedef enum { DORA_F32 = 0, DORA_BF16 = 1 } dora_dtype_t;
@@ -387,6 +389,20 @@ void dora_set_timing_events(void *before, void *after);
  * NULL turns it off.  The buffer must outlive every call made while it is
  * set. */
 void dora_set_trace_buffer(void *buf);
+/* Host-only self-check of the fused norm's schedule (no device, no launch):
+ * plans `count` modules (sizes d_out[i] x d_in[i], rank r[i]; `grouped`
+ * non-zero plans them as one grouped call, else count must be 1) for
+ * `pairs` CTA pairs (1 .. 512; 74 on a B200) and walks every segment the
+ * kernel's roles would take -- each pair's static Gram jobs and W0 range,
+ * then every pool item (W0 chunks, G items) -- to check that every W0 and G
+ * unit of every tile is covered exactly once, that the Gram jobs partition
+ * the wave's jobs, and that the partial slots of every tile are distinct,
+ * numbered 0 .. nseg-1, agree on nseg and fit the workspace's slot count.
+ * Returns DORA_OK; DORA_ERR_INVALID_ARG / DORA_ERR_UNSUPPORTED for sizes the
+ * norm rejects; DORA_ERR_INTERNAL with the first failed invariant in
+ * dora_last_error(). */
+dora_status_t dora_norm_plan_check(const int64_t *d_out, const int64_t *d_in, const int64_t *r,
+                                   int count, int grouped, int pairs);
 /* Launches one thread that waits, with the same bounded wait the
  * tensor-core pipelines use, on a barrier that nothing ever signals, giving
  * up after `timeout_ns` (clamped to [1 us, 1 s]).  The give-up is recorded as

@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(built_library):
 
 def test_status_strings_and_version(built_library):
     lib = dora.load_library(built_library)
-    for code in range(7):
+    for code in range(8):
         assert len(dora.status_string(code)) > 0
     assert dora.status_string(99) == "unknown status"
     assert dora.dora_version() == 100
