@@ -322,23 +322,31 @@ void set_gram_split(ModulePlan& p, int kp) {
       ceil_div_ll(ceil_div_ll(p.kb_w, kp) * (256 + p.nc), 256 + p.n_pad) + kGramJobCharge);
 }
 
-void plan_module(int64_t d_out, int64_t d_in, int64_t r, ModulePlan& p) {
+void plan_module(int64_t d_out, int64_t d_in, int64_t r, bool wide_gram, ModulePlan& p) {
   plan_n_side(static_cast<int>(r), p);
   p.kb_w = static_cast<int>(ceil_div_ll(d_in, kBlockK));
   p.kb_r = static_cast<int>(ceil_div_ll(r, kBlockK));
   p.tiles = static_cast<int>(ceil_div_ll(d_out, kPairM));
   p.pg_tiles = static_cast<int>(ceil_div_ll(r, kPairM));
   p.r8 = round_up_int(static_cast<int>(r), 8);
-  // Gram blocks of up to 128 columns, one chunk (one MMA issuer).  At
-  // r = 384 that is five blocks (two on the first pseudo-tile, three on the
-  // second) where 256-column blocks made three: a job's k-block stages
-  // 24 KiB instead of 32, the second pseudo-tile's padded rows cost
-  // 128-column blocks instead of 256, and the jobs spread over more pairs,
-  // so S is written sooner (headline: by ~32 us of the call against ~40 us,
-  // the kernel 60 us against 64 us).  The kernel also runs two chunks of
-  // 128 (gchunks = 2) should a block be made 256 wide.
-  p.nc = std::min(kGramCols, p.n_pad);
-  p.gchunks = 1;
+  // Gram blocks.  A single module: blocks of up to 128 columns, one chunk
+  // (one MMA issuer).  At r = 384 that is five blocks (two on the first
+  // pseudo-tile, three on the second) where 256-column blocks made three: a
+  // job's k-block stages 24 KiB instead of 32, the second pseudo-tile's
+  // padded rows cost 128-column blocks instead of 256, and the jobs spread
+  // over more pairs, so S is written sooner (headline: by ~32 us of the call
+  // against ~40 us, the kernel 60 us against 64 us).  Several modules
+  // (`wide_gram`): 256-column blocks as two chunks of 128 (one per MMA
+  // issuer) where the slab region holds them -- a layer's nine modules would
+  // otherwise make 45 jobs of its 74 pairs, leaving the static W0 units to
+  // the other 29 (the 56-module stack took ~1680-1770 us against ~1640).
+  if (wide_gram && p.n_pad >= 2 * kGramCols) {
+    p.nc = 2 * kGramCols;
+    p.gchunks = 2;
+  } else {
+    p.nc = std::min(kGramCols, p.n_pad);
+    p.gchunks = 1;
+  }
   p.gn = p.nc / p.gchunks;
   p.gj0 = gram_jobs_of_tile(static_cast<int>(r), p.nc, 0);
   p.gblocks = p.gj0 + (p.pg_tiles > 1 ? gram_jobs_of_tile(static_cast<int>(r), p.nc, 1) : 0);
@@ -541,7 +549,7 @@ struct GroupLayout {
 bool layout_group(const int64_t* d_out, const int64_t* d_in, const int64_t* r, int count,
                   bool grouped, int workers, GroupLayout& L) {
   L.plans.resize(count);
-  for (int i = 0; i < count; ++i) plan_module(d_out[i], d_in[i], r[i], L.plans[i]);
+  for (int i = 0; i < count; ++i) plan_module(d_out[i], d_in[i], r[i], count > 1, L.plans[i]);
   long long total_w = 0;
   for (const auto& p : L.plans) {
     L.b_region = std::max(L.b_region, p.b_region);
