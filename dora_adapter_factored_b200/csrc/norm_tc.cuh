@@ -58,7 +58,10 @@ constexpr int kMaxChunksPerHalf = 8;         // 32-column TMEM chunks per epilog
 constexpr int kPrefetchChunks = 6;           // of which B is prefetched into registers (r <= 384)
 constexpr int kPartBufs = 4;                 // epilogue -> finisher hand-over buffers
 constexpr int kFinBatch = 8;                 // partial slots loaded together when finalising
-constexpr int kChunkKb = 16;                 // k-blocks per W0 chunk of the pool (at most)
+// k-blocks per W0 chunk of the pool (at most): a pool item costs a segment
+// boundary (accumulator drain, operand refill), so chunks are large; on the
+// 56-module stack 64 gave ~1530 us against ~1630 us with 16.
+constexpr int kChunkKb = 64;
 constexpr int kItemRing = 8;                 // pool items in flight between the roles of a pair
 // Roles that read each pool item: rank 0's two MMA issuers, eight epilogue
 // warps and finisher; rank 1's producer, eight epilogue warps and finisher.
