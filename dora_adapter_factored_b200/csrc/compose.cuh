@@ -28,9 +28,10 @@ namespace dora {
 // only (not on the device), so that the backward's partial layout -- and
 // therefore dm's summation order -- is the same on every run.
 constexpr int kStreamThreads = 256;
+constexpr int kStreamCtasPerSm = 2;  // resident blocks per SM the kernels are built for
 constexpr int kFwdRowUnroll = 8;
 constexpr int kBwdRowUnroll = 4;
-constexpr int kStreamSlots = 148 * 2;
+constexpr int kStreamSlots = 148 * kStreamCtasPerSm;
 
 // Backward variants: what the pass reads besides dy, and whether dm is formed.
 enum BwdMode : int {
@@ -319,7 +320,7 @@ __device__ __forceinline__ void colsum_column(const float* __restrict__ partial,
 // Idx is the element-offset type: 32-bit when T * d_out < 2^31 (fewer live
 // registers per in-flight row), 64-bit otherwise.
 template <typename T, int VEC, typename Idx, int kOut>
-__global__ void __launch_bounds__(kStreamThreads, 2)
+__global__ void __launch_bounds__(kStreamThreads, kStreamCtasPerSm)
     compose_fwd_kernel(const T* __restrict__ base, const T* __restrict__ lora,
                        const float* __restrict__ m, const float* __restrict__ n, float s,
                        float eps, long long T_rows, int d_out, T* y, T* inner) {
@@ -339,7 +340,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
 // partials of sum_t dy (base + s lora), or of sum_t dy inner, written to
 // partial[blockIdx.y][d_out].
 template <typename T, int VEC, typename Idx, int kMode>
-__global__ void __launch_bounds__(kStreamThreads, 2)
+__global__ void __launch_bounds__(kStreamThreads, kStreamCtasPerSm)
     compose_bwd_kernel(const T* dy, const T* __restrict__ x1, const T* __restrict__ x2,
                        const float* __restrict__ m, const float* __restrict__ n, float s,
                        float eps, long long T_rows, int d_out, T* d_base, T* __restrict__ d_lora,
@@ -419,7 +420,7 @@ __device__ __forceinline__ int compose_item_of_block(const ComposeGroup& grp, in
 }
 
 template <typename T, int VEC, typename Idx>
-__global__ void __launch_bounds__(kStreamThreads, 2)
+__global__ void __launch_bounds__(kStreamThreads, kStreamCtasPerSm)
     compose_fwd_grouped_kernel(const __grid_constant__ ComposeGroup grp) {
   grid_dependency_wait();
   grid_dependency_trigger();
@@ -444,7 +445,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
 }
 
 template <typename T, int VEC, typename Idx, int kMode>
-__global__ void __launch_bounds__(kStreamThreads, 2)
+__global__ void __launch_bounds__(kStreamThreads, kStreamCtasPerSm)
     compose_bwd_grouped_kernel(const __grid_constant__ ComposeGroup grp) {
   __shared__ float red[kStreamThreads * VEC];
   grid_dependency_wait();

@@ -151,6 +151,58 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return e;
 }
 
+// The streaming kernels (the compose passes) keep many 16-byte global loads in
+// flight per SM, and those need L1 capacity.  Without a stated preference a
+// CTA may land on an SM still split for the shared-memory-heavy norm or merge
+// kernel, with a small L1: the forward pass at [4096, 8192] then ran ~9 us
+// (30 %) slower after a norm call than after another forward pass.  So each
+// streaming kernel asks, once per device, for the smallest shared-memory
+// split that still holds the kStreamCtasPerSm CTAs per SM it is built for
+// (its static shared memory plus the per-block reserve, each) -- not simply
+// the largest L1, which gave the backward pass's 8 KB reduction buffer a
+// split with room for one CTA per SM (the [8192, 25600] backward went from
+// 347 to 446 us).  It is a hint: if the runtime refuses it, the launch goes
+// ahead without it.
+void prefer_l1(const void* kernel) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return;
+  }
+  static std::mutex mu;
+  static std::vector<std::pair<int, const void*>> done;
+  std::lock_guard<std::mutex> lk(mu);
+  const std::pair<int, const void*> key(dev, kernel);
+  if (std::find(done.begin(), done.end(), key) != done.end()) return;
+  cudaFuncAttributes fa = {};
+  int sm_smem = 0, reserve = 0;
+  if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
+          cudaSuccess ||
+      cudaDeviceGetAttribute(&reserve, cudaDevAttrReservedSharedMemoryPerBlock, dev) !=
+          cudaSuccess ||
+      sm_smem <= 0) {
+    (void)cudaGetLastError();
+    return;
+  }
+  const long long need = static_cast<long long>(kStreamCtasPerSm) *
+                         (static_cast<long long>(fa.sharedSizeBytes) + reserve);
+  const int percent =
+      static_cast<int>(std::min<long long>(100, (100 * need + sm_smem - 1) / sm_smem));
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, percent) ==
+      cudaSuccess)
+    done.push_back(key);
+  else
+    (void)cudaGetLastError();
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_stream(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t st, Args&&... args) {
+  prefer_l1(reinterpret_cast<const void*>(kernel));
+  return launch_pdl(kernel, grid, block, smem, st, std::forward<Args>(args)...);
+}
+
 dora_status_t launch_status() {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   const cudaError_t e = cudaGetLastError();
@@ -882,11 +934,11 @@ void launch_fwd(bool small, int64_t rows, int64_t d_out, const void* base, const
   auto go = [&](auto out) {
     constexpr int kOut = decltype(out)::value;
     if (small)
-      launch_pdl(compose_fwd_kernel<E, VEC, uint32_t, kOut>, grid, block, 0, cs, b, l, m, n, s,
-                 eps, R, D, yo, io);
+      launch_stream(compose_fwd_kernel<E, VEC, uint32_t, kOut>, grid, block, 0, cs, b, l, m, n,
+                    s, eps, R, D, yo, io);
     else
-      launch_pdl(compose_fwd_kernel<E, VEC, uint64_t, kOut>, grid, block, 0, cs, b, l, m, n, s,
-                 eps, R, D, yo, io);
+      launch_stream(compose_fwd_kernel<E, VEC, uint64_t, kOut>, grid, block, 0, cs, b, l, m, n,
+                    s, eps, R, D, yo, io);
   };
   if (delta)
     go(std::integral_constant<int, kFwdDelta>());
@@ -909,11 +961,11 @@ void launch_bwd(bool small, const StreamGrid& g, int64_t rows, int64_t d_out, co
   const long long R = rows;
   const int D = static_cast<int>(d_out);
   if (small)
-    launch_pdl(compose_bwd_kernel<E, VEC, uint32_t, kMode>, grid, block, 0, cs, d, a1, a2, m, n,
-               s, eps, R, D, ob, ol, partial);
+    launch_stream(compose_bwd_kernel<E, VEC, uint32_t, kMode>, grid, block, 0, cs, d, a1, a2,
+                  m, n, s, eps, R, D, ob, ol, partial);
   else
-    launch_pdl(compose_bwd_kernel<E, VEC, uint64_t, kMode>, grid, block, 0, cs, d, a1, a2, m, n,
-               s, eps, R, D, ob, ol, partial);
+    launch_stream(compose_bwd_kernel<E, VEC, uint64_t, kMode>, grid, block, 0, cs, d, a1, a2,
+                  m, n, s, eps, R, D, ob, ol, partial);
 }
 
 template <int kMode>
@@ -1687,21 +1739,21 @@ int compose_group_vec(const dora_compose_problem_t* pr, int count, dora_dtype_t 
 template <typename E, int VEC>
 void launch_fwd_grouped(const ComposePlan& P, cudaStream_t cs) {
   if (P.small)
-    launch_pdl(compose_fwd_grouped_kernel<E, VEC, uint32_t>, dim3(P.blocks), dim3(kStreamThreads),
-               0, cs, P.grp);
+    launch_stream(compose_fwd_grouped_kernel<E, VEC, uint32_t>, dim3(P.blocks),
+                  dim3(kStreamThreads), 0, cs, P.grp);
   else
-    launch_pdl(compose_fwd_grouped_kernel<E, VEC, uint64_t>, dim3(P.blocks), dim3(kStreamThreads),
-               0, cs, P.grp);
+    launch_stream(compose_fwd_grouped_kernel<E, VEC, uint64_t>, dim3(P.blocks),
+                  dim3(kStreamThreads), 0, cs, P.grp);
 }
 
 template <typename E, int VEC, int kMode>
 void launch_bwd_grouped(const ComposePlan& P, cudaStream_t cs) {
   if (P.small)
-    launch_pdl(compose_bwd_grouped_kernel<E, VEC, uint32_t, kMode>, dim3(P.blocks),
-               dim3(kStreamThreads), 0, cs, P.grp);
+    launch_stream(compose_bwd_grouped_kernel<E, VEC, uint32_t, kMode>, dim3(P.blocks),
+                  dim3(kStreamThreads), 0, cs, P.grp);
   else
-    launch_pdl(compose_bwd_grouped_kernel<E, VEC, uint64_t, kMode>, dim3(P.blocks),
-               dim3(kStreamThreads), 0, cs, P.grp);
+    launch_stream(compose_bwd_grouped_kernel<E, VEC, uint64_t, kMode>, dim3(P.blocks),
+                  dim3(kStreamThreads), 0, cs, P.grp);
 }
 
 template <int kMode>
