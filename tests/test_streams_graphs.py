@@ -1,5 +1,9 @@
 """The C ABI on a non-default stream and captured in a CUDA graph gives the
 same bits as on the default stream (all reductions have a fixed order)."""
+import os
+import subprocess
+import sys
+
 import pytest
 import torch
 
@@ -63,3 +67,46 @@ def test_side_stream_and_graph_match_default_stream():
     for k in ("n", "g", "y", "db", "dl", "dm"):
         assert torch.equal(ref[k], side[k]), k
         assert torch.equal(ref[k], gr[k]), k
+
+
+# A fresh process whose first compose launches happen inside a stream capture:
+# the one-time per-kernel setup of the streaming kernels (their L1/shared
+# split preference) then runs during the capture, which must neither break
+# the capture nor change a bit of the results.
+_FIRST_CALL_IN_CAPTURE = r"""
+import sys
+sys.path.insert(0, sys.argv[1])
+import torch
+import dora_adapter_factored_b200 as dora
+g = torch.Generator().manual_seed(5)
+T, d = 300, 640
+base, lora, dy = (torch.randn(T, d, generator=g).bfloat16().cuda() for _ in range(3))
+m = (1 + 0.01 * torch.randn(d, generator=g)).cuda()
+n = (1 + 0.05 * torch.rand(d, generator=g)).cuda()
+y, db, dl = (torch.empty_like(base) for _ in range(3))
+dm = torch.empty(d, device="cuda")
+wsb = torch.empty(max(256, dora.dora_compose_bwd_workspace_size(T, d, torch.bfloat16)),
+                  dtype=torch.uint8, device="cuda")
+assert dora.dora_launch_count() == 0
+graph = torch.cuda.CUDAGraph()
+with torch.cuda.graph(graph):
+    dora.dora_compose_fwd(base, lora, m, n, 2.0, 2.0 ** -7, y=y)
+    dora.dora_compose_bwd(dy, base, lora, m, n, 2.0, 2.0 ** -7, d_base=db, d_lora=dl, dm=dm,
+                          ws=wsb)
+graph.replay()
+torch.cuda.synchronize()
+y2 = dora.dora_compose_fwd(base, lora, m, n, 2.0, 2.0 ** -7)
+db2, dl2, dm2 = dora.dora_compose_bwd(dy, base, lora, m, n, 2.0, 2.0 ** -7)
+torch.cuda.synchronize()
+assert dora.dora_get_device_status() == 0
+for name, a, b in (("y", y, y2), ("d_base", db, db2), ("d_lora", dl, dl2), ("dm", dm, dm2)):
+    assert torch.equal(a, b), name
+print("OK")
+"""
+
+
+def test_first_compose_calls_inside_a_capture():
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = subprocess.run([sys.executable, "-c", _FIRST_CALL_IN_CAPTURE, root],
+                         capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0 and "OK" in res.stdout, res.stdout + res.stderr
